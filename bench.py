@@ -1,0 +1,450 @@
+"""Benchmark of split-value-cache decode attention (and the prefill chunk).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lrkv|reference] [--workload NAME]
+
+Default workload: the Qwen2.5-Coder-1.5B-shaped decode (28 layers, 12 query /
+2 KV heads, d = 128, three roles in BaseShared mode at r = 16, 32 sessions,
+8192 shared tokens, offsets 6000 / 7000 / 7800).  One step = one decode query
+per (session, agent) through the attention of all 28 layers (28 launches of
+the decode kernel, captured once in a CUDA graph and replayed).  Inputs are
+synthetic (seeded N(0, 1) draws of the model's shapes) and resident in HBM;
+each layer has its own buffers, so a step streams 7.5 GB (> L2) and no L2
+flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  Under torchrun each rank runs the same
+workload on its own data (weak scaling, no collective on the data path); the
+step time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on
+a bounded sample of the same workload (the one other place this script runs
+the oracle besides the cpu_baseline leg).
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from workloads import CONFIGS, make_decode_inputs, make_prefill_inputs  # noqa: E402
+
+METRIC = "LoRA-split KV attention: decode queries/s, HBM GB/s vs ~8 TB/s peak"
+UNIT = "queries/s"
+BF16 = 2
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+
+def decode_layer_bytes(cfg, offsets_cpu):
+    """Bytes one decode launch must move: K and V once for all agents, the U rows
+    at or past each offset (once per U cache; shared by the KV heads), q, out, B,
+    and the page table."""
+    S, N, Hq, Hkv, d, r, L = cfg.S, cfg.N, cfg.Hq, cfg.Hkv, cfg.d, cfg.r, cfg.L
+    kv = 2 * S * Hkv * L * d * BF16
+    offs = np.clip(offsets_cpu.numpy().astype(np.int64), 0, L)
+    if cfg.mode == 0:
+        u_rows = int(np.sum(L - offs))
+    else:
+        u_rows = int(np.sum(L - offs.min(axis=1)))
+    u = u_rows * r * BF16
+    qo = 2 * S * N * Hq * d * BF16
+    b = N * r * Hkv * d * BF16
+    pt = S * math.ceil(L / cfg.page_size) * 4 if cfg.paged else 0
+    return kv + u + qo + b + pt
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.out = []
+        self.dev = device_index
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50"] + sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = [ln.split(",") for ln in out.strip().splitlines() if ln.count(",") >= 8]
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                for i, nm in enumerate(names):
+                    if r[5 + i].strip().lower() == "active":
+                        reasons.add(nm)
+            except ValueError:
+                continue
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# decode workload on the GPU
+# ---------------------------------------------------------------------------
+
+class DecodeRunner:
+    def __init__(self, cfg, device, seed_offset=0):
+        import lora_shared_kv_b200 as lrkv
+        self.lrkv = lrkv
+        self.cfg = cfg
+        self.dev = device
+        from workloads.gen import seed_for
+        self.inp = make_decode_inputs(cfg, device=device, seed=seed_for(cfg) + seed_offset)
+        c = cfg
+        self.prob = lrkv.make_problem(c.S, c.N, c.Hq, c.Hkv, c.d, c.r, c.mode)
+        nws = lrkv.lrkv_decode_workspace_bytes(self.prob, c.L)
+        self.ws = torch.zeros(nws, dtype=torch.uint8, device=device)
+        self.outs = [torch.empty((c.S, c.N, c.Hq, c.d), dtype=torch.bfloat16, device=device) for _ in self.inp.layers]
+        self.kvs = []
+        self.uvs = []
+        for lay in self.inp.layers:
+            if c.paged:
+                self.kvs.append(lrkv.kv_view_paged(lay.k, lay.v, lay.page_table))
+            else:
+                self.kvs.append(lrkv.kv_view_dense(lay.k, lay.v))
+            self.uvs.append(lrkv.u_view(lay.u))
+        self.graph = None
+
+    def step_eager(self, qs=None, outs=None, stream=None):
+        lrkv, c, inp = self.lrkv, self.cfg, self.inp
+        for li, lay in enumerate(inp.layers):
+            q = lay.q if qs is None else qs[li]
+            out = self.outs[li] if outs is None else outs[li]
+            lrkv.lrkv_attn_decode(self.prob, q, self.kvs[li], inp.seq_lens, c.L, self.uvs[li], lay.b, inp.offsets,
+                                  out, self.ws, stream=stream)
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.step_eager()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step_eager()
+        torch.cuda.synchronize()
+
+    def step(self):
+        self.graph.replay()
+
+    @property
+    def launches_per_step(self):
+        return len(self.inp.layers)
+
+    def layer_bytes(self):
+        return decode_layer_bytes(self.cfg, self.inp.offsets.cpu())
+
+
+def _timed(fn, steps, warmup, sync_all):
+    for _ in range(warmup):
+        fn()
+    sync_all()
+    st = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    e1.synchronize()
+    sync_all()
+    return e0.elapsed_time(e1)
+
+
+def cpu_baseline_decode(runner, max_seconds=20.0):
+    """fp64 oracle on the host cores: sessions x all layers until about max_seconds."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    cfg, inp = runner.cfg, runner.inp
+    cores = len(os.sched_getaffinity(0))
+    blas_threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    host = []
+    for lay in inp.layers:
+        if cfg.paged:
+            host.append(None)
+        else:
+            host.append((lay.q[:1].cpu(), lay.k[:1].cpu(), lay.v[:1].cpu(), lay.u[:1].cpu(), lay.b.cpu()))
+    offs = inp.offsets[:1].cpu()
+    sl = inp.seq_lens[:1].cpu()
+    t0 = time.perf_counter()
+    done_layers = 0
+    for li in range(len(inp.layers)):
+        q, k, v, u, b = host[li]
+        oracle.decode(q, k, v, u, b, offs, sl, cfg.mode)
+        done_layers += 1
+        if time.perf_counter() - t0 > max_seconds:
+            break
+    dt = time.perf_counter() - t0
+    queries = cfg.N * done_layers / len(inp.layers)
+    return {"value": queries / dt, "unit": UNIT, "cores": min(cores, blas_threads) if blas_threads else cores,
+            "kind": "oracle",
+            "sample": f"session 0 ({cfg.N} queries) x {done_layers} of {len(inp.layers)} layers, fp64 numpy, "
+                      f"{dt:.1f} s; {cores} cores visible, BLAS threads {blas_threads}"}
+
+
+def run_e2e(runner, steps, warmup, sync_all):
+    """Public API with host buffers: per step copy every layer's q from pinned host
+    memory, run the 28 decode calls, copy every layer's output back."""
+    c = runner.cfg
+    nl = len(runner.inp.layers)
+    q_host = torch.stack([lay.q for lay in runner.inp.layers]).cpu().pin_memory()
+    out_host = torch.empty((nl, c.S, c.N, c.Hq, c.d), dtype=torch.bfloat16).pin_memory()
+    q_dev = torch.empty_like(q_host, device=runner.dev)
+    out_dev = torch.empty_like(out_host, device=runner.dev)
+
+    def step():
+        q_dev.copy_(q_host, non_blocking=True)
+        runner.step_eager(qs=q_dev, outs=out_dev)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    ms = _timed(step, steps, warmup, sync_all)
+    return ms / steps, q_host.numel() * 2, out_host.numel() * 2
+
+
+def bench_prefill(device, steps=20, warmup=5):
+    """Prefill chunk workload: append the chunk's U rows, then the causal chunk
+    attention for 4 agents (one layer).  Returns a dict, or None if unavailable."""
+    import lora_shared_kv_b200 as lrkv
+    cfg = CONFIGS["cfg4"]
+    inp = make_prefill_inputs(cfg, device=device)
+    prob = lrkv.make_problem(1, cfg.N, cfg.Hq, cfg.Hkv, cfg.d, cfg.r, cfg.mode)
+    kv = lrkv.kv_view_dense(inp.k, inp.v)
+    uv = lrkv.u_view(inp.u)
+    nws = lrkv.lrkv_prefill_workspace_bytes(prob, cfg.L0, cfg.T)
+    ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=device)
+    out = torch.empty((cfg.N, cfg.T, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=device)
+
+    def step():
+        lrkv.lrkv_append_lr_cache(inp.x, inp.a_down, inp.u, session=0, start_row=cfg.L0, uview=uv)
+        lrkv.lrkv_attn_prefill_chunk(prob, inp.q, kv, 0, cfg.L0, cfg.T, uv, inp.b, inp.offsets, out, ws)
+
+    try:
+        step()
+    except Exception as e:  # noqa: BLE001
+        return {"status": f"unavailable: {e}"}
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    times = []
+    for i in range(warmup + steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    keys = cfg.T * cfg.L0 + cfg.T * (cfg.T + 1) // 2
+    rows = cfg.N * cfg.Hq
+    flops = 2.0 * rows * keys * cfg.d * 2 + 2.0 * rows * keys * cfg.r + 2.0 * rows * cfg.T * cfg.r * cfg.d
+    flops += 2.0 * cfg.N * cfg.T * cfg.Dm * cfg.r
+    _, bf16_peak, _, src = _peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": cfg.name, "ms_per_step": ms, "tflops": tf, "flops_per_step": flops,
+            "peak_tflops": bf16_peak, "frac": tf / bf16_peak, "peak_source": src,
+            "l2": "256 MB flush before each step"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="lrkv", choices=["lrkv", "reference"])
+    ap.add_argument("--workload", default="cfg2", choices=[k for k in CONFIGS if k != "cfg4"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the layer count (small profiling cases only; not a bench line)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = CONFIGS[args.workload]
+    if args.layers is not None:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, layers=args.layers)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        return run_reference(cfg, args, world)
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+        def sync_all():
+            torch.cuda.synchronize()
+            dist.barrier()
+    else:
+        def sync_all():
+            torch.cuda.synchronize()
+
+    runner = DecodeRunner(cfg, dev, seed_offset=7919 * rank)
+    runner.capture()
+    clocks = ClockSampler(local)
+    clocks.start()
+    sync_all()
+    ms = _timed(runner.step, args.steps, args.warmup, sync_all)
+    ck = clocks.stop()
+    ms_step = ms / args.steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    queries = cfg.queries_per_step * world
+    value = queries / (ms_step * 1e-3)
+
+    hbm, _, _, peak_src = _peaks()
+    lb = runner.layer_bytes()
+    per_launch_ms = ms_step / runner.launches_per_step
+    achieved = lb / (per_launch_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+            "kernel": "decode_kernel", "algorithmic_bytes_per_launch": lb,
+            "launch_ms": per_launch_ms, "launch_ms_note": "step time / launches per step (gaps included)"}
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, hb, db = run_e2e(runner, max(10, args.steps // 10), args.warmup, sync_all)
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": queries / (e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
+               "ms_per_step": e_ms}
+
+    prefill = None
+    if not args.no_prefill and rank == 0:
+        prefill = bench_prefill(dev)
+
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        cpu = cpu_baseline_decode(runner)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) draws of the model shapes)",
+            "config": {"workload": cfg.name, "layers": cfg.layers, "sessions": cfg.S, "agents": cfg.N,
+                       "q_heads": cfg.Hq, "kv_heads": cfg.Hkv, "head_dim": cfg.d, "rank": cfg.r,
+                       "context": cfg.L, "mode": "BaseShared" if cfg.mode == 0 else "BaseLRShared",
+                       "paged": cfg.paged, "queries_per_step": cfg.queries_per_step,
+                       "parallelism": f"replicas x{world} (sessions sharded, no collective)",
+                       "l2": f"inputs larger than L2: {lb * runner.launches_per_step / 1e9:.2f} GB streamed per step"},
+            "hbm_gbs": achieved,
+            "roofline": roof,
+            "e2e": e2e,
+            "gpu_launches": runner.launches_per_step * args.steps,
+            "clocks": ck,
+            "cpu_baseline": cpu,
+            "prefill": prefill,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        del runner
+        dist.destroy_process_group()
+
+
+def run_reference(cfg, args, world):
+    """The oracle as it stands, timed on the host cores, one bounded sample per step."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    from workloads.gen import make_decode_layer, _draw_offsets, seed_for
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed_for(cfg))
+    offsets = _draw_offsets(cfg, gen, "cpu")
+    import dataclasses
+    small = dataclasses.replace(cfg, S=1)
+    lay = make_decode_layer(small, gen, "cpu", offsets[:1])
+    sl = torch.full((1,), cfg.L, dtype=torch.int32)
+
+    def step():
+        oracle.decode(lay.q, lay.k, lay.v, lay.u, lay.b, offsets[:1], sl, cfg.mode, page_table=lay.page_table)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    queries = cfg.N / cfg.layers          # one session, one layer of the 28
+    value = queries / dt
+    cores = len(os.sched_getaffinity(0))
+    blas = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) draws of the model shapes)",
+        "config": {"workload": cfg.name, "layers": cfg.layers, "sessions": cfg.S, "agents": cfg.N,
+                   "context": cfg.L, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(cores, blas), "kind": "oracle",
+                         "sample": f"one session, one layer of {cfg.layers} per step ({cfg.N} agents), fp64 numpy"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,239 @@
+/*
+ * lrkv.h - C ABI of the split-value-cache attention library (liblrkv.so).
+ *
+ * Several LoRA role adapters ("agents") attend over ONE shared base K/V cache.
+ * The value projection of agent i splits exactly as
+ *     V_i = X W0 + (X A_i) B_i
+ * ("LRAgent: Efficient KV Cache Sharing for Multi-LoRA LLM Agents", Pith
+ * review, "What carries the argument", Eq. 3), so the base cache X W0 is stored
+ * once and each agent keeps only the rank-r cache U_i = X A_i.  Attention is
+ * computed in the reordered form of Eq. 12 of the same page,
+ *     O_h = P_h V_base,g + (P_h Umask_i) B_i,g,   P_h = softmax(q_h K_base,g^T * scale),
+ * without ever forming an L x d_out adapter cache.  Keys carry no adapter term
+ * (same page: key caches are shared, Fig. 7).  Umask_i is U_i with the rows
+ * before the agent's aLoRA activation offset a_i removed ("RoleKV", Devpost,
+ * "What it does": the adapter switches on only after the role header; the
+ * offsets are passed explicitly, "Challenges we ran into").
+ *
+ * Notation: S sessions, N agents, Hq query heads, Hkv KV heads, G = Hq / Hkv,
+ * d head_dim, r rank.  Query head h of agent i reads KV head g = h / G and the
+ * column slice B_i[:, g*d : (g+1)*d].  U_i is one [rows, r] cache per
+ * (session, agent) shared by every KV head.  Sharing modes (LRAgent page,
+ * Fig. 2-3): LRKV_BASE_SHARED keeps one U_i per agent; LRKV_BASE_LR_SHARED
+ * (one shared down-projection A) keeps ONE U for all agents, still masked by
+ * each agent's own offset.
+ *
+ * Conventions of every entry point:
+ *  - Ownership: the caller owns every buffer.  The library allocates and frees
+ *    nothing, and never copies device memory to the host (the one exception is
+ *    lrkv_query_device_status, which exists to do exactly that).
+ *  - Pointers documented as "device" must be device (or managed) memory of the
+ *    current device.  Tensors are bf16 unless stated.  Base addresses of q, K,
+ *    V, U, B and out must be 16-byte aligned, and the token/head/session/page
+ *    strides of K, V and U must be multiples of 8 elements (16 bytes): the
+ *    tiles are moved by the Tensor Memory Accelerator.
+ *  - Streams: every launch goes on the caller's stream (a cudaStream_t; 0 is
+ *    the legacy default stream).  No call synchronises, except
+ *    lrkv_query_device_status.
+ *  - Errors: every call returns an lrkv_status and never throws.  Host-side
+ *    argument errors return before anything is launched.  Device-side checks
+ *    (a seq_len beyond max_seq_len, a negative offset, a page id out of range,
+ *    a bounded wait that gave up) never fault: they record a flag in the
+ *    workspace and are read back with lrkv_query_device_status.
+ *    lrkv_last_error_detail() gives a thread-local text for the last failure.
+ *  - Supported: head_dim in {64, 128}; rank in {8, 16, 32}; Hq a multiple of
+ *    Hkv; page_size 64; at most 16 agents per call.  Anything else returns
+ *    LRKV_ERR_UNSUPPORTED.
+ */
+#ifndef LRKV_H
+#define LRKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* lrkv_stream_t;
+
+typedef enum {
+  LRKV_OK = 0,
+  LRKV_ERR_INVALID_ARGUMENT = 1,   /* null pointer, bad size, inconsistent view        */
+  LRKV_ERR_UNSUPPORTED = 2,        /* head_dim / rank / page size / GPU not supported  */
+  LRKV_ERR_MISALIGNED = 3,         /* base address or stride not 16-byte aligned       */
+  LRKV_ERR_WORKSPACE_TOO_SMALL = 4,
+  LRKV_ERR_CUDA = 5,               /* a CUDA runtime or driver call failed             */
+  LRKV_ERR_DEVICE_FAULT = 6,       /* a device-side check flagged bad data             */
+  LRKV_ERR_TIMEOUT = 7             /* a bounded wait inside a kernel gave up           */
+} lrkv_status;
+
+typedef enum { LRKV_BASE_SHARED = 0, LRKV_BASE_LR_SHARED = 1 } lrkv_mode;
+typedef enum { LRKV_BF16 = 0, LRKV_F32 = 1 } lrkv_dtype;
+
+/* Problem shape shared by the attention calls. */
+typedef struct {
+  int32_t num_sessions;   /* S  (decode: sessions in the batch; prefill: sessions the views index) */
+  int32_t num_agents;     /* N                                                                     */
+  int32_t num_q_heads;    /* Hq                                                                    */
+  int32_t num_kv_heads;   /* Hkv, Hq % Hkv == 0                                                    */
+  int32_t head_dim;       /* d in {64, 128}                                                        */
+  int32_t rank;           /* r in {8, 16, 32}                                                      */
+  int32_t mode;           /* lrkv_mode                                                             */
+  float softmax_scale;    /* 0 => 1/sqrt(head_dim); LoRA's alpha/r is folded into B by the caller  */
+} lrkv_problem;
+
+/*
+ * The shared base K/V cache (bf16, head_dim contiguous).  K and V use the same
+ * layout and strides (in elements).
+ *  Dense  (page_table == NULL): element (s, g, t, e) at s*stride_session +
+ *         g*stride_head + t*stride_token + e.  Each (s, g) holds at least the
+ *         call's max_seq_len (decode) or ctx_len+T (prefill) token rows.
+ *  Paged  (page_table != NULL): physical page p holds page_size tokens of every
+ *         KV head: element (p, g, j, e) at p*stride_page + g*stride_head +
+ *         j*stride_token + e.  Logical token t of session s lives in page
+ *         page_table[s*page_table_stride + t/page_size], slot t % page_size
+ *         (a paged cache is the route to physical sharing named in "Shared-Prefix
+ *         KV Reuse Across Standard LoRA Adapters", section 3.2).  page_table is
+ *         device int32; num_pages bounds every id (an id outside [0, num_pages)
+ *         is skipped and flagged on the device).
+ */
+typedef struct {
+  const void* k;
+  const void* v;
+  int64_t stride_session;
+  int64_t stride_head;
+  int64_t stride_token;
+  const int32_t* page_table;
+  int64_t page_table_stride;
+  int64_t stride_page;
+  int32_t page_size;
+  int32_t num_pages;
+} lrkv_kv_view;
+
+/*
+ * Low-rank caches U (bf16, rank contiguous).  Row t of agent slot i of
+ * session s at u + s*stride_session + i*stride_agent + t*stride_token.
+ * Agent slots: N in BaseShared, 1 in BaseLRShared.  num_rows is the row
+ * capacity of each (session, agent) cache.  Rows before an agent's offset and
+ * rows at or past seq_len are never read into the result (they may hold
+ * anything, NaN included).
+ */
+typedef struct {
+  void* u;
+  int64_t stride_session;
+  int64_t stride_agent;
+  int64_t stride_token;
+  int32_t num_rows;
+} lrkv_u_view;
+
+/* ---------------------------------------------------------------------- */
+/* Low-rank cache append.                                                  */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * U_i[start_row + t, :] = X[t, :] A_i  for t in [0, T) and every agent slot
+ * i in [0, n_a), in session `session` of u_dst (LRAgent page, Eq. 3: the
+ * rank-r cache X A_i; Fig. 3: it is computed for the tokens the agent has not
+ * processed yet).  In BaseLRShared pass the one shared A with n_a = 1.
+ *   x   device bf16 [T, Dm], row-major (one X shared by all agents)
+ *   a   device bf16 [n_a, Dm, r], row-major
+ * Numerics, a fixed contract: acc = +0.0f; for k = 0 .. Dm-1 in order,
+ * acc = fmaf(x[t,k], a[k,j], acc); then round to nearest even bf16.  The
+ * bf16 x bf16 product is exact in fp32, so the result is bit-determined.
+ * Errors: start_row < 0, start_row + T > u_dst->num_rows, n_a < 1, T < 0,
+ * Dm < 1 return LRKV_ERR_INVALID_ARGUMENT.  T == 0 is a no-op.
+ */
+lrkv_status lrkv_append_lr_cache(const void* x, const void* a, int32_t n_a, int32_t T,
+                                 int32_t Dm, int32_t r, const lrkv_u_view* u_dst,
+                                 int32_t session, int32_t start_row, lrkv_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Decode: one query token per (session, agent) over the shared cache.     */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Bytes of workspace lrkv_attn_decode needs for this shape and host-side
+ * bound max_seq_len on the current device; 0 if the shape is invalid.
+ */
+size_t lrkv_decode_workspace_bytes(const lrkv_problem* p, int32_t max_seq_len);
+
+/*
+ * out[s, i, h, :] = sum_{t < seq_lens[s]} P[t] (V_base,g[t] + [t >= a_{s,i}] U_i[t] B_i,g)
+ * with P = softmax(q[s,i,h] . K_base,g[t] * scale) over t < seq_lens[s].
+ * Computed as P V_base + (P Umask_i) B_i: the rank-r accumulator is kept
+ * per query row and B_i is applied once per row in the epilogue.
+ *   q              device bf16 [S, N, Hq, d] contiguous
+ *   kv             the shared base cache (dense or paged)
+ *   seq_lens       device int32 [S]; each in [0, max_seq_len]
+ *   max_seq_len    host-side bound on seq_lens (sizes the split of the work)
+ *   u              low-rank caches; u->num_rows >= max_seq_len
+ *   b              device bf16 [N, r, Hkv*d] contiguous
+ *   alora_offsets  device int32 [S, N] (a_{s,i}), or NULL for all zero
+ *   out            device [S, N, Hq, d] contiguous, bf16 or fp32 (out_dtype)
+ *   workspace      device, >= lrkv_decode_workspace_bytes(p, max_seq_len),
+ *                  16-byte aligned, zero-filled once before its first use
+ *                  (lrkv_workspace_reset); every call leaves it reusable.
+ *                  Calls that share a workspace must be ordered (same stream).
+ * A session with seq_len 0 gets a zero output.
+ */
+lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv,
+                             const int32_t* seq_lens, int32_t max_seq_len,
+                             const lrkv_u_view* u, const void* b,
+                             const int32_t* alora_offsets, void* out, int32_t out_dtype,
+                             void* workspace, size_t workspace_bytes, lrkv_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Prefill chunk: T new rows per agent, causal, over one session.          */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes of workspace lrkv_attn_prefill_chunk needs; 0 if the shape is invalid. */
+size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T);
+
+/*
+ * Row j of agent i sits at absolute position ctx_len + j and attends to keys
+ * t <= ctx_len + j of session `session` (bottom-right causal alignment):
+ * out[i, j, h, :] = sum_t P[t] (V_base,g[t] + [t >= a_i] U_i[t] B_i,g).
+ * The chunk's own base K/V must already be in the cache at rows
+ * [ctx_len, ctx_len + T), and its U rows appended (lrkv_append_lr_cache).
+ *   q              device bf16 [N, T, Hq, d] contiguous
+ *   kv, u          views as above (u->num_rows >= ctx_len + T)
+ *   b              device bf16 [N, r, Hkv*d]
+ *   alora_offsets  device int32 [N], or NULL for all zero
+ *   out            device [N, T, Hq, d] contiguous, bf16 or fp32
+ *   workspace      device, >= lrkv_prefill_workspace_bytes, zero-filled once
+ */
+lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv,
+                                    int32_t session, int32_t ctx_len, int32_t T,
+                                    const lrkv_u_view* u, const void* b,
+                                    const int32_t* alora_offsets, void* out, int32_t out_dtype,
+                                    void* workspace, size_t workspace_bytes,
+                                    lrkv_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
+/* Workspace and status.                                                   */
+/* ---------------------------------------------------------------------- */
+
+/* Zero-fill a workspace on `stream` (asynchronous). */
+lrkv_status lrkv_workspace_reset(void* workspace, size_t workspace_bytes, lrkv_stream_t stream);
+
+/*
+ * Synchronise `stream`, read the device-side flags of `workspace` and, when
+ * `clear` is non-zero, reset them.  Returns LRKV_OK, LRKV_ERR_DEVICE_FAULT
+ * (bad seq_len, offset or page id seen) or LRKV_ERR_TIMEOUT (a bounded wait
+ * gave up).  *flags_out (if not NULL) receives the raw flag bits.
+ */
+lrkv_status lrkv_query_device_status(const void* workspace, int32_t clear, uint32_t* flags_out,
+                                     lrkv_stream_t stream);
+
+const char* lrkv_status_string(lrkv_status s);
+const char* lrkv_last_error_detail(void);
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t lrkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LRKV_H */

@@ -1,0 +1,394 @@
+// C ABI of liblrkv.so: argument checks, work partition, TMA descriptors,
+// launches.  No allocation, no host<->device copies, no synchronisation
+// (except lrkv_query_device_status, whose job it is).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "lrkv_internal.h"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+lrkv_status fail(lrkv_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+lrkv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(LRKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------
+// device facts
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+  int smem_optin = 0;
+};
+
+lrkv_status device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LRKV_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!have[dev]) {
+    DeviceInfo d;
+    if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(major)");
+    if ((e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(smem)");
+    cache[dev] = d;
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  if (out->major != 10) return fail(LRKV_ERR_UNSUPPORTED, "needs an sm_100 GPU (found compute capability %d.x)", out->major);
+  return LRKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor map, dims/strides innermost first (strides in elements,
+// for dims 1..3).  A dimension of extent 1 gets a packed stride.
+lrkv_status make_map4(CUtensorMap* m, const void* base, const uint64_t dims[4], const int64_t strides_el[3],
+                      const uint32_t box[4], CUtensorMapSwizzle swz, const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(LRKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t gdim[4];
+  cuuint64_t gstr[3];
+  uint64_t packed = dims[0] * 2;
+  for (int i = 0; i < 4; ++i) gdim[i] = dims[i];
+  for (int i = 0; i < 3; ++i) {
+    uint64_t s = strides_el[i] > 0 ? (uint64_t)strides_el[i] * 2 : 0;
+    if (dims[i + 1] == 1 || s == 0) s = packed < 16 ? 16 : (packed + 15) / 16 * 16;
+    if (s % 16 != 0) return fail(LRKV_ERR_MISALIGNED, "%s: stride %d (%llu bytes) is not a multiple of 16 bytes", what, i + 1, (unsigned long long)s);
+    gstr[i] = s;
+    packed = s * dims[i + 1];
+  }
+  cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gdim, gstr, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LRKV_ERR_INVALID_ARGUMENT, "%s: cuTensorMapEncodeTiled failed (%d)", what, (int)r);
+  return LRKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// shared checks
+// ---------------------------------------------------------------------------
+lrkv_status check_problem(const lrkv_problem* p) {
+  if (!p) return fail(LRKV_ERR_INVALID_ARGUMENT, "problem is NULL");
+  if (p->num_sessions < 1 || p->num_agents < 1 || p->num_q_heads < 1 || p->num_kv_heads < 1)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "sessions, agents and heads must be >= 1");
+  if (p->num_q_heads % p->num_kv_heads != 0)
+    return fail(LRKV_ERR_UNSUPPORTED, "num_q_heads (%d) must be a multiple of num_kv_heads (%d)", p->num_q_heads, p->num_kv_heads);
+  if (p->head_dim != 64 && p->head_dim != 128) return fail(LRKV_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", p->head_dim);
+  if (p->rank != 8 && p->rank != 16 && p->rank != 32) return fail(LRKV_ERR_UNSUPPORTED, "rank %d (supported: 8, 16, 32)", p->rank);
+  if (p->mode != LRKV_BASE_SHARED && p->mode != LRKV_BASE_LR_SHARED) return fail(LRKV_ERR_INVALID_ARGUMENT, "mode %d", p->mode);
+  if (p->num_agents > lrkv::kMaxAgents) return fail(LRKV_ERR_UNSUPPORTED, "at most %d agents per call", lrkv::kMaxAgents);
+  if (!(p->softmax_scale >= 0.f) || isinf(p->softmax_scale)) return fail(LRKV_ERR_INVALID_ARGUMENT, "softmax_scale must be finite and >= 0");
+  return LRKV_OK;
+}
+
+float scale_of(const lrkv_problem* p) {
+  return p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf((float)p->head_dim);
+}
+
+lrkv_status check_kv(const lrkv_kv_view* kv, const lrkv_problem* p) {
+  if (!kv || !kv->k || !kv->v) return fail(LRKV_ERR_INVALID_ARGUMENT, "kv view or its k/v pointer is NULL");
+  if (!aligned16(kv->k) || !aligned16(kv->v)) return fail(LRKV_ERR_MISALIGNED, "k and v must be 16-byte aligned");
+  if (kv->stride_token < p->head_dim || kv->stride_head < 1) return fail(LRKV_ERR_INVALID_ARGUMENT, "kv strides too small");
+  if (kv->stride_token % 8 || kv->stride_head % 8) return fail(LRKV_ERR_MISALIGNED, "kv token/head strides must be multiples of 8 elements");
+  if (kv->page_table) {
+    if (kv->page_size != lrkv::kKeysPerTile) return fail(LRKV_ERR_UNSUPPORTED, "page_size %d (supported: 64)", kv->page_size);
+    if (kv->num_pages < 1 || kv->stride_page < 1 || kv->stride_page % 8) return fail(LRKV_ERR_INVALID_ARGUMENT, "paged view needs num_pages >= 1 and a stride_page that is a positive multiple of 8");
+    if (kv->page_table_stride < 1) return fail(LRKV_ERR_INVALID_ARGUMENT, "page_table_stride must be >= 1");
+  } else {
+    if (p->num_sessions > 1 && (kv->stride_session < 1 || kv->stride_session % 8)) return fail(LRKV_ERR_MISALIGNED, "kv session stride must be a positive multiple of 8 elements");
+  }
+  return LRKV_OK;
+}
+
+lrkv_status check_u(const lrkv_u_view* u, const lrkv_problem* p, int rows_needed) {
+  if (!u || !u->u) return fail(LRKV_ERR_INVALID_ARGUMENT, "u view or its pointer is NULL");
+  if (!aligned16(u->u)) return fail(LRKV_ERR_MISALIGNED, "u must be 16-byte aligned");
+  if (u->stride_token < p->rank || u->stride_token % 8) return fail(LRKV_ERR_MISALIGNED, "u stride_token must be >= rank and a multiple of 8");
+  const int slots = p->mode == LRKV_BASE_SHARED ? p->num_agents : 1;
+  if (slots > 1 && (u->stride_agent < 1 || u->stride_agent % 8)) return fail(LRKV_ERR_MISALIGNED, "u stride_agent must be a positive multiple of 8");
+  if (p->num_sessions > 1 && (u->stride_session < 1 || u->stride_session % 8)) return fail(LRKV_ERR_MISALIGNED, "u stride_session must be a positive multiple of 8");
+  if (u->num_rows < rows_needed) return fail(LRKV_ERR_INVALID_ARGUMENT, "u num_rows %d < %d rows needed", u->num_rows, rows_needed);
+  return LRKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// decode plan
+// ---------------------------------------------------------------------------
+struct DecodePlan {
+  int G, R, n_rg, rows_per_group, NT, n_u_slots, nt, items, ctas, max_segs, stages, smem;
+  long long W;
+  size_t tickets_off, partials_off, bytes;
+};
+
+lrkv_status plan_decode(const lrkv_problem* p, int max_seq_len, const DeviceInfo& dev, DecodePlan* pl) {
+  lrkv_status s = check_problem(p);
+  if (s != LRKV_OK) return s;
+  if (max_seq_len < 0) return fail(LRKV_ERR_INVALID_ARGUMENT, "max_seq_len must be >= 0");
+  pl->G = p->num_q_heads / p->num_kv_heads;
+  pl->R = p->num_agents * pl->G;
+  pl->n_rg = (pl->R + lrkv::kMaxRowsPerItem - 1) / lrkv::kMaxRowsPerItem;
+  pl->rows_per_group = (pl->R + pl->n_rg - 1) / pl->n_rg;
+  pl->NT = (pl->rows_per_group + 7) / 8;
+  int max_ag = 0;
+  for (int rg = 0; rg < pl->n_rg; ++rg) {
+    const int lo = rg * pl->rows_per_group;
+    const int hi = lo + pl->rows_per_group < pl->R ? lo + pl->rows_per_group : pl->R;
+    if (hi <= lo) continue;
+    const int n = (hi - 1) / pl->G - lo / pl->G + 1;
+    max_ag = n > max_ag ? n : max_ag;
+  }
+  pl->n_u_slots = p->mode == LRKV_BASE_SHARED ? max_ag : 1;
+  pl->nt = max_seq_len > 0 ? (max_seq_len + lrkv::kKeysPerTile - 1) / lrkv::kKeysPerTile : 1;
+  pl->items = p->num_sessions * p->num_kv_heads * pl->n_rg;
+  pl->W = (long long)pl->items * pl->nt;
+  const int sms = dev.sms > 0 ? dev.sms : 148;
+  pl->ctas = (int)(pl->W < sms ? pl->W : sms);
+  int ms = 1;
+  for (int it = 0; it < pl->items; ++it) {
+    const long long cf = lrkv::owner_cta((long long)it * pl->nt, pl->W, pl->ctas);
+    const long long cl = lrkv::owner_cta((long long)(it + 1) * pl->nt - 1, pl->W, pl->ctas);
+    const int n = (int)(cl - cf + 1);
+    ms = n > ms ? n : ms;
+  }
+  pl->max_segs = ms;
+  // shared memory: as many stages as fit (2..8)
+  const int optin = dev.smem_optin > 0 ? dev.smem_optin : 232448;
+  int stages = 8;
+  for (; stages >= 2; --stages) {
+    lrkv::DecodeSmem lay = lrkv::decode_smem_plan(p->head_dim, pl->NT, p->rank, pl->n_u_slots, stages);
+    if (lay.total + 1024 <= optin) break;
+  }
+  if (stages < 2) return fail(LRKV_ERR_UNSUPPORTED, "decode tiles do not fit in shared memory");
+  pl->stages = stages;
+  pl->smem = lrkv::decode_smem_plan(p->head_dim, pl->NT, p->rank, pl->n_u_slots, stages).total + 1024;
+  pl->tickets_off = lrkv::kWsHeaderBytes;
+  pl->partials_off = pl->tickets_off + ((size_t)pl->items * 4 + 255) / 256 * 256;
+  const size_t rec = lrkv::decode_record_floats(pl->NT, p->head_dim, p->rank) * 4;
+  pl->bytes = pl->partials_off + (pl->max_segs > 1 ? (size_t)pl->items * pl->max_segs * rec : 0);
+  return LRKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lrkv_status_string(lrkv_status s) {
+  switch (s) {
+    case LRKV_OK: return "ok";
+    case LRKV_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case LRKV_ERR_UNSUPPORTED: return "unsupported";
+    case LRKV_ERR_MISALIGNED: return "misaligned";
+    case LRKV_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case LRKV_ERR_CUDA: return "CUDA error";
+    case LRKV_ERR_DEVICE_FAULT: return "device-side check failed";
+    case LRKV_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* lrkv_last_error_detail(void) { return g_detail; }
+
+int32_t lrkv_version(void) { return 100; }
+
+lrkv_status lrkv_workspace_reset(void* workspace, size_t workspace_bytes, lrkv_stream_t stream) {
+  if (!workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "workspace is NULL");
+  cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  return LRKV_OK;
+}
+
+lrkv_status lrkv_query_device_status(const void* workspace, int32_t clear, uint32_t* flags_out,
+                                     lrkv_stream_t stream) {
+  if (!workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "workspace is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t flags = 0;
+  cudaError_t e = cudaMemcpyAsync(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace flags");
+  if (clear && flags) {
+    e = cudaMemsetAsync(const_cast<void*>(workspace), 0, sizeof(uint32_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace flags");
+  }
+  if (flags_out) *flags_out = flags;
+  if (flags & LRKV_DEVFLAG_TIMEOUT) return fail(LRKV_ERR_TIMEOUT, "a bounded wait inside a kernel gave up (flags 0x%x)", flags);
+  if (flags) return fail(LRKV_ERR_DEVICE_FAULT, "device-side checks flagged bad data (flags 0x%x: %s%s%s)", flags,
+                         (flags & LRKV_DEVFLAG_SEQLEN) ? "seq_len " : "", (flags & LRKV_DEVFLAG_OFFSET) ? "offset " : "",
+                         (flags & LRKV_DEVFLAG_PAGE) ? "page-id" : "");
+  return LRKV_OK;
+}
+
+lrkv_status lrkv_append_lr_cache(const void* x, const void* a, int32_t n_a, int32_t T, int32_t Dm, int32_t r,
+                                 const lrkv_u_view* u_dst, int32_t session, int32_t start_row,
+                                 lrkv_stream_t stream) {
+  if (!x || !a || !u_dst || !u_dst->u) return fail(LRKV_ERR_INVALID_ARGUMENT, "x, a and u_dst->u must not be NULL");
+  if (T < 0 || Dm < 1 || n_a < 1 || session < 0 || start_row < 0)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "need T >= 0, Dm >= 1, n_a >= 1, session >= 0, start_row >= 0");
+  if (r != 8 && r != 16 && r != 32) return fail(LRKV_ERR_UNSUPPORTED, "rank %d (supported: 8, 16, 32)", r);
+  if ((long long)start_row + T > u_dst->num_rows)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "rows [%d, %lld) exceed the U capacity %d", start_row, (long long)start_row + T, u_dst->num_rows);
+  if (u_dst->stride_token < r) return fail(LRKV_ERR_INVALID_ARGUMENT, "u stride_token < rank");
+  if (n_a > 1 && u_dst->stride_agent < 1) return fail(LRKV_ERR_INVALID_ARGUMENT, "u stride_agent must be >= 1 when n_a > 1");
+  if (session > 0 && u_dst->stride_session < 1) return fail(LRKV_ERR_INVALID_ARGUMENT, "u stride_session must be >= 1");
+  if (T == 0) return LRKV_OK;
+  DeviceInfo dev;
+  lrkv_status s = device_info(&dev);
+  if (s != LRKV_OK) return s;
+  s = lrkv::launch_append(x, a, n_a, T, Dm, r, u_dst->u, u_dst->stride_session, u_dst->stride_agent,
+                          u_dst->stride_token, session, start_row, stream);
+  if (s != LRKV_OK) return fail(s, "append launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+  return LRKV_OK;
+}
+
+size_t lrkv_decode_workspace_bytes(const lrkv_problem* p, int32_t max_seq_len) {
+  DeviceInfo dev;
+  if (device_info(&dev) != LRKV_OK) {
+    dev.sms = 148;
+    dev.smem_optin = 232448;
+  }
+  DecodePlan pl;
+  if (plan_decode(p, max_seq_len, dev, &pl) != LRKV_OK) return 0;
+  return pl.bytes;
+}
+
+lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv, const int32_t* seq_lens,
+                             int32_t max_seq_len, const lrkv_u_view* u, const void* b,
+                             const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
+                             size_t workspace_bytes, lrkv_stream_t stream) {
+  lrkv_status s = check_problem(p);
+  if (s != LRKV_OK) return s;
+  if (!q || !seq_lens || !b || !out || !workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "q, seq_lens, b, out and workspace must not be NULL");
+  if (!aligned16(q) || !aligned16(b) || !aligned16(out) || !aligned16(workspace)) return fail(LRKV_ERR_MISALIGNED, "q, b, out and workspace must be 16-byte aligned");
+  if (out_dtype != LRKV_BF16 && out_dtype != LRKV_F32) return fail(LRKV_ERR_INVALID_ARGUMENT, "out_dtype %d", out_dtype);
+  if ((s = check_kv(kv, p)) != LRKV_OK) return s;
+  if ((s = check_u(u, p, max_seq_len)) != LRKV_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(&dev)) != LRKV_OK) return s;
+  DecodePlan pl;
+  if ((s = plan_decode(p, max_seq_len, dev, &pl)) != LRKV_OK) return s;
+  if (workspace_bytes < pl.bytes) return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, pl.bytes);
+
+  const int D = p->head_dim, RK = p->rank;
+  const int Lmap = max_seq_len > 0 ? max_seq_len : 1;
+  alignas(64) CUtensorMap tmK, tmV, tmU;
+  const uint32_t kbox[4] = {64, (uint32_t)lrkv::kKeysPerTile, 1, 1};
+  if (kv->page_table) {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)kv->page_size, (uint64_t)p->num_kv_heads, (uint64_t)kv->num_pages};
+    const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_page};
+    if ((s = make_map4(&tmK, kv->k, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "K pages")) != LRKV_OK) return s;
+    if ((s = make_map4(&tmV, kv->v, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "V pages")) != LRKV_OK) return s;
+  } else {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Lmap, (uint64_t)p->num_kv_heads, (uint64_t)p->num_sessions};
+    const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_session};
+    if ((s = make_map4(&tmK, kv->k, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "K")) != LRKV_OK) return s;
+    if ((s = make_map4(&tmV, kv->v, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "V")) != LRKV_OK) return s;
+  }
+  {
+    const int slots = p->mode == LRKV_BASE_SHARED ? p->num_agents : 1;
+    const uint64_t dims[4] = {(uint64_t)RK, (uint64_t)u->num_rows, (uint64_t)slots, (uint64_t)p->num_sessions};
+    const int64_t str[3] = {u->stride_token, u->stride_agent, u->stride_session};
+    const uint32_t ubox[4] = {(uint32_t)RK, (uint32_t)lrkv::kKeysPerTile, 1, 1};
+    if ((s = make_map4(&tmU, u->u, dims, str, ubox, CU_TENSOR_MAP_SWIZZLE_NONE, "U")) != LRKV_OK) return s;
+  }
+
+  lrkv::DecodeParams dp = {};
+  dp.q = q;
+  dp.b = b;
+  dp.seq_lens = seq_lens;
+  dp.offsets = alora_offsets;
+  dp.page_table = kv->page_table;
+  dp.pt_stride = kv->page_table_stride;
+  dp.out = out;
+  dp.out_f32 = out_dtype == LRKV_F32;
+  dp.S = p->num_sessions;
+  dp.N = p->num_agents;
+  dp.Hq = p->num_q_heads;
+  dp.Hkv = p->num_kv_heads;
+  dp.G = pl.G;
+  dp.rows_total = pl.R;
+  dp.rows_per_group = pl.rows_per_group;
+  dp.n_rg = pl.n_rg;
+  dp.n_u_slots = pl.n_u_slots;
+  dp.mode = p->mode;
+  dp.max_seq_len = max_seq_len;
+  dp.u_rows = u->num_rows;
+  dp.num_pages = kv->page_table ? kv->num_pages : 0;
+  dp.paged = kv->page_table != nullptr;
+  dp.nt = pl.nt;
+  dp.items = pl.items;
+  dp.W = pl.W;
+  dp.max_segs = pl.max_segs;
+  dp.stages = pl.stages;
+  dp.scale_log2 = scale_of(p) * 1.4426950408889634f;
+  char* ws = static_cast<char*>(workspace);
+  dp.flags = reinterpret_cast<unsigned*>(ws);
+  dp.tickets = reinterpret_cast<int*>(ws + pl.tickets_off);
+  dp.partials = reinterpret_cast<float*>(ws + pl.partials_off);
+  s = lrkv::launch_decode(dp, D, pl.NT, RK, &tmK, &tmV, &tmU, pl.smem, pl.ctas, stream);
+  if (s != LRKV_OK) return fail(s, "decode launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+  return LRKV_OK;
+}
+
+size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T) {
+  (void)p;
+  (void)ctx_len;
+  (void)T;
+  return 0;
+}
+
+lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv, int32_t session,
+                                    int32_t ctx_len, int32_t T, const lrkv_u_view* u, const void* b,
+                                    const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
+                                    size_t workspace_bytes, lrkv_stream_t stream) {
+  (void)p; (void)q; (void)kv; (void)session; (void)ctx_len; (void)T; (void)u; (void)b;
+  (void)alora_offsets; (void)out; (void)out_dtype; (void)workspace; (void)workspace_bytes; (void)stream;
+  return fail(LRKV_ERR_UNSUPPORTED, "prefill chunk not built yet");
+}
+
+}  // extern "C"

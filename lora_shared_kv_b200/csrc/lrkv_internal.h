@@ -1,0 +1,98 @@
+// Internal definitions shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/lrkv.h"
+
+// Device-side flag bits, kept in the first word of every workspace.
+#define LRKV_DEVFLAG_SEQLEN 0x1u    // a seq_len outside [0, max_seq_len] or past the U capacity
+#define LRKV_DEVFLAG_OFFSET 0x2u    // a negative aLoRA offset (treated as 0)
+#define LRKV_DEVFLAG_PAGE 0x4u      // a page id outside [0, num_pages) (tile skipped)
+#define LRKV_DEVFLAG_TIMEOUT 0x8u   // a bounded wait gave up
+
+namespace lrkv {
+
+constexpr int kWsHeaderBytes = 256;     // flags word + padding at the start of a workspace
+constexpr int kKeysPerTile = 64;        // keys per K/V tile (one TMA box, one page)
+constexpr int kMaxRowsPerItem = 32;     // query rows (agents x GQA heads) per decode work item
+constexpr int kMaxAgents = 16;
+
+// ---------------------------------------------------------------------------
+// decode
+// ---------------------------------------------------------------------------
+struct DecodeParams {
+  const void* q;             // bf16 [S, N, Hq, d]
+  const void* b;             // bf16 [N, r, Hkv*d]
+  const int32_t* seq_lens;   // [S]
+  const int32_t* offsets;    // [S, N] or null
+  const int32_t* page_table; // null => dense
+  long long pt_stride;
+  void* out;
+  int out_f32;
+  int S, N, Hq, Hkv, G;
+  int rows_total;            // N * G
+  int rows_per_group;        // rows of one work item (<= 32)
+  int n_rg;                  // row groups per (session, KV head)
+  int n_u_slots;             // U tiles staged per K/V tile
+  int mode;
+  int max_seq_len;
+  int u_rows;
+  int num_pages;
+  int paged;
+  int nt;                    // key tiles per work item
+  int items;                 // S * Hkv * n_rg
+  long long W;               // items * nt (flattened tile count)
+  int max_segs;              // partial slots per item
+  int stages;
+  float scale_log2;          // softmax_scale * log2(e)
+  float* partials;
+  int* tickets;
+  unsigned* flags;
+};
+
+// Shared-memory plan of the decode kernel (bytes from a 1024-aligned base).
+struct DecodeSmem {
+  int stage_bytes, ring_bytes, q_off, merge_off, scw_off, a_off, bar_off, total;
+};
+
+__host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+__host__ __device__ inline DecodeSmem decode_smem_plan(int D, int NT, int RK, int n_u_slots, int stages) {
+  DecodeSmem s;
+  const int RP = NT * 8;
+  s.stage_bytes = round_up(2 * kKeysPerTile * D * 2 + n_u_slots * kKeysPerTile * RK * 2, 1024);
+  s.ring_bytes = stages * s.stage_bytes;
+  s.q_off = s.ring_bytes;
+  s.merge_off = s.q_off + round_up(RP * D * 2, 128);
+  const int rec = RP * (D + RK + 2) * 4;
+  s.scw_off = s.merge_off + 4 * rec;
+  s.a_off = s.scw_off + 8 * RP * 4;
+  s.bar_off = round_up(s.a_off + kMaxAgents * 4, 16);
+  s.total = s.bar_off + 2 * stages * 8 + 64;
+  return s;
+}
+
+inline size_t decode_record_floats(int NT, int D, int RK) { return (size_t)NT * 8 * (D + RK + 2); }
+
+// Owner CTA of flattened tile t when W tiles are split evenly over C CTAs:
+// CTA c covers [c*W/C, (c+1)*W/C).
+__host__ __device__ inline long long owner_cta(long long t, long long W, long long C) {
+  return ((t + 1) * C - 1) / W;
+}
+
+// ---------------------------------------------------------------------------
+// launchers (defined in the kernel translation units)
+// ---------------------------------------------------------------------------
+struct TmaMaps;  // opaque; holds CUtensorMap objects
+
+lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, const void* tmK, const void* tmV,
+                          const void* tmU, int smem_bytes, int ctas, void* stream);
+int decode_max_smem_optin();
+
+lrkv_status launch_append(const void* x, const void* a, int n_a, int T, int Dm, int r, void* u,
+                          long long u_ss, long long u_sa, long long u_st, int session, int start_row,
+                          void* stream);
+
+}  // namespace lrkv

@@ -1,0 +1,104 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+and rejects bad arguments with status codes before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import lora_shared_kv_b200 as lrkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "lrkv.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lrkv_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = lrkv.lib()
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(lrkv.EXPORTS) == names
+
+
+def test_status_strings_and_version():
+    L = lrkv.lib()
+    for s in range(8):
+        assert L.lrkv_status_string(s)
+    assert lrkv.version() >= 100
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _problem(**kw):
+    base = dict(S=2, N=3, Hq=12, Hkv=2, d=128, r=16, mode=0)
+    base.update(kw)
+    return lrkv.make_problem(base["S"], base["N"], base["Hq"], base["Hkv"], base["d"], base["r"], base["mode"])
+
+
+def _views(misaligned=False):
+    p = FAKE + (2 if misaligned else 0)
+    kv = lrkv.KVView(p, FAKE, 2 * 8192 * 128, 8192 * 128, 128, None, 0, 0, 0, 0)
+    uv = lrkv.UView(FAKE, 3 * 8192 * 16, 8192 * 16, 16, 8192)
+    return kv, uv
+
+
+def _decode(prob, kv, uv, q=FAKE, max_len=8192, ws_bytes=1 << 20):
+    L = lrkv.lib()
+    return L.lrkv_attn_decode(ctypes.byref(prob), ctypes.c_void_p(q), ctypes.byref(kv), ctypes.c_void_p(FAKE),
+                              max_len, ctypes.byref(uv), ctypes.c_void_p(FAKE), None, ctypes.c_void_p(FAKE), 0,
+                              ctypes.c_void_p(FAKE), ws_bytes, None)
+
+
+def test_decode_argument_errors():
+    kv, uv = _views()
+    assert _decode(_problem(d=96), kv, uv) == 2            # unsupported head_dim
+    assert _decode(_problem(r=12), kv, uv) == 2            # unsupported rank
+    assert _decode(_problem(Hq=10, Hkv=4), kv, uv) == 2    # Hq not a multiple of Hkv
+    assert _decode(_problem(S=0), kv, uv) == 1
+    assert _decode(_problem(mode=5), kv, uv) == 1
+    assert _decode(_problem(N=17), kv, uv) == 2            # too many agents
+    assert _decode(_problem(), kv, uv, q=0) == 1           # NULL q
+    assert _decode(_problem(), kv, uv, q=FAKE + 8) == 3    # misaligned q
+    kvm, _ = _views(misaligned=True)
+    assert _decode(_problem(), kvm, uv) == 3               # misaligned k
+    assert _decode(_problem(), kv, uv, max_len=9000) == 1  # U capacity below max_seq_len
+    L = lrkv.lib()
+    assert L.lrkv_attn_decode(None, None, None, None, 0, None, None, None, None, 0, None, 0, None) == 1
+    assert "q" in L.lrkv_last_error_detail().decode() or L.lrkv_last_error_detail()
+
+
+def test_append_argument_errors():
+    L = lrkv.lib()
+    uv = lrkv.UView(FAKE, 0, 100 * 16, 16, 100)
+    f = lambda **k: L.lrkv_append_lr_cache(ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), k.get("n_a", 1),
+                                           k.get("T", 10), k.get("Dm", 64), k.get("r", 16), ctypes.byref(uv),
+                                           0, k.get("start", 0), None)
+    assert f(T=-1) == 1
+    assert f(r=12) == 2
+    assert f(start=95) == 1          # rows past the capacity
+    assert f(n_a=0) == 1
+    assert f(T=0) == 0               # empty append is a no-op, no launch
+    assert L.lrkv_append_lr_cache(None, None, 1, 1, 1, 16, None, 0, 0, None) == 1
+
+
+def test_workspace_bytes_shape_rules():
+    # without a device the plan falls back to 148 SMs; invalid shapes give 0
+    assert lrkv.lib().lrkv_decode_workspace_bytes(ctypes.byref(_problem(d=96)), 128) == 0
+    n = lrkv.lib().lrkv_decode_workspace_bytes(ctypes.byref(_problem()), 8192)
+    assert n >= 256
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(lrkv, "_lib", None)
+    monkeypatch.setattr(lrkv, "LIB_PATH", str(tmp_path / "liblrkv.so"))
+    with pytest.raises(ImportError):
+        lrkv.lib()

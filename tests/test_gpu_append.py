@@ -1,0 +1,56 @@
+"""Low-rank cache append: the CUDA path is bit-exact against the oracle's
+fixed-order fp32 reference, and writes only the rows it is asked to."""
+
+import numpy as np
+import pytest
+import torch
+
+import lora_shared_kv_b200 as lrkv
+import oracle
+from workloads import CONFIGS, make_prefill_inputs
+from workloads.gen import _normal
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("T,Dm,r,n_a,start,cap", [
+    (1, 128, 8, 2, 0, 256),
+    (37, 1536, 16, 3, 100, 200),
+    (512, 2048, 32, 4, 16384, 16896),
+    (5, 65, 16, 1, 3, 8),
+])
+def test_append_bit_exact(T, Dm, r, n_a, start, cap):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(T * 7 + Dm)
+    x = _normal((T, Dm), 1.0, g, DEV)
+    a = _normal((n_a, Dm, r), Dm ** -0.5, g, DEV)
+    S = 2
+    u = torch.full((S, n_a, cap, r), float("nan"), dtype=torch.bfloat16, device=DEV)
+    before = u.clone()
+    lrkv.lrkv_append_lr_cache(x, a, u, session=1, start_row=start)
+    torch.cuda.synchronize()
+    want = oracle.ref_append_fp32(x.cpu(), a.cpu())              # [n_a, T, r] bits
+    got = _bits(u[1, :, start:start + T])
+    assert np.array_equal(got, want)
+    # nothing else touched
+    mask = torch.ones_like(u, dtype=torch.bool)
+    mask[1, :, start:start + T] = False
+    assert torch.equal(_nan_bits(u[mask]), _nan_bits(before[mask]))
+
+
+def _nan_bits(t):
+    return t.view(torch.int16)
+
+
+def test_append_prefill_workload_rows():
+    cfg = CONFIGS["cfg4"]
+    inp = make_prefill_inputs(cfg, device=DEV)
+    lrkv.lrkv_append_lr_cache(inp.x, inp.a_down, inp.u, session=0, start_row=cfg.L0)
+    torch.cuda.synchronize()
+    want = oracle.ref_append_fp32(inp.x.cpu(), inp.a_down.cpu())
+    assert np.array_equal(_bits(inp.u[0, :, cfg.L0:]), want)
