@@ -37,8 +37,6 @@ namespace lrkv {
 namespace {
 
 constexpr int KT = kKeysPerTile;
-constexpr int NCW = 4;                     // consumer warps
-constexpr int DEC_THREADS = (NCW + 1) * 32;
 constexpr int SEG_CHUNK = 8;               // partial records combined per pass
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -195,7 +193,98 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
 // ---------------------------------------------------------------------------
 // consumer warps
 // ---------------------------------------------------------------------------
+// NG warpgroups of four warps.  Tile n of the CTA (counted over all its
+// segments) belongs to group n % NG; warp w of a group owns keys
+// [16 w, 16 w + 16) of its tiles.  Each warp keeps its own online-softmax
+// state; the states are merged in shared memory at the end of a segment.
 template <int D, int NT, int RK>
+struct WarpState {
+  static constexpr int MT = D / 16;
+  static constexpr int MTZ = RK >= 16 ? RK / 16 : 1;
+  float m[NT][2], l[NT][2];
+  float o[MT][NT][4];
+  float z[MTZ][NT][4];
+};
+
+// Write a warp's state (l already reduced over its lanes) to a record
+// [m(RP) | l(RP) | O(RP x D) | Z(RP x RK)].
+template <int D, int NT, int RK>
+__device__ __forceinline__ void store_state(const WarpState<D, NT, RK>& st, float* mr, int g8, int t4) {
+  constexpr int RP = NT * 8;
+  float* mO = mr + 2 * RP;
+  float* mZ = mO + RP * D;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int r0 = nt * 8 + 2 * t4;
+    if (g8 == 0) {
+      mr[r0] = st.m[nt][0];
+      mr[r0 + 1] = st.m[nt][1];
+      mr[RP + r0] = st.l[nt][0];
+      mr[RP + r0 + 1] = st.l[nt][1];
+    }
+#pragma unroll
+    for (int mt = 0; mt < WarpState<D, NT, RK>::MT; ++mt) {
+      const int d0 = mt * 16 + g8;
+      mO[r0 * D + d0] = st.o[mt][nt][0];
+      mO[(r0 + 1) * D + d0] = st.o[mt][nt][1];
+      mO[r0 * D + d0 + 8] = st.o[mt][nt][2];
+      mO[(r0 + 1) * D + d0 + 8] = st.o[mt][nt][3];
+    }
+#pragma unroll
+    for (int mz = 0; mz < WarpState<D, NT, RK>::MTZ; ++mz) {
+      const int k0 = mz * 16 + g8;
+      mZ[r0 * RK + k0] = st.z[mz][nt][0];
+      mZ[(r0 + 1) * RK + k0] = st.z[mz][nt][1];
+      if (k0 + 8 < RK) {
+        mZ[r0 * RK + k0 + 8] = st.z[mz][nt][2];
+        mZ[(r0 + 1) * RK + k0 + 8] = st.z[mz][nt][3];
+      }
+    }
+  }
+}
+
+// st <- merge(st, record): the online-softmax combination of two partial states.
+template <int D, int NT, int RK>
+__device__ __forceinline__ void absorb_state(WarpState<D, NT, RK>& st, const float* mr, int g8, int t4) {
+  constexpr int RP = NT * 8;
+  const float* mO = mr + 2 * RP;
+  const float* mZ = mO + RP * D;
+  const float NEG_INF = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int r0 = nt * 8 + 2 * t4;
+    float sa[2], so[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float mo = mr[r0 + e];
+      const float M = fmaxf(st.m[nt][e], mo);
+      sa[e] = st.m[nt][e] == NEG_INF ? 0.f : fast_exp2(st.m[nt][e] - M);
+      so[e] = mo == NEG_INF ? 0.f : fast_exp2(mo - M);
+      st.l[nt][e] = st.l[nt][e] * sa[e] + mr[RP + r0 + e] * so[e];
+      st.m[nt][e] = M;
+    }
+#pragma unroll
+    for (int mt = 0; mt < WarpState<D, NT, RK>::MT; ++mt) {
+      const int d0 = mt * 16 + g8;
+      st.o[mt][nt][0] = st.o[mt][nt][0] * sa[0] + mO[r0 * D + d0] * so[0];
+      st.o[mt][nt][1] = st.o[mt][nt][1] * sa[1] + mO[(r0 + 1) * D + d0] * so[1];
+      st.o[mt][nt][2] = st.o[mt][nt][2] * sa[0] + mO[r0 * D + d0 + 8] * so[0];
+      st.o[mt][nt][3] = st.o[mt][nt][3] * sa[1] + mO[(r0 + 1) * D + d0 + 8] * so[1];
+    }
+#pragma unroll
+    for (int mz = 0; mz < WarpState<D, NT, RK>::MTZ; ++mz) {
+      const int k0 = mz * 16 + g8;
+      st.z[mz][nt][0] = st.z[mz][nt][0] * sa[0] + mZ[r0 * RK + k0] * so[0];
+      st.z[mz][nt][1] = st.z[mz][nt][1] * sa[1] + mZ[(r0 + 1) * RK + k0] * so[1];
+      if (k0 + 8 < RK) {
+        st.z[mz][nt][2] = st.z[mz][nt][2] * sa[0] + mZ[r0 * RK + k0 + 8] * so[0];
+        st.z[mz][nt][3] = st.z[mz][nt][3] * sa[1] + mZ[(r0 + 1) * RK + k0 + 8] * so[1];
+      }
+    }
+  }
+}
+
+template <int D, int NT, int RK, int NG>
 __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const DecodeSmem& lay, uint64_t* full,
                                  uint64_t* empty, volatile int* abort_flag, int* bcast, long long t_begin,
                                  long long t_end) {
@@ -206,8 +295,13 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   constexpr int KV_BYTES = KT * D * 2;
   constexpr int U_BYTES = KT * RK * 2;
   constexpr int REC = RP * (D + RK + 2);
-  const int tid = threadIdx.x;  // 0..127
+  constexpr int CT = NG * 4 * 32;  // consumer threads
+  const int tid = threadIdx.x - 128;  // 0 .. CT-1 (warpgroup 0 is the producer)
   const int warp = tid >> 5, lane = tid & 31;
+  constexpr int NOG = NG * 2;      // owner groups: pairs of warps, tile n goes to pair n % NOG
+  static_assert(NOG == (NT <= 3 ? 2 : 1) * 2, "owner groups must match decode_owner_groups()");
+  const int og = warp >> 1;        // owner group of this warp
+  const int kh = warp & 1;         // key half (32 of the 64 keys of a tile) of this warp
   const int g8 = lane >> 2, t4 = lane & 3;
   const uint32_t ring_s = smem_u32(smem);
   const uint32_t q_s = smem_u32(smem + lay.q_off);
@@ -220,6 +314,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
 
   int stage = 0;
   uint32_t phase = 0;
+  int ntile = 0;  // tiles seen by this CTA so far (all groups)
 
   for (long long t = t_begin; t < t_end;) {
     Seg sg = make_seg(p, t, t_end, tid == 0);
@@ -231,7 +326,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     // ---- stage this item's queries (rows x d, 16B chunks, XOR-swizzled) and offsets
     {
       constexpr int CH = D / 8;
-      for (int idx = tid; idx < RP * CH; idx += NCW * 32) {
+      for (int idx = tid; idx < RP * CH; idx += CT) {
         const int row = idx / CH, ch = idx % CH;
         uint4 val = make_uint4(0, 0, 0, 0);
         if (row < sg.rows) {
@@ -246,7 +341,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
         *reinterpret_cast<uint4*>(smem + lay.q_off + row * (D * 2) + pch * 16) = val;
       }
       if (tid < sg.n_ag) a_sm[tid] = load_offset(p, sg.s, sg.i_lo + tid, true);
-      named_bar_sync(1, NCW * 32);
+      named_bar_sync(1, CT);
     }
     int a_max = 0;
     for (int j = 0; j < sg.n_ag; ++j) a_max = max(a_max, a_sm[j]);
@@ -257,47 +352,59 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       my_agent[nt] = r < sg.rows ? (sg.row_lo + r) / p.G - sg.i_lo : -1;
     }
 
-    float m_run[NT][2], l_run[NT][2];
-    float oacc[MT][NT][4];
-    float zacc[MTZ][NT][4];
+    WarpState<D, NT, RK> st;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      m_run[nt][0] = m_run[nt][1] = NEG_INF;
-      l_run[nt][0] = l_run[nt][1] = 0.f;
+      st.m[nt][0] = st.m[nt][1] = NEG_INF;
+      st.l[nt][0] = st.l[nt][1] = 0.f;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) oacc[mt][nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) st.o[mt][nt][e] = 0.f;
 #pragma unroll
       for (int mz = 0; mz < MTZ; ++mz)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) zacc[mz][nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) st.z[mz][nt][e] = 0.f;
     }
 
     for (int tile = sg.lo; tile < hi_e; ++tile) {
-      mbar_wait_bounded(&full[stage], phase, abort_flag, p.flags);
-      const uint32_t Ks = ring_s + stage * lay.stage_bytes;
+      const bool mine = (ntile % NOG) == og;
+      const int my_stage = stage;
+      const uint32_t my_phase = phase;
+      ++ntile;
+      if (++stage == p.stages) {
+        stage = 0;
+        phase ^= 1;
+      }
+      if (!mine) continue;
+      mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags);
+      const uint32_t Ks = ring_s + my_stage * lay.stage_bytes;
       const uint32_t Vs = Ks + KV_BYTES;
       const uint32_t Us = Vs + KV_BYTES;
-      const int kbase = tile * KT + 16 * warp;
+      const int kw = 32 * kh;                 // first key of this warp inside the tile
+      const int kbase = tile * KT + kw;       // absolute key
 
-      // ---- S^T = K Q^T : 16 keys x RP rows per warp
-      float sacc[NT][4];
+      // ---- S^T = K Q^T : two 16-key blocks x RP rows (2 x NT independent chains)
+      float sacc[2][NT][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[kb][nt][e] = 0.f;
 #pragma unroll
       for (int ks = 0; ks < KS; ks += 2) {
-        uint32_t a[2][4];
+        uint32_t a[2][2][4];  // [kb][k-step][reg]
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int j = lane >> 3;
-          const int key = 16 * warp + (j & 1) * 8 + (lane & 7);
-          const int ch = (ks + kk) * 2 + (j >> 1);
-          const uint32_t addr = Ks + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
-          ldsm_x4(a[kk][0], a[kk][1], a[kk][2], a[kk][3], addr);
-        }
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const int j = lane >> 3;
+            const int key = kw + 16 * kb + (j & 1) * 8 + (lane & 7);
+            const int ch = (ks + kk) * 2 + (j >> 1);
+            const uint32_t addr = Ks + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+            ldsm_x4(a[kb][kk][0], a[kb][kk][1], a[kb][kk][2], a[kb][kk][3], addr);
+          }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int row = nt * 8 + (lane & 7);
@@ -305,89 +412,142 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           const uint32_t addr = q_s + row * (D * 2) + (((ch & ~7) | ((ch & 7) ^ (row & 7))) << 4);
           uint32_t b0, b1, b2, b3;
           ldsm_x4(b0, b1, b2, b3, addr);
-          mma_bf16_16816(sacc[nt], a[0][0], a[0][1], a[0][2], a[0][3], b0, b1);
-          mma_bf16_16816(sacc[nt], a[1][0], a[1][1], a[1][2], a[1][3], b2, b3);
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            mma_bf16_16816(sacc[kb][nt], a[kb][0][0], a[kb][0][1], a[kb][0][2], a[kb][0][3], b0, b1);
+            mma_bf16_16816(sacc[kb][nt], a[kb][1][0], a[kb][1][1], a[kb][1][2], a[kb][1][3], b2, b3);
+          }
         }
       }
 
-      // ---- online softmax over this warp's 16 keys (rows are columns of S^T)
-      const int key_a = kbase + g8, key_b = key_a + 8;
-      const bool va = key_a < sl, vb = key_b < sl;
-      uint32_t pb[NT][2];
+      // ---- online softmax over this warp's 32 keys (rows are columns of S^T).
+      // The reference max of a row only moves when the tile max exceeds it by
+      // more than 2^8 (log2 units): probabilities then stay <= 2^8 and the
+      // accumulators need rescaling only on those rare tiles.  The result is
+      // exact either way, since numerator and denominator share the reference.
+      bool valid[2][2];
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        valid[kb][0] = kbase + 16 * kb + g8 < sl;
+        valid[kb][1] = kbase + 16 * kb + g8 + 8 < sl;
+      }
+      float mx[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float s0 = va ? sacc[nt][0] * p.scale_log2 : NEG_INF;
-        float s1 = va ? sacc[nt][1] * p.scale_log2 : NEG_INF;
-        float s2 = vb ? sacc[nt][2] * p.scale_log2 : NEG_INF;
-        float s3 = vb ? sacc[nt][3] * p.scale_log2 : NEG_INF;
-        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        for (int kb = 0; kb < 2; ++kb) {
+          sacc[kb][nt][0] = valid[kb][0] ? sacc[kb][nt][0] * p.scale_log2 : NEG_INF;
+          sacc[kb][nt][1] = valid[kb][0] ? sacc[kb][nt][1] * p.scale_log2 : NEG_INF;
+          sacc[kb][nt][2] = valid[kb][1] ? sacc[kb][nt][2] * p.scale_log2 : NEG_INF;
+          sacc[kb][nt][3] = valid[kb][1] ? sacc[kb][nt][3] * p.scale_log2 : NEG_INF;
         }
-        const float mn0 = fmaxf(m_run[nt][0], mx0), mn1 = fmaxf(m_run[nt][1], mx1);
-        const float mu0 = mn0 == NEG_INF ? 0.f : mn0, mu1 = mn1 == NEG_INF ? 0.f : mn1;
-        const float al0 = fast_exp2(m_run[nt][0] - mu0), al1 = fast_exp2(m_run[nt][1] - mu1);
-        m_run[nt][0] = mn0;
-        m_run[nt][1] = mn1;
-        const float p0 = fast_exp2(s0 - mu0), p1 = fast_exp2(s1 - mu1);
-        const float p2 = fast_exp2(s2 - mu0), p3 = fast_exp2(s3 - mu1);
-        l_run[nt][0] = l_run[nt][0] * al0 + (p0 + p2);
-        l_run[nt][1] = l_run[nt][1] * al1 + (p1 + p3);
+        mx[nt][0] = fmaxf(fmaxf(sacc[0][nt][0], sacc[0][nt][2]), fmaxf(sacc[1][nt][0], sacc[1][nt][2]));
+        mx[nt][1] = fmaxf(fmaxf(sacc[0][nt][1], sacc[0][nt][3]), fmaxf(sacc[1][nt][1], sacc[1][nt][3]));
+      }
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          oacc[mt][nt][0] *= al0;
-          oacc[mt][nt][1] *= al1;
-          oacc[mt][nt][2] *= al0;
-          oacc[mt][nt][3] *= al1;
-        }
+      for (int o = 4; o < 32; o <<= 1)
 #pragma unroll
-        for (int mz = 0; mz < MTZ; ++mz) {
-          zacc[mz][nt][0] *= al0;
-          zacc[mz][nt][1] *= al1;
-          zacc[mz][nt][2] *= al0;
-          zacc[mz][nt][3] *= al1;
+        for (int nt = 0; nt < NT; ++nt) {
+          mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], o));
+          mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], o));
         }
-        pb[nt][0] = movmatrix_t(pack_bf16x2(p0, p1));
-        pb[nt][1] = movmatrix_t(pack_bf16x2(p2, p3));
+      bool need = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        need |= (mx[nt][0] > st.m[nt][0] + 8.f) || (mx[nt][1] > st.m[nt][1] + 8.f);
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float al[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float mn = fmaxf(st.m[nt][e], mx[nt][e]);
+            al[e] = mn == NEG_INF ? 1.f : fast_exp2(st.m[nt][e] - mn);
+            st.m[nt][e] = mn;
+            st.l[nt][e] *= al[e];
+          }
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            st.o[mt][nt][0] *= al[0];
+            st.o[mt][nt][1] *= al[1];
+            st.o[mt][nt][2] *= al[0];
+            st.o[mt][nt][3] *= al[1];
+          }
+#pragma unroll
+          for (int mz = 0; mz < MTZ; ++mz) {
+            st.z[mz][nt][0] *= al[0];
+            st.z[mz][nt][1] *= al[1];
+            st.z[mz][nt][2] *= al[0];
+            st.z[mz][nt][3] *= al[1];
+          }
+        }
+      }
+      uint32_t pb[2][NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float mu0 = st.m[nt][0] == NEG_INF ? 0.f : st.m[nt][0];
+        const float mu1 = st.m[nt][1] == NEG_INF ? 0.f : st.m[nt][1];
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          const float p0 = fast_exp2(sacc[kb][nt][0] - mu0), p1 = fast_exp2(sacc[kb][nt][1] - mu1);
+          const float p2 = fast_exp2(sacc[kb][nt][2] - mu0), p3 = fast_exp2(sacc[kb][nt][3] - mu1);
+          st.l[nt][0] += p0 + p2;
+          st.l[nt][1] += p1 + p3;
+          pb[kb][nt][0] = movmatrix_t(pack_bf16x2(p0, p1));
+          pb[kb][nt][1] = movmatrix_t(pack_bf16x2(p2, p3));
+        }
       }
 
       // ---- O^T += V^T P^T ; V rows past seq_len are selected out
       const bool boundary = tile * KT + KT > sl;
-      uint32_t vm_lo = 0xffffffffu, vm_hi = 0xffffffffu;
-      if (boundary) {
-        const int k0 = kbase + 2 * t4;
-        vm_lo = (k0 < sl ? 0x0000ffffu : 0u) | (k0 + 1 < sl ? 0xffff0000u : 0u);
-        vm_hi = (k0 + 8 < sl ? 0x0000ffffu : 0u) | (k0 + 9 < sl ? 0xffff0000u : 0u);
-      }
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const int j = lane >> 3;
-        const int key = 16 * warp + (j >> 1) * 8 + (lane & 7);
-        const int ch = 2 * mt + (j & 1);
-        const uint32_t addr = Vs + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(a0, a1, a2, a3, addr);
-        a0 &= vm_lo;
-        a1 &= vm_lo;
-        a2 &= vm_hi;
-        a3 &= vm_hi;
+      for (int kb = 0; kb < 2; ++kb) {
+        uint32_t vm_lo = 0xffffffffu, vm_hi = 0xffffffffu;
+        if (boundary) {
+          const int k0 = kbase + 16 * kb + 2 * t4;
+          vm_lo = (k0 < sl ? 0x0000ffffu : 0u) | (k0 + 1 < sl ? 0xffff0000u : 0u);
+          vm_hi = (k0 + 8 < sl ? 0x0000ffffu : 0u) | (k0 + 9 < sl ? 0xffff0000u : 0u);
+        }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(oacc[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+        for (int mt = 0; mt < MT; ++mt) {
+          const int j = lane >> 3;
+          const int key = kw + 16 * kb + (j >> 1) * 8 + (lane & 7);
+          const int ch = 2 * mt + (j & 1);
+          const uint32_t addr = Vs + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(a0, a1, a2, a3, addr);
+          a0 &= vm_lo;
+          a1 &= vm_lo;
+          a2 &= vm_hi;
+          a3 &= vm_hi;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(st.o[mt][nt], a0, a1, a2, a3, pb[kb][nt][0], pb[kb][nt][1]);
+        }
       }
 
       // ---- Z^T += U_i^T P^T over rows of agent i; U rows < a_i or >= seq_len selected out
       const int tile_key0 = tile * KT;
-      if (tile_key0 + KT > 0) {
-        const bool lr_full = p.mode == LRKV_BASE_LR_SHARED && !boundary && a_max <= tile_key0;
-        for (int ag = 0; ag < (lr_full ? 1 : sg.n_ag); ++ag) {
-          const int a_i = lr_full ? 0 : a_sm[ag];
-          if (tile_key0 + KT <= a_i) continue;         // producer did not load this U tile
-          if (kbase + 16 <= a_i || kbase >= sl) continue;  // nothing of this warp's slice is adapted
-          const int slot = p.mode == LRKV_BASE_SHARED ? ag : 0;
-          const uint32_t ub = Us + slot * U_BYTES;
-          const int k0 = kbase + 2 * t4;
+      const bool lr_full = p.mode == LRKV_BASE_LR_SHARED && !boundary && a_max <= tile_key0;
+      const int n_pass = lr_full ? 1 : sg.n_ag;
+      for (int ag = 0; ag < n_pass; ++ag) {
+        const int a_i = lr_full ? 0 : a_sm[ag];
+        if (tile_key0 + KT <= a_i) continue;            // producer did not load this U tile
+        if (kbase + 32 <= a_i || kbase >= sl) continue;  // nothing of this warp's keys is adapted
+        const int slot = p.mode == LRKV_BASE_SHARED ? ag : 0;
+        const uint32_t ub = Us + slot * U_BYTES;
+        int nt_lo = 0, nt_hi = NT - 1;
+        if (!lr_full) {
+          const int r_first = (sg.i_lo + ag) * p.G - sg.row_lo;
+          const int r_last = r_first + p.G - 1;
+          nt_lo = r_first > 0 ? r_first / 8 : 0;
+          nt_hi = r_last / 8 < NT - 1 ? r_last / 8 : NT - 1;
+        }
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb) {
+          const int k16 = kbase + 16 * kb;
+          if (k16 + 16 <= a_i || k16 >= sl) continue;
+          const int k0 = k16 + 2 * t4;
           const bool ok0 = k0 >= a_i && k0 < sl, ok1 = k0 + 1 >= a_i && k0 + 1 < sl;
           const bool ok8 = k0 + 8 >= a_i && k0 + 8 < sl, ok9 = k0 + 9 >= a_i && k0 + 9 < sl;
           const uint32_t um_lo = (ok0 ? 0x0000ffffu : 0u) | (ok1 ? 0xffff0000u : 0u);
@@ -396,11 +556,11 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           for (int mz = 0; mz < MTZ; ++mz) {
             uint32_t a0, a1 = 0, a2, a3 = 0;
             if constexpr (RK == 8) {
-              const int key = 16 * warp + ((lane >> 3) & 1) * 8 + (lane & 7);
+              const int key = kw + 16 * kb + ((lane >> 3) & 1) * 8 + (lane & 7);
               ldsm_x2_t(a0, a2, ub + key * (RK * 2));
             } else {
               const int j = lane >> 3;
-              const int key = 16 * warp + (j >> 1) * 8 + (lane & 7);
+              const int key = kw + 16 * kb + (j >> 1) * 8 + (lane & 7);
               const int ch = 2 * mz + (j & 1);
               ldsm_x4_t(a0, a1, a2, a3, ub + key * (RK * 2) + ch * 16);
             }
@@ -410,99 +570,63 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
             a3 &= um_hi;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              const bool mine = lr_full ? (my_agent[nt] >= 0) : (my_agent[nt] == ag);
-              const uint32_t b0 = mine ? pb[nt][0] : 0u, b1 = mine ? pb[nt][1] : 0u;
-              // skip n-tiles holding none of this agent's rows (warp-uniform test)
-              if (!lr_full) {
-                const int r_first = (sg.i_lo + ag) * p.G - sg.row_lo;
-                const int r_last = r_first + p.G - 1;
-                if (r_last < nt * 8 || r_first > nt * 8 + 7) continue;
-              }
-              mma_bf16_16816(zacc[mz][nt], a0, a1, a2, a3, b0, b1);
+              if (nt < nt_lo || nt > nt_hi) continue;  // no row of this agent in this n-tile
+              const bool use = lr_full ? (my_agent[nt] >= 0) : (my_agent[nt] == ag);
+              const uint32_t b0 = use ? pb[kb][nt][0] : 0u, b1 = use ? pb[kb][nt][1] : 0u;
+              mma_bf16_16816(st.z[mz][nt], a0, a1, a2, a3, b0, b1);
             }
           }
         }
       }
 
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
-      if (++stage == p.stages) {
-        stage = 0;
-        phase ^= 1;
-      }
+      if (lane == 0) mbar_arrive(&empty[my_stage]);
     }
 
-    // ---- per-warp state -> shared memory (rows x [m, l, O, Z])
+    // ---- reduce l over the lanes that share a row, then merge the warps:
+    // owner groups pairwise (same key half), then the two key halves.
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float v = l_run[nt][e];
+        float v = st.l[nt][e];
         v += __shfl_xor_sync(0xffffffffu, v, 4);
         v += __shfl_xor_sync(0xffffffffu, v, 8);
         v += __shfl_xor_sync(0xffffffffu, v, 16);
-        l_run[nt][e] = v;
+        st.l[nt][e] = v;
       }
-    {
-      float* mr = merge + warp * REC;
-      float* mO = mr + 2 * RP;
-      float* mZ = mO + RP * D;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int r0 = nt * 8 + 2 * t4;
-        if (g8 == 0) {
-          mr[r0] = m_run[nt][0];
-          mr[r0 + 1] = m_run[nt][1];
-          mr[RP + r0] = l_run[nt][0];
-          mr[RP + r0 + 1] = l_run[nt][1];
-        }
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int d0 = mt * 16 + g8;
-          mO[r0 * D + d0] = oacc[mt][nt][0];
-          mO[(r0 + 1) * D + d0] = oacc[mt][nt][1];
-          mO[r0 * D + d0 + 8] = oacc[mt][nt][2];
-          mO[(r0 + 1) * D + d0 + 8] = oacc[mt][nt][3];
-        }
-#pragma unroll
-        for (int mz = 0; mz < MTZ; ++mz) {
-          const int k0 = mz * 16 + g8;
-          mZ[r0 * RK + k0] = zacc[mz][nt][0];
-          mZ[(r0 + 1) * RK + k0] = zacc[mz][nt][1];
-          if (k0 + 8 < RK) {
-            mZ[r0 * RK + k0 + 8] = zacc[mz][nt][2];
-            mZ[(r0 + 1) * RK + k0 + 8] = zacc[mz][nt][3];
-          }
-        }
-      }
+    // a chain NOG-1 -> ... -> 1 -> 0 through one shared record per key half
+    for (int src = NOG - 1; src >= 1; --src) {
+      if (og == src) store_state<D, NT, RK>(st, merge + kh * REC, g8, t4);
+      named_bar_sync(1, CT);
+      if (og == src - 1) absorb_state<D, NT, RK>(st, merge + kh * REC, g8, t4);
+      named_bar_sync(1, CT);
     }
-    named_bar_sync(1, NCW * 32);
+    if (og == 0) store_state<D, NT, RK>(st, merge + kh * REC, g8, t4);
+    named_bar_sync(1, CT);
 
-    // ---- merge the four warps into record 0
+    // ---- merge the two key halves into record 0
     if (tid < RP) {
-      float M = NEG_INF;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) M = fmaxf(M, merge[w * REC + tid]);
-      float L = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float mw = merge[w * REC + tid];
-        const float sc = mw == NEG_INF ? 0.f : fast_exp2(mw - M);
-        scw[w * RP + tid] = sc;
-        L += merge[w * REC + RP + tid] * sc;
-      }
+      const float m0 = merge[tid], m1 = merge[REC + tid];
+      const float M = fmaxf(m0, m1);
+      const float s0 = m0 == NEG_INF ? 0.f : fast_exp2(m0 - M);
+      const float s1 = m1 == NEG_INF ? 0.f : fast_exp2(m1 - M);
+      scw[tid] = s0;
+      scw[RP + tid] = s1;
+      merge[RP + tid] = merge[RP + tid] * s0 + merge[REC + RP + tid] * s1;
       merge[tid] = M;
-      merge[RP + tid] = L;
     }
-    named_bar_sync(1, NCW * 32);
-    for (int e = tid; e < RP * (D + RK); e += NCW * 32) {
+    named_bar_sync(1, CT);
+    for (int e4 = tid; e4 < RP * (D + RK) / 4; e4 += CT) {
+      const int e = e4 * 4;
       const int row = e < RP * D ? e / D : (e - RP * D) / RK;
-      float v = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) v += merge[w * REC + 2 * RP + e] * scw[w * RP + row];
-      merge[2 * RP + e] = v;
+      const float4 x0 = *reinterpret_cast<const float4*>(merge + 2 * RP + e);
+      const float4 x1 = *reinterpret_cast<const float4*>(merge + REC + 2 * RP + e);
+      const float s0 = scw[row], s1 = scw[RP + row];
+      *reinterpret_cast<float4*>(merge + 2 * RP + e) =
+          make_float4(x0.x * s0 + x1.x * s1, x0.y * s0 + x1.y * s1, x0.z * s0 + x1.z * s1, x0.w * s0 + x1.w * s1);
     }
-    named_bar_sync(1, NCW * 32);
+    named_bar_sync(1, CT);
 
     // ---- publish or finish this item
     const long long W = p.W;
@@ -512,9 +636,9 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     bool finish = true;
     if (segs > 1) {
       float* rec = p.partials + ((size_t)sg.item * p.max_segs + (size_t)(c - c_first)) * REC;
-      for (int e = tid * 4; e < REC; e += NCW * 32 * 4)
+      for (int e = tid * 4; e < REC; e += CT * 4)
         __stcg(reinterpret_cast<float4*>(rec + e), *reinterpret_cast<const float4*>(merge + e));
-      named_bar_sync(1, NCW * 32);
+      named_bar_sync(1, CT);
       if (tid == 0) {
         __threadfence();
         const int prev = atomicAdd(p.tickets + sg.item, 1);
@@ -522,7 +646,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
         if (last) p.tickets[sg.item] = 0;
         *bcast = last;
       }
-      named_bar_sync(1, NCW * 32);
+      named_bar_sync(1, CT);
       finish = *bcast != 0;
       if (finish) {
         __threadfence();
@@ -538,7 +662,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           merge[tid] = M;
           merge[RP + tid] = L;
         }
-        named_bar_sync(1, NCW * 32);
+        named_bar_sync(1, CT);
         for (int j0 = 0; j0 < segs; j0 += SEG_CHUNK) {
           const int nj = min(SEG_CHUNK, segs - j0);
           if (tid < RP) {
@@ -548,49 +672,95 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
               scw[jj * RP + tid] = mj == NEG_INF ? 0.f : fast_exp2(mj - M);
             }
           }
-          named_bar_sync(1, NCW * 32);
-          for (int e = tid; e < RP * (D + RK); e += NCW * 32) {
-            const int row = e < RP * D ? e / D : (e - RP * D) / RK;
-            float v = j0 == 0 ? 0.f : merge[2 * RP + e];
-            for (int jj = 0; jj < nj; ++jj) v += __ldcg(base + (size_t)(j0 + jj) * REC + 2 * RP + e) * scw[jj * RP + row];
-            merge[2 * RP + e] = v;
+          named_bar_sync(1, CT);
+          constexpr int E4 = RP * (D + RK) / 4;
+          for (int e4 = tid; e4 < E4; e4 += 2 * CT) {
+            float4 acc[2];
+            int rows2[2];
+#pragma unroll
+            for (int u2 = 0; u2 < 2; ++u2) {
+              const int e = (e4 + u2 * CT) * 4;
+              rows2[u2] = e < RP * D ? e / D : (e - RP * D) / RK;
+              acc[u2] = (j0 == 0 || e4 + u2 * CT >= E4) ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                                          : *reinterpret_cast<const float4*>(merge + 2 * RP + e);
+            }
+            for (int jj = 0; jj < nj; ++jj) {
+              const float* rj = base + (size_t)(j0 + jj) * REC + 2 * RP;
+#pragma unroll
+              for (int u2 = 0; u2 < 2; ++u2) {
+                if (e4 + u2 * CT >= E4) continue;
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(rj + (e4 + u2 * CT) * 4));
+                const float sc = scw[jj * RP + rows2[u2]];
+                acc[u2].x += x.x * sc;
+                acc[u2].y += x.y * sc;
+                acc[u2].z += x.z * sc;
+                acc[u2].w += x.w * sc;
+              }
+            }
+#pragma unroll
+            for (int u2 = 0; u2 < 2; ++u2)
+              if (e4 + u2 * CT < E4) *reinterpret_cast<float4*>(merge + 2 * RP + (e4 + u2 * CT) * 4) = acc[u2];
           }
-          named_bar_sync(1, NCW * 32);
+          named_bar_sync(1, CT);
         }
       }
     }
 
     if (finish) {
-      // out = (O + Z B_i,g) / l, once per row: the up-projection of Eq. 12
+      // out = (O + Z B_i,g) / l, once per row: the up-projection of Eq. 12.
+      // One thread per (agent, dim): the agent's B column is loaded once and
+      // reused by every GQA row of that agent.
       const float* mL = merge + RP;
       const float* mO = merge + 2 * RP;
       const float* mZ = mO + RP * D;
       const int HD = p.Hkv * D;
-      for (int e = tid; e < sg.rows * D; e += NCW * 32) {
-        const int row = e / D, dim = e % D;
-        const int grow = sg.row_lo + row;
-        const int agent = grow / p.G;
-        const int h = sg.g * p.G + grow % p.G;
-        const uint16_t* bcol =
-            static_cast<const uint16_t*>(p.b) + ((size_t)agent * RK) * HD + (size_t)sg.g * D + dim;
-        float acc = mO[row * D + dim];
+      for (int e = tid; e < sg.n_ag * D; e += CT) {
+        const int a_loc = e / D, dim = e % D;
+        const int agent = sg.i_lo + a_loc;
+        const uint16_t* bcol = static_cast<const uint16_t*>(p.b) + ((size_t)agent * RK) * HD + (size_t)sg.g * D + dim;
+        float bk[RK];
 #pragma unroll
-        for (int k = 0; k < RK; ++k) acc = fmaf(mZ[row * RK + k], bf16_to_f32(__ldg(bcol + (size_t)k * HD)), acc);
-        const float L = mL[row];
-        const float o = L > 0.f ? acc / L : 0.f;
-        const size_t oi = (((size_t)sg.s * p.N + agent) * p.Hq + h) * D + dim;
-        if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
-        else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+        for (int k = 0; k < RK; ++k) bk[k] = bf16_to_f32(__ldg(bcol + (size_t)k * HD));
+        int r_begin = agent * p.G - sg.row_lo, r_end = r_begin + p.G;
+        r_begin = r_begin < 0 ? 0 : r_begin;
+        r_end = r_end > sg.rows ? sg.rows : r_end;
+        for (int row = r_begin; row < r_end; ++row) {
+          float acc = mO[row * D + dim];
+#pragma unroll
+          for (int k = 0; k < RK; ++k) acc = fmaf(mZ[row * RK + k], bk[k], acc);
+          const float L = mL[row];
+          const float o = L > 0.f ? acc / L : 0.f;
+          const int grow = sg.row_lo + row;
+          const int h = sg.g * p.G + grow % p.G;
+          const size_t oi = (((size_t)sg.s * p.N + agent) * p.Hq + h) * D + dim;
+          if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
+          else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+        }
       }
     }
-    named_bar_sync(1, NCW * 32);
+    named_bar_sync(1, CT);
   }
 }
 
+// Warp roles: warpgroup 0 is the producer (one warp issues the copies, its
+// register budget is cut to kProducerRegs), warpgroups 1..NG consume.  The
+// block is launched with THREADS x kLaunchRegs registers; the split
+// kProducerRegs x 128 + kConsumerRegs x 128 x NG must not exceed that total.
+template <int NT>
+struct Groups {
+  static constexpr int NG = NT <= 3 ? 2 : 1;  // 32 padded rows need the whole register file: one group
+  static constexpr int THREADS = (NG + 1) * 128;
+};
+constexpr int kLaunchRegs = 168;     // 65536 / 384, rounded down to a multiple of 8
+constexpr int kProducerRegs = 32;
+constexpr int kConsumerRegs = 232;
+static_assert(kProducerRegs * 128 + kConsumerRegs * 256 <= kLaunchRegs * 384, "register split exceeds the launch");
+
 template <int D, int NT, int RK>
-__global__ void __launch_bounds__(DEC_THREADS, 1)
+__global__ void __launch_bounds__(Groups<NT>::THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmU, const DecodeParams p) {
+  constexpr int NG = Groups<NT>::NG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const DecodeSmem lay = decode_smem_plan(D, NT, RK, p.n_u_slots, p.stages);
@@ -599,31 +769,38 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + p.stages);
   int* bcast = const_cast<int*>(abort_flag) + 1;
   const int warp = threadIdx.x >> 5;
+  if (p.stages % decode_owner_groups(NT) != 0) {  // every stage must keep one owner group
+    if (threadIdx.x == 0) atomicOr(p.flags, LRKV_DEVFLAG_TIMEOUT);
+    return;
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NCW);
+      mbar_init(&empty[s], 2);  // the two warps of the pair that owns the tile
     }
     *abort_flag = 0;
     *bcast = 0;
     fence_barrier_init();
   }
-  if (warp == NCW && (threadIdx.x & 31) == 0) {
+  if (warp == 0 && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmU);
   }
   __syncthreads();
   pdl_wait();
+  pdl_launch_dependents();
   const long long C = gridDim.x;
   const long long t_begin = (long long)blockIdx.x * p.W / C;
   const long long t_end = (long long)(blockIdx.x + 1) * p.W / C;
-  if (warp == NCW) {
-    decode_producer<D, RK>(p, &tmK, &tmV, &tmU, smem, lay.stage_bytes, full, empty, abort_flag, t_begin, t_end);
+  if (warp < 4) {
+    if constexpr (NG == 2) setmaxnreg_dec<kProducerRegs>();
+    if (warp == 0)
+      decode_producer<D, RK>(p, &tmK, &tmV, &tmU, smem, lay.stage_bytes, full, empty, abort_flag, t_begin, t_end);
   } else {
-    decode_consumers<D, NT, RK>(p, smem, lay, full, empty, abort_flag, bcast, t_begin, t_end);
+    if constexpr (NG == 2) setmaxnreg_inc<kConsumerRegs>();
+    decode_consumers<D, NT, RK, NG>(p, smem, lay, full, empty, abort_flag, bcast, t_begin, t_end);
   }
-  pdl_launch_dependents();
 }
 
 template <int D, int NT, int RK>
@@ -638,7 +815,7 @@ lrkv_status launch_one(const DecodeParams& p, const void* tmK, const void* tmV, 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
-  cfg.blockDim = dim3(DEC_THREADS);
+  cfg.blockDim = dim3(Groups<NT>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -681,7 +858,5 @@ lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, const vo
   }
   return LRKV_ERR_UNSUPPORTED;
 }
-
-int decode_threads() { return DEC_THREADS; }
 
 }  // namespace lrkv

@@ -67,7 +67,7 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int D, int NT, int RK, in
   s.q_off = s.ring_bytes;
   s.merge_off = s.q_off + round_up(RP * D * 2, 128);
   const int rec = RP * (D + RK + 2) * 4;
-  s.scw_off = s.merge_off + 4 * rec;
+  s.scw_off = s.merge_off + 2 * rec;
   s.a_off = s.scw_off + 8 * RP * 4;
   s.bar_off = round_up(s.a_off + kMaxAgents * 4, 16);
   s.total = s.bar_off + 2 * stages * 8 + 64;
@@ -75,6 +75,14 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int D, int NT, int RK, in
 }
 
 inline size_t decode_record_floats(int NT, int D, int RK) { return (size_t)NT * 8 * (D + RK + 2); }
+
+// Consumer warps of the decode kernel form owner groups (pairs of warps);
+// tile n of a CTA goes to group n % groups and to ring stage n % stages.
+// The stage count must be a multiple of the group count so that every stage
+// always has the same owner: an mbarrier parity wait can only tell a phase
+// from the one just before it, so a group must never wait for use u+1 of a
+// stage while another group still holds use u.
+__host__ __device__ inline int decode_owner_groups(int NT) { return (NT <= 3 ? 2 : 1) * 2; }
 
 // Owner CTA of flattened tile t when W tiles are split evenly over C CTAs:
 // CTA c covers [c*W/C, (c+1)*W/C).
