@@ -103,10 +103,17 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_floa
 // ---------------------------------------------------------------------------
 // producer warp
 // ---------------------------------------------------------------------------
+// Tile n of the CTA (counted over all its segments) goes to ring stage
+// n % stages.  Before copying, the producer writes n into seq[stage]; a
+// consumer waits for its tile number there before it waits on the stage's
+// mbarrier, so that a parity wait can never be satisfied by an older phase
+// of the same stage (the stage count need not be a multiple of the number
+// of consumer groups).
 template <int D, int RK>
 __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                 const CUtensorMap* tmU, uint8_t* ring, int stage_bytes, uint64_t* full,
-                                uint64_t* empty, volatile int* abort_flag, long long t_begin, long long t_end) {
+                                uint64_t* empty, volatile int* seq, volatile int* abort_flag, long long t_begin,
+                                long long t_end) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = policy_evict_first();
   const uint64_t pol_u = policy_evict_last();
@@ -114,7 +121,7 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
   constexpr int U_BYTES = KT * RK * 2;
   int stage = 0;
   uint32_t phase = 0;
-  long long issued = 0;
+  int n = 0;
   for (long long t = t_begin; t < t_end;) {
     Seg sg = make_seg(p, t, t_end, false);
     t += sg.hi - sg.lo;
@@ -123,7 +130,7 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
     // lane j < n_ag holds the offset of agent i_lo + j
     const int my_a = lane < sg.n_ag ? load_offset(p, sg.s, sg.i_lo + lane, false) : 0x7fffffff;
     int pid_reg = 0;
-    for (int tile = sg.lo; tile < hi_e; ++tile) {
+    for (int tile = sg.lo; tile < hi_e; ++tile, ++n) {
       const int k = tile - sg.lo;
       if (p.paged && (k & 31) == 0) {
         const int tt = tile + lane;
@@ -132,24 +139,23 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
       const int phys = p.paged ? __shfl_sync(0xffffffffu, pid_reg, k & 31) : 0;
       const int tile_end_key = tile * KT + KT;
       const unsigned need = __ballot_sync(0xffffffffu, lane < sg.n_ag && tile_end_key > my_a);
-      unsigned umask;
-      if (p.mode == LRKV_BASE_SHARED) umask = need;
-      else umask = need ? 1u : 0u;
+      const unsigned umask = p.mode == LRKV_BASE_SHARED ? need : (need ? 1u : 0u);
       const bool page_ok = !p.paged || (phys >= 0 && phys < p.num_pages);
       const uint32_t bytes = (page_ok ? 2 * KV_BYTES : 0) + __popc(umask) * U_BYTES;
       mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.flags);
       if (lane == 0) {
         if (!page_ok) atomicOr(p.flags, LRKV_DEVFLAG_PAGE);
+        seq[stage] = n;
         uint8_t* st = ring + (size_t)stage * stage_bytes;
         if (bytes == 0) {
           mbar_arrive(&full[stage]);
         } else {
           mbar_arrive_expect_tx(&full[stage], bytes);
           if (page_ok) {
+            const int c1 = p.paged ? 0 : tile * KT;
+            const int c3 = p.paged ? phys : sg.s;
 #pragma unroll
             for (int hh = 0; hh < D / 64; ++hh) {
-              const int c1 = p.paged ? 0 : tile * KT;
-              const int c3 = p.paged ? phys : sg.s;
               tma_load_4d(st + hh * (KT * 128), tmK, &full[stage], hh * 64, c1, sg.g, c3, pol_kv);
               tma_load_4d(st + KV_BYTES + hh * (KT * 128), tmV, &full[stage], hh * 64, c1, sg.g, c3, pol_kv);
             }
@@ -165,7 +171,6 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
         }
       }
       __syncwarp();
-      ++issued;
       if (++stage == p.stages) {
         stage = 0;
         phase ^= 1;
@@ -175,10 +180,10 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
   // After an abort the consumers may stop waiting; make sure no copy issued by
   // this CTA is still landing in shared memory when the CTA exits.
   if (*abort_flag && lane == 0) {
-    long long n = issued < p.stages ? issued : p.stages;
+    const int m = n < p.stages ? n : p.stages;
     int st = stage;
     uint32_t ph = phase;
-    for (long long j = 0; j < n; ++j) {
+    for (int j = 0; j < m; ++j) {
       if (--st < 0) {
         st = p.stages - 1;
         ph ^= 1;
@@ -193,101 +198,92 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
 // ---------------------------------------------------------------------------
 // consumer warps
 // ---------------------------------------------------------------------------
-// NG warpgroups of four warps.  Tile n of the CTA (counted over all its
-// segments) belongs to group n % NG; warp w of a group owns keys
-// [16 w, 16 w + 16) of its tiles.  Each warp keeps its own online-softmax
-// state; the states are merged in shared memory at the end of a segment.
-template <int D, int NT, int RK>
-struct WarpState {
+// NOG groups of NT warps.  Tile n of the CTA belongs to group n % NOG; warp
+// w of a group owns query rows [8 w, 8 w + 8) of the work item and runs them
+// over all 64 keys of its group's tiles.  The groups hold the same rows for
+// different tiles and are merged at the end of a segment.
+template <int D, int RK>
+struct RowState {
   static constexpr int MT = D / 16;
   static constexpr int MTZ = RK >= 16 ? RK / 16 : 1;
-  float m[NT][2], l[NT][2];
-  float o[MT][NT][4];
-  float z[MTZ][NT][4];
+  float m[2], l[2];       // rows 2 t4, 2 t4 + 1 of the warp's 8
+  float o[MT][4];         // O^T: dims (16 mt + g8, + 8) x rows
+  float z[MTZ][4];        // Z^T: ranks x rows
 };
 
-// Write a warp's state (l already reduced over its lanes) to a record
-// [m(RP) | l(RP) | O(RP x D) | Z(RP x RK)].
-template <int D, int NT, int RK>
-__device__ __forceinline__ void store_state(const WarpState<D, NT, RK>& st, float* mr, int g8, int t4) {
-  constexpr int RP = NT * 8;
-  float* mO = mr + 2 * RP;
+// Record layout: [m(RP) | l(RP) | O(RP x D) | Z(RP x RK)], rows r0.. of this warp.
+template <int D, int RK>
+__device__ __forceinline__ void store_rows(const RowState<D, RK>& st, float* rec, int RP, int rbase, int g8, int t4) {
+  float* mO = rec + 2 * RP;
   float* mZ = mO + RP * D;
+  const int r0 = rbase + 2 * t4;
+  if (g8 == 0) {
+    rec[r0] = st.m[0];
+    rec[r0 + 1] = st.m[1];
+    rec[RP + r0] = st.l[0];
+    rec[RP + r0 + 1] = st.l[1];
+  }
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int r0 = nt * 8 + 2 * t4;
-    if (g8 == 0) {
-      mr[r0] = st.m[nt][0];
-      mr[r0 + 1] = st.m[nt][1];
-      mr[RP + r0] = st.l[nt][0];
-      mr[RP + r0 + 1] = st.l[nt][1];
-    }
+  for (int mt = 0; mt < RowState<D, RK>::MT; ++mt) {
+    const int d0 = mt * 16 + g8;
+    mO[r0 * D + d0] = st.o[mt][0];
+    mO[(r0 + 1) * D + d0] = st.o[mt][1];
+    mO[r0 * D + d0 + 8] = st.o[mt][2];
+    mO[(r0 + 1) * D + d0 + 8] = st.o[mt][3];
+  }
 #pragma unroll
-    for (int mt = 0; mt < WarpState<D, NT, RK>::MT; ++mt) {
-      const int d0 = mt * 16 + g8;
-      mO[r0 * D + d0] = st.o[mt][nt][0];
-      mO[(r0 + 1) * D + d0] = st.o[mt][nt][1];
-      mO[r0 * D + d0 + 8] = st.o[mt][nt][2];
-      mO[(r0 + 1) * D + d0 + 8] = st.o[mt][nt][3];
-    }
-#pragma unroll
-    for (int mz = 0; mz < WarpState<D, NT, RK>::MTZ; ++mz) {
-      const int k0 = mz * 16 + g8;
-      mZ[r0 * RK + k0] = st.z[mz][nt][0];
-      mZ[(r0 + 1) * RK + k0] = st.z[mz][nt][1];
-      if (k0 + 8 < RK) {
-        mZ[r0 * RK + k0 + 8] = st.z[mz][nt][2];
-        mZ[(r0 + 1) * RK + k0 + 8] = st.z[mz][nt][3];
-      }
+  for (int mz = 0; mz < RowState<D, RK>::MTZ; ++mz) {
+    const int k0 = mz * 16 + g8;
+    mZ[r0 * RK + k0] = st.z[mz][0];
+    mZ[(r0 + 1) * RK + k0] = st.z[mz][1];
+    if (k0 + 8 < RK) {
+      mZ[r0 * RK + k0 + 8] = st.z[mz][2];
+      mZ[(r0 + 1) * RK + k0 + 8] = st.z[mz][3];
     }
   }
 }
 
-// st <- merge(st, record): the online-softmax combination of two partial states.
-template <int D, int NT, int RK>
-__device__ __forceinline__ void absorb_state(WarpState<D, NT, RK>& st, const float* mr, int g8, int t4) {
-  constexpr int RP = NT * 8;
-  const float* mO = mr + 2 * RP;
+// st <- the online-softmax combination of st and the stored rows.
+template <int D, int RK>
+__device__ __forceinline__ void absorb_rows(RowState<D, RK>& st, const float* rec, int RP, int rbase, int g8, int t4) {
+  const float* mO = rec + 2 * RP;
   const float* mZ = mO + RP * D;
   const float NEG_INF = -INFINITY;
+  const int r0 = rbase + 2 * t4;
+  float sa[2], so[2];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int r0 = nt * 8 + 2 * t4;
-    float sa[2], so[2];
+  for (int e = 0; e < 2; ++e) {
+    const float mo = rec[r0 + e];
+    const float M = fmaxf(st.m[e], mo);
+    sa[e] = st.m[e] == NEG_INF ? 0.f : fast_exp2(st.m[e] - M);
+    so[e] = mo == NEG_INF ? 0.f : fast_exp2(mo - M);
+    st.l[e] = st.l[e] * sa[e] + rec[RP + r0 + e] * so[e];
+    st.m[e] = M;
+  }
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float mo = mr[r0 + e];
-      const float M = fmaxf(st.m[nt][e], mo);
-      sa[e] = st.m[nt][e] == NEG_INF ? 0.f : fast_exp2(st.m[nt][e] - M);
-      so[e] = mo == NEG_INF ? 0.f : fast_exp2(mo - M);
-      st.l[nt][e] = st.l[nt][e] * sa[e] + mr[RP + r0 + e] * so[e];
-      st.m[nt][e] = M;
-    }
+  for (int mt = 0; mt < RowState<D, RK>::MT; ++mt) {
+    const int d0 = mt * 16 + g8;
+    st.o[mt][0] = st.o[mt][0] * sa[0] + mO[r0 * D + d0] * so[0];
+    st.o[mt][1] = st.o[mt][1] * sa[1] + mO[(r0 + 1) * D + d0] * so[1];
+    st.o[mt][2] = st.o[mt][2] * sa[0] + mO[r0 * D + d0 + 8] * so[0];
+    st.o[mt][3] = st.o[mt][3] * sa[1] + mO[(r0 + 1) * D + d0 + 8] * so[1];
+  }
 #pragma unroll
-    for (int mt = 0; mt < WarpState<D, NT, RK>::MT; ++mt) {
-      const int d0 = mt * 16 + g8;
-      st.o[mt][nt][0] = st.o[mt][nt][0] * sa[0] + mO[r0 * D + d0] * so[0];
-      st.o[mt][nt][1] = st.o[mt][nt][1] * sa[1] + mO[(r0 + 1) * D + d0] * so[1];
-      st.o[mt][nt][2] = st.o[mt][nt][2] * sa[0] + mO[r0 * D + d0 + 8] * so[0];
-      st.o[mt][nt][3] = st.o[mt][nt][3] * sa[1] + mO[(r0 + 1) * D + d0 + 8] * so[1];
-    }
-#pragma unroll
-    for (int mz = 0; mz < WarpState<D, NT, RK>::MTZ; ++mz) {
-      const int k0 = mz * 16 + g8;
-      st.z[mz][nt][0] = st.z[mz][nt][0] * sa[0] + mZ[r0 * RK + k0] * so[0];
-      st.z[mz][nt][1] = st.z[mz][nt][1] * sa[1] + mZ[(r0 + 1) * RK + k0] * so[1];
-      if (k0 + 8 < RK) {
-        st.z[mz][nt][2] = st.z[mz][nt][2] * sa[0] + mZ[r0 * RK + k0 + 8] * so[0];
-        st.z[mz][nt][3] = st.z[mz][nt][3] * sa[1] + mZ[(r0 + 1) * RK + k0 + 8] * so[1];
-      }
+  for (int mz = 0; mz < RowState<D, RK>::MTZ; ++mz) {
+    const int k0 = mz * 16 + g8;
+    st.z[mz][0] = st.z[mz][0] * sa[0] + mZ[r0 * RK + k0] * so[0];
+    st.z[mz][1] = st.z[mz][1] * sa[1] + mZ[(r0 + 1) * RK + k0] * so[1];
+    if (k0 + 8 < RK) {
+      st.z[mz][2] = st.z[mz][2] * sa[0] + mZ[r0 * RK + k0 + 8] * so[0];
+      st.z[mz][3] = st.z[mz][3] * sa[1] + mZ[(r0 + 1) * RK + k0 + 8] * so[1];
     }
   }
 }
 
-template <int D, int NT, int RK, int NG>
+template <int D, int NT, int RK>
 __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const DecodeSmem& lay, uint64_t* full,
-                                 uint64_t* empty, volatile int* abort_flag, int* bcast, long long t_begin,
-                                 long long t_end) {
+                                 uint64_t* empty, volatile int* seq, volatile int* abort_flag, int* bcast,
+                                 long long t_begin, long long t_end) {
   constexpr int RP = NT * 8;
   constexpr int KS = D / 16;
   constexpr int MT = D / 16;
@@ -295,16 +291,15 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   constexpr int KV_BYTES = KT * D * 2;
   constexpr int U_BYTES = KT * RK * 2;
   constexpr int REC = RP * (D + RK + 2);
-  constexpr int CT = NG * 4 * 32;  // consumer threads
-  const int tid = threadIdx.x - 128;  // 0 .. CT-1 (warpgroup 0 is the producer)
+  constexpr int NOG = kDecodeGroups;
+  constexpr int CT = NOG * NT * 32;   // consumer threads
+  const int tid = threadIdx.x;        // consumers are warps 0 .. NOG*NT-1
   const int warp = tid >> 5, lane = tid & 31;
-  constexpr int NOG = NG * 2;      // owner groups: pairs of warps, tile n goes to pair n % NOG
-  static_assert(NOG == (NT <= 3 ? 2 : 1) * 2, "owner groups must match decode_owner_groups()");
-  const int og = warp >> 1;        // owner group of this warp
-  const int kh = warp & 1;         // key half (32 of the 64 keys of a tile) of this warp
+  const int og = warp / NT;           // owner group
+  const int nw = warp % NT;           // n-tile (8 rows) of this warp
+  const int rbase = nw * 8;
   const int g8 = lane >> 2, t4 = lane & 3;
   const uint32_t ring_s = smem_u32(smem);
-  const uint32_t q_s = smem_u32(smem + lay.q_off);
   float* merge = reinterpret_cast<float*>(smem + lay.merge_off);
   float* scw = reinterpret_cast<float*>(smem + lay.scw_off);
   int* a_sm = reinterpret_cast<int*>(smem + lay.a_off);
@@ -323,51 +318,46 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     const int hi_e = seg_tiles_end(sg);
     const int sl = sg.sl;
 
-    // ---- stage this item's queries (rows x d, 16B chunks, XOR-swizzled) and offsets
-    {
-      constexpr int CH = D / 8;
-      for (int idx = tid; idx < RP * CH; idx += CT) {
-        const int row = idx / CH, ch = idx % CH;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (row < sg.rows) {
-          const int grow = sg.row_lo + row;
-          const int agent = grow / p.G;
-          const int h = sg.g * p.G + grow % p.G;
-          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
-                                                            (((size_t)sg.s * p.N + agent) * p.Hq + h) * D) + ch;
-          val = __ldg(src);
-        }
-        const int pch = (ch & ~7) | ((ch & 7) ^ (row & 7));
-        *reinterpret_cast<uint4*>(smem + lay.q_off + row * (D * 2) + pch * 16) = val;
-      }
-      if (tid < sg.n_ag) a_sm[tid] = load_offset(p, sg.s, sg.i_lo + tid, true);
-      named_bar_sync(1, CT);
+    if (tid < sg.n_ag) a_sm[tid] = load_offset(p, sg.s, sg.i_lo + tid, true);
+    // this warp's query rows as the B operand of S^T = K Q^T (kept in registers)
+    const int qrow = rbase + g8;  // row of this lane's B fragment
+    const bool qvalid = qrow < sg.rows;
+    const __nv_bfloat16* qptr = nullptr;
+    if (qvalid) {
+      const int grow = sg.row_lo + qrow;
+      qptr = static_cast<const __nv_bfloat16*>(p.q) +
+             (((size_t)sg.s * p.N + grow / p.G) * p.Hq + sg.g * p.G + grow % p.G) * D;
     }
+    uint32_t qf[KS][2];
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      qf[ks][0] = qvalid ? __ldg(reinterpret_cast<const unsigned int*>(qptr + ks * 16 + 2 * t4)) : 0u;
+      qf[ks][1] = qvalid ? __ldg(reinterpret_cast<const unsigned int*>(qptr + ks * 16 + 8 + 2 * t4)) : 0u;
+    }
+    named_bar_sync(1, CT);
     int a_max = 0;
     for (int j = 0; j < sg.n_ag; ++j) a_max = max(a_max, a_sm[j]);
-    int my_agent[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int r = nt * 8 + g8;
-      my_agent[nt] = r < sg.rows ? (sg.row_lo + r) / p.G - sg.i_lo : -1;
-    }
+    // agents whose rows meet this warp's 8 rows, and this lane's row's agent
+    const int w_row_lo = sg.row_lo + rbase;
+    const int w_rows = min(8, sg.rows - rbase);
+    const int ag_lo = w_rows > 0 ? w_row_lo / p.G - sg.i_lo : 0;
+    const int ag_hi = w_rows > 0 ? (w_row_lo + w_rows - 1) / p.G - sg.i_lo : -1;
+    const int my_agent = qvalid ? (sg.row_lo + qrow) / p.G - sg.i_lo : -1;
 
-    WarpState<D, NT, RK> st;
+    RowState<D, RK> st;
+    st.m[0] = st.m[1] = NEG_INF;
+    st.l[0] = st.l[1] = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      st.m[nt][0] = st.m[nt][1] = NEG_INF;
-      st.l[nt][0] = st.l[nt][1] = 0.f;
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
+      for (int e = 0; e < 4; ++e) st.o[mt][e] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) st.o[mt][nt][e] = 0.f;
+    for (int mz = 0; mz < MTZ; ++mz)
 #pragma unroll
-      for (int mz = 0; mz < MTZ; ++mz)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) st.z[mz][nt][e] = 0.f;
-    }
+      for (int e = 0; e < 4; ++e) st.z[mz][e] = 0.f;
 
     for (int tile = sg.lo; tile < hi_e; ++tile) {
+      const int my_n = ntile;
       const bool mine = (ntile % NOG) == og;
       const int my_stage = stage;
       const uint32_t my_phase = phase;
@@ -377,190 +367,167 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
         phase ^= 1;
       }
       if (!mine) continue;
+      // wait until the producer has issued this tile into the stage, then for its bytes
+      {
+        uint32_t spins = 0;
+        while (seq[my_stage] != my_n) {
+          if (*abort_flag || ++spins >= kSpinCap) {
+            if (!*abort_flag) {
+              *abort_flag = 1;
+              atomicOr(p.flags, LRKV_DEVFLAG_TIMEOUT);
+            }
+            break;
+          }
+        }
+      }
       mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags);
       const uint32_t Ks = ring_s + my_stage * lay.stage_bytes;
       const uint32_t Vs = Ks + KV_BYTES;
       const uint32_t Us = Vs + KV_BYTES;
-      const int kw = 32 * kh;                 // first key of this warp inside the tile
-      const int kbase = tile * KT + kw;       // absolute key
+      const int tile_key0 = tile * KT;
 
-      // ---- S^T = K Q^T : two 16-key blocks x RP rows (2 x NT independent chains)
-      float sacc[2][NT][4];
+      // ---- S^T = K Q^T : 4 blocks of 16 keys x this warp's 8 rows (4 independent chains)
+      float sacc[4][4];
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb)
+      for (int kb = 0; kb < 4; ++kb)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int e = 0; e < 4; ++e) sacc[kb][e] = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sacc[kb][nt][e] = 0.f;
+      for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
-      for (int ks = 0; ks < KS; ks += 2) {
-        uint32_t a[2][2][4];  // [kb][k-step][reg]
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const int j = lane >> 3;
-            const int key = kw + 16 * kb + (j & 1) * 8 + (lane & 7);
-            const int ch = (ks + kk) * 2 + (j >> 1);
-            const uint32_t addr = Ks + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
-            ldsm_x4(a[kb][kk][0], a[kb][kk][1], a[kb][kk][2], a[kb][kk][3], addr);
-          }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int row = nt * 8 + (lane & 7);
-          const int ch = ks * 2 + (lane >> 3);
-          const uint32_t addr = q_s + row * (D * 2) + (((ch & ~7) | ((ch & 7) ^ (row & 7))) << 4);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(b0, b1, b2, b3, addr);
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            mma_bf16_16816(sacc[kb][nt], a[kb][0][0], a[kb][0][1], a[kb][0][2], a[kb][0][3], b0, b1);
-            mma_bf16_16816(sacc[kb][nt], a[kb][1][0], a[kb][1][1], a[kb][1][2], a[kb][1][3], b2, b3);
-          }
+        for (int kb = 0; kb < 4; ++kb) {
+          const int j = lane >> 3;
+          const int key = 16 * kb + (j & 1) * 8 + (lane & 7);
+          const int ch = ks * 2 + (j >> 1);
+          const uint32_t addr = Ks + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a0, a1, a2, a3, addr);
+          mma_bf16_16816(sacc[kb], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
         }
       }
 
-      // ---- online softmax over this warp's 32 keys (rows are columns of S^T).
+      // ---- online softmax over the 64 keys (rows are columns of S^T).
       // The reference max of a row only moves when the tile max exceeds it by
       // more than 2^8 (log2 units): probabilities then stay <= 2^8 and the
       // accumulators need rescaling only on those rare tiles.  The result is
       // exact either way, since numerator and denominator share the reference.
-      bool valid[2][2];
+      float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        valid[kb][0] = kbase + 16 * kb + g8 < sl;
-        valid[kb][1] = kbase + 16 * kb + g8 + 8 < sl;
-      }
-      float mx[NT][2];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          sacc[kb][nt][0] = valid[kb][0] ? sacc[kb][nt][0] * p.scale_log2 : NEG_INF;
-          sacc[kb][nt][1] = valid[kb][0] ? sacc[kb][nt][1] * p.scale_log2 : NEG_INF;
-          sacc[kb][nt][2] = valid[kb][1] ? sacc[kb][nt][2] * p.scale_log2 : NEG_INF;
-          sacc[kb][nt][3] = valid[kb][1] ? sacc[kb][nt][3] * p.scale_log2 : NEG_INF;
-        }
-        mx[nt][0] = fmaxf(fmaxf(sacc[0][nt][0], sacc[0][nt][2]), fmaxf(sacc[1][nt][0], sacc[1][nt][2]));
-        mx[nt][1] = fmaxf(fmaxf(sacc[0][nt][1], sacc[0][nt][3]), fmaxf(sacc[1][nt][1], sacc[1][nt][3]));
+      for (int kb = 0; kb < 4; ++kb) {
+        const bool va = tile_key0 + 16 * kb + g8 < sl;
+        const bool vb = tile_key0 + 16 * kb + g8 + 8 < sl;
+        sacc[kb][0] = va ? sacc[kb][0] * p.scale_log2 : NEG_INF;
+        sacc[kb][1] = va ? sacc[kb][1] * p.scale_log2 : NEG_INF;
+        sacc[kb][2] = vb ? sacc[kb][2] * p.scale_log2 : NEG_INF;
+        sacc[kb][3] = vb ? sacc[kb][3] * p.scale_log2 : NEG_INF;
+        mx0 = fmaxf(mx0, fmaxf(sacc[kb][0], sacc[kb][2]));
+        mx1 = fmaxf(mx1, fmaxf(sacc[kb][1], sacc[kb][3]));
       }
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mx[nt][0] = fmaxf(mx[nt][0], __shfl_xor_sync(0xffffffffu, mx[nt][0], o));
-          mx[nt][1] = fmaxf(mx[nt][1], __shfl_xor_sync(0xffffffffu, mx[nt][1], o));
-        }
-      bool need = false;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        need |= (mx[nt][0] > st.m[nt][0] + 8.f) || (mx[nt][1] > st.m[nt][1] + 8.f);
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const bool need = (mx0 > st.m[0] + 8.f) || (mx1 > st.m[1] + 8.f);
       if (__any_sync(0xffffffffu, need)) {
+        float al[2];
+        const float mxv[2] = {mx0, mx1};
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          float al[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float mn = fmaxf(st.m[nt][e], mx[nt][e]);
-            al[e] = mn == NEG_INF ? 1.f : fast_exp2(st.m[nt][e] - mn);
-            st.m[nt][e] = mn;
-            st.l[nt][e] *= al[e];
-          }
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            st.o[mt][nt][0] *= al[0];
-            st.o[mt][nt][1] *= al[1];
-            st.o[mt][nt][2] *= al[0];
-            st.o[mt][nt][3] *= al[1];
-          }
-#pragma unroll
-          for (int mz = 0; mz < MTZ; ++mz) {
-            st.z[mz][nt][0] *= al[0];
-            st.z[mz][nt][1] *= al[1];
-            st.z[mz][nt][2] *= al[0];
-            st.z[mz][nt][3] *= al[1];
-          }
-        }
-      }
-      uint32_t pb[2][NT][2];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float mu0 = st.m[nt][0] == NEG_INF ? 0.f : st.m[nt][0];
-        const float mu1 = st.m[nt][1] == NEG_INF ? 0.f : st.m[nt][1];
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          const float p0 = fast_exp2(sacc[kb][nt][0] - mu0), p1 = fast_exp2(sacc[kb][nt][1] - mu1);
-          const float p2 = fast_exp2(sacc[kb][nt][2] - mu0), p3 = fast_exp2(sacc[kb][nt][3] - mu1);
-          st.l[nt][0] += p0 + p2;
-          st.l[nt][1] += p1 + p3;
-          pb[kb][nt][0] = movmatrix_t(pack_bf16x2(p0, p1));
-          pb[kb][nt][1] = movmatrix_t(pack_bf16x2(p2, p3));
-        }
-      }
-
-      // ---- O^T += V^T P^T ; V rows past seq_len are selected out
-      const bool boundary = tile * KT + KT > sl;
-#pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        uint32_t vm_lo = 0xffffffffu, vm_hi = 0xffffffffu;
-        if (boundary) {
-          const int k0 = kbase + 16 * kb + 2 * t4;
-          vm_lo = (k0 < sl ? 0x0000ffffu : 0u) | (k0 + 1 < sl ? 0xffff0000u : 0u);
-          vm_hi = (k0 + 8 < sl ? 0x0000ffffu : 0u) | (k0 + 9 < sl ? 0xffff0000u : 0u);
+        for (int e = 0; e < 2; ++e) {
+          const float mn = fmaxf(st.m[e], mxv[e]);
+          al[e] = mn == NEG_INF ? 1.f : fast_exp2(st.m[e] - mn);
+          st.m[e] = mn;
+          st.l[e] *= al[e];
         }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
+          st.o[mt][0] *= al[0];
+          st.o[mt][1] *= al[1];
+          st.o[mt][2] *= al[0];
+          st.o[mt][3] *= al[1];
+        }
+#pragma unroll
+        for (int mz = 0; mz < MTZ; ++mz) {
+          st.z[mz][0] *= al[0];
+          st.z[mz][1] *= al[1];
+          st.z[mz][2] *= al[0];
+          st.z[mz][3] *= al[1];
+        }
+      }
+      const float mu0 = st.m[0] == NEG_INF ? 0.f : st.m[0];
+      const float mu1 = st.m[1] == NEG_INF ? 0.f : st.m[1];
+      uint32_t pb[4][2];
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) {
+        const float p0 = fast_exp2(sacc[kb][0] - mu0), p1 = fast_exp2(sacc[kb][1] - mu1);
+        const float p2 = fast_exp2(sacc[kb][2] - mu0), p3 = fast_exp2(sacc[kb][3] - mu1);
+        st.l[0] += p0 + p2;
+        st.l[1] += p1 + p3;
+        pb[kb][0] = movmatrix_t(pack_bf16x2(p0, p1));
+        pb[kb][1] = movmatrix_t(pack_bf16x2(p2, p3));
+      }
+
+      // ---- O^T += V^T P^T ; V rows past seq_len are selected out
+      const bool boundary = tile_key0 + KT > sl;
+      uint32_t vm[4][2];
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) {
+        vm[kb][0] = vm[kb][1] = 0xffffffffu;
+        if (boundary) {
+          const int k0 = tile_key0 + 16 * kb + 2 * t4;
+          vm[kb][0] = (k0 < sl ? 0x0000ffffu : 0u) | (k0 + 1 < sl ? 0xffff0000u : 0u);
+          vm[kb][1] = (k0 + 8 < sl ? 0x0000ffffu : 0u) | (k0 + 9 < sl ? 0xffff0000u : 0u);
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
           const int j = lane >> 3;
-          const int key = kw + 16 * kb + (j >> 1) * 8 + (lane & 7);
+          const int key = 16 * kb + (j >> 1) * 8 + (lane & 7);
           const int ch = 2 * mt + (j & 1);
           const uint32_t addr = Vs + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
           uint32_t a0, a1, a2, a3;
           ldsm_x4_t(a0, a1, a2, a3, addr);
-          a0 &= vm_lo;
-          a1 &= vm_lo;
-          a2 &= vm_hi;
-          a3 &= vm_hi;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_bf16_16816(st.o[mt][nt], a0, a1, a2, a3, pb[kb][nt][0], pb[kb][nt][1]);
+          if (boundary) {
+            a0 &= vm[kb][0];
+            a1 &= vm[kb][0];
+            a2 &= vm[kb][1];
+            a3 &= vm[kb][1];
+          }
+          mma_bf16_16816(st.o[mt], a0, a1, a2, a3, pb[kb][0], pb[kb][1]);
         }
       }
 
-      // ---- Z^T += U_i^T P^T over rows of agent i; U rows < a_i or >= seq_len selected out
-      const int tile_key0 = tile * KT;
+      // ---- Z^T += U_i^T P^T over this warp's rows of agent i; U rows < a_i or >= seq_len selected out
       const bool lr_full = p.mode == LRKV_BASE_LR_SHARED && !boundary && a_max <= tile_key0;
-      const int n_pass = lr_full ? 1 : sg.n_ag;
-      for (int ag = 0; ag < n_pass; ++ag) {
+      const int pass_lo = lr_full ? 0 : ag_lo;
+      const int pass_hi = lr_full ? 0 : ag_hi;
+      for (int ag = pass_lo; ag <= pass_hi; ++ag) {
         const int a_i = lr_full ? 0 : a_sm[ag];
-        if (tile_key0 + KT <= a_i) continue;            // producer did not load this U tile
-        if (kbase + 32 <= a_i || kbase >= sl) continue;  // nothing of this warp's keys is adapted
+        if (tile_key0 + KT <= a_i) continue;  // producer did not load this U tile
         const int slot = p.mode == LRKV_BASE_SHARED ? ag : 0;
         const uint32_t ub = Us + slot * U_BYTES;
-        int nt_lo = 0, nt_hi = NT - 1;
-        if (!lr_full) {
-          const int r_first = (sg.i_lo + ag) * p.G - sg.row_lo;
-          const int r_last = r_first + p.G - 1;
-          nt_lo = r_first > 0 ? r_first / 8 : 0;
-          nt_hi = r_last / 8 < NT - 1 ? r_last / 8 : NT - 1;
-        }
+        const bool use = lr_full ? (my_agent >= 0) : (my_agent == ag);
 #pragma unroll
-        for (int kb = 0; kb < 2; ++kb) {
-          const int k16 = kbase + 16 * kb;
-          if (k16 + 16 <= a_i || k16 >= sl) continue;
+        for (int kb = 0; kb < 4; ++kb) {
+          const int k16 = tile_key0 + 16 * kb;
+          if (k16 + 16 <= a_i || k16 >= sl) continue;  // warp-uniform
           const int k0 = k16 + 2 * t4;
           const bool ok0 = k0 >= a_i && k0 < sl, ok1 = k0 + 1 >= a_i && k0 + 1 < sl;
           const bool ok8 = k0 + 8 >= a_i && k0 + 8 < sl, ok9 = k0 + 9 >= a_i && k0 + 9 < sl;
           const uint32_t um_lo = (ok0 ? 0x0000ffffu : 0u) | (ok1 ? 0xffff0000u : 0u);
           const uint32_t um_hi = (ok8 ? 0x0000ffffu : 0u) | (ok9 ? 0xffff0000u : 0u);
+          const uint32_t b0 = use ? pb[kb][0] : 0u, b1 = use ? pb[kb][1] : 0u;
 #pragma unroll
           for (int mz = 0; mz < MTZ; ++mz) {
             uint32_t a0, a1 = 0, a2, a3 = 0;
             if constexpr (RK == 8) {
-              const int key = kw + 16 * kb + ((lane >> 3) & 1) * 8 + (lane & 7);
+              const int key = 16 * kb + ((lane >> 3) & 1) * 8 + (lane & 7);
               ldsm_x2_t(a0, a2, ub + key * (RK * 2));
             } else {
               const int j = lane >> 3;
-              const int key = kw + 16 * kb + (j >> 1) * 8 + (lane & 7);
+              const int key = 16 * kb + (j >> 1) * 8 + (lane & 7);
               const int ch = 2 * mz + (j & 1);
               ldsm_x4_t(a0, a1, a2, a3, ub + key * (RK * 2) + ch * 16);
             }
@@ -568,13 +535,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
             a1 &= um_lo;
             a2 &= um_hi;
             a3 &= um_hi;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              if (nt < nt_lo || nt > nt_hi) continue;  // no row of this agent in this n-tile
-              const bool use = lr_full ? (my_agent[nt] >= 0) : (my_agent[nt] == ag);
-              const uint32_t b0 = use ? pb[kb][nt][0] : 0u, b1 = use ? pb[kb][nt][1] : 0u;
-              mma_bf16_16816(st.z[mz][nt], a0, a1, a2, a3, b0, b1);
-            }
+            mma_bf16_16816(st.z[mz], a0, a1, a2, a3, b0, b1);
           }
         }
       }
@@ -583,49 +544,22 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       if (lane == 0) mbar_arrive(&empty[my_stage]);
     }
 
-    // ---- reduce l over the lanes that share a row, then merge the warps:
-    // owner groups pairwise (same key half), then the two key halves.
+    // ---- reduce l over the lanes that share a row; chain the groups into record 0
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float v = st.l[nt][e];
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        st.l[nt][e] = v;
-      }
-    // a chain NOG-1 -> ... -> 1 -> 0 through one shared record per key half
+    for (int e = 0; e < 2; ++e) {
+      float v = st.l[e];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      st.l[e] = v;
+    }
     for (int src = NOG - 1; src >= 1; --src) {
-      if (og == src) store_state<D, NT, RK>(st, merge + kh * REC, g8, t4);
+      if (og == src) store_rows<D, RK>(st, merge, RP, rbase, g8, t4);
       named_bar_sync(1, CT);
-      if (og == src - 1) absorb_state<D, NT, RK>(st, merge + kh * REC, g8, t4);
+      if (og == src - 1) absorb_rows<D, RK>(st, merge, RP, rbase, g8, t4);
       named_bar_sync(1, CT);
     }
-    if (og == 0) store_state<D, NT, RK>(st, merge + kh * REC, g8, t4);
-    named_bar_sync(1, CT);
-
-    // ---- merge the two key halves into record 0
-    if (tid < RP) {
-      const float m0 = merge[tid], m1 = merge[REC + tid];
-      const float M = fmaxf(m0, m1);
-      const float s0 = m0 == NEG_INF ? 0.f : fast_exp2(m0 - M);
-      const float s1 = m1 == NEG_INF ? 0.f : fast_exp2(m1 - M);
-      scw[tid] = s0;
-      scw[RP + tid] = s1;
-      merge[RP + tid] = merge[RP + tid] * s0 + merge[REC + RP + tid] * s1;
-      merge[tid] = M;
-    }
-    named_bar_sync(1, CT);
-    for (int e4 = tid; e4 < RP * (D + RK) / 4; e4 += CT) {
-      const int e = e4 * 4;
-      const int row = e < RP * D ? e / D : (e - RP * D) / RK;
-      const float4 x0 = *reinterpret_cast<const float4*>(merge + 2 * RP + e);
-      const float4 x1 = *reinterpret_cast<const float4*>(merge + REC + 2 * RP + e);
-      const float s0 = scw[row], s1 = scw[RP + row];
-      *reinterpret_cast<float4*>(merge + 2 * RP + e) =
-          make_float4(x0.x * s0 + x1.x * s1, x0.y * s0 + x1.y * s1, x0.z * s0 + x1.z * s1, x0.w * s0 + x1.w * s1);
-    }
+    if (og == 0) store_rows<D, RK>(st, merge, RP, rbase, g8, t4);
     named_bar_sync(1, CT);
 
     // ---- publish or finish this item
@@ -742,47 +676,38 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   }
 }
 
-// Warp roles: warpgroup 0 is the producer (one warp issues the copies, its
-// register budget is cut to kProducerRegs), warpgroups 1..NG consume.  The
-// block is launched with THREADS x kLaunchRegs registers; the split
-// kProducerRegs x 128 + kConsumerRegs x 128 x NG must not exceed that total.
+// Warp roles: warps 0 .. kDecodeGroups*NT-1 consume, the last warp produces.
 template <int NT>
-struct Groups {
-  static constexpr int NG = NT <= 3 ? 2 : 1;  // 32 padded rows need the whole register file: one group
-  static constexpr int THREADS = (NG + 1) * 128;
+struct Roles {
+  static constexpr int CONSUMER_WARPS = kDecodeGroups * NT;
+  static constexpr int THREADS = (CONSUMER_WARPS + 1) * 32;
 };
-constexpr int kLaunchRegs = 168;     // 65536 / 384, rounded down to a multiple of 8
-constexpr int kProducerRegs = 32;
-constexpr int kConsumerRegs = 232;
-static_assert(kProducerRegs * 128 + kConsumerRegs * 256 <= kLaunchRegs * 384, "register split exceeds the launch");
 
 template <int D, int NT, int RK>
-__global__ void __launch_bounds__(Groups<NT>::THREADS, 1)
+__global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmU, const DecodeParams p) {
-  constexpr int NG = Groups<NT>::NG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const DecodeSmem lay = decode_smem_plan(D, NT, RK, p.n_u_slots, p.stages);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar_off);
   uint64_t* empty = full + p.stages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + p.stages);
+  volatile int* seq = reinterpret_cast<volatile int*>(empty + p.stages);
+  volatile int* abort_flag = seq + p.stages;
   int* bcast = const_cast<int*>(abort_flag) + 1;
   const int warp = threadIdx.x >> 5;
-  if (p.stages % decode_owner_groups(NT) != 0) {  // every stage must keep one owner group
-    if (threadIdx.x == 0) atomicOr(p.flags, LRKV_DEVFLAG_TIMEOUT);
-    return;
-  }
+  constexpr int PRODUCER = Roles<NT>::CONSUMER_WARPS;
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 2);  // the two warps of the pair that owns the tile
+      mbar_init(&empty[s], NT);  // the NT warps of the group that owns the tile
+      seq[s] = -1;
     }
     *abort_flag = 0;
     *bcast = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && (threadIdx.x & 31) == 0) {
+  if (warp == PRODUCER && (threadIdx.x & 31) == 0) {
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmU);
@@ -793,13 +718,11 @@ __global__ void __launch_bounds__(Groups<NT>::THREADS, 1)
   const long long C = gridDim.x;
   const long long t_begin = (long long)blockIdx.x * p.W / C;
   const long long t_end = (long long)(blockIdx.x + 1) * p.W / C;
-  if (warp < 4) {
-    if constexpr (NG == 2) setmaxnreg_dec<kProducerRegs>();
-    if (warp == 0)
-      decode_producer<D, RK>(p, &tmK, &tmV, &tmU, smem, lay.stage_bytes, full, empty, abort_flag, t_begin, t_end);
+  if (warp == PRODUCER) {
+    decode_producer<D, RK>(p, &tmK, &tmV, &tmU, smem, lay.stage_bytes, full, empty, seq, abort_flag, t_begin,
+                           t_end);
   } else {
-    if constexpr (NG == 2) setmaxnreg_inc<kConsumerRegs>();
-    decode_consumers<D, NT, RK, NG>(p, smem, lay, full, empty, abort_flag, bcast, t_begin, t_end);
+    decode_consumers<D, NT, RK>(p, smem, lay, full, empty, seq, abort_flag, bcast, t_begin, t_end);
   }
 }
 
@@ -815,7 +738,7 @@ lrkv_status launch_one(const DecodeParams& p, const void* tmK, const void* tmV, 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
-  cfg.blockDim = dim3(Groups<NT>::THREADS);
+  cfg.blockDim = dim3(Roles<NT>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

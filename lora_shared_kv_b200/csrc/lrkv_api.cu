@@ -197,15 +197,14 @@ lrkv_status plan_decode(const lrkv_problem* p, int max_seq_len, const DeviceInfo
     ms = n > ms ? n : ms;
   }
   pl->max_segs = ms;
-  // shared memory: as many stages as fit, a multiple of the owner groups (<= 8)
+  // shared memory: as many stages as fit (2..8)
   const int optin = dev.smem_optin > 0 ? dev.smem_optin : 232448;
-  const int nog = lrkv::decode_owner_groups(pl->NT);
   int stages = 8;
-  for (; stages >= nog; stages -= nog) {
+  for (; stages >= 2; --stages) {
     lrkv::DecodeSmem lay = lrkv::decode_smem_plan(p->head_dim, pl->NT, p->rank, pl->n_u_slots, stages);
     if (lay.total + 1024 <= optin) break;
   }
-  if (stages < nog || stages % nog != 0) return fail(LRKV_ERR_UNSUPPORTED, "decode tiles do not fit in shared memory");
+  if (stages < 2) return fail(LRKV_ERR_UNSUPPORTED, "decode tiles do not fit in shared memory");
   pl->stages = stages;
   pl->smem = lrkv::decode_smem_plan(p->head_dim, pl->NT, p->rank, pl->n_u_slots, stages).total + 1024;
   pl->tickets_off = lrkv::kWsHeaderBytes;

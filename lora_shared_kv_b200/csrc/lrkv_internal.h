@@ -52,9 +52,14 @@ struct DecodeParams {
   unsigned* flags;
 };
 
+// Consumer warp groups of the decode kernel.  Tile n of a CTA goes to group
+// n % kDecodeGroups and to ring stage n % stages; the warps of a group split
+// the query rows, eight each.
+constexpr int kDecodeGroups = 2;
+
 // Shared-memory plan of the decode kernel (bytes from a 1024-aligned base).
 struct DecodeSmem {
-  int stage_bytes, ring_bytes, q_off, merge_off, scw_off, a_off, bar_off, total;
+  int stage_bytes, ring_bytes, merge_off, scw_off, a_off, bar_off, total;
 };
 
 __host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
@@ -64,25 +69,16 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int D, int NT, int RK, in
   const int RP = NT * 8;
   s.stage_bytes = round_up(2 * kKeysPerTile * D * 2 + n_u_slots * kKeysPerTile * RK * 2, 1024);
   s.ring_bytes = stages * s.stage_bytes;
-  s.q_off = s.ring_bytes;
-  s.merge_off = s.q_off + round_up(RP * D * 2, 128);
+  s.merge_off = s.ring_bytes;
   const int rec = RP * (D + RK + 2) * 4;
-  s.scw_off = s.merge_off + 2 * rec;
+  s.scw_off = s.merge_off + rec;
   s.a_off = s.scw_off + 8 * RP * 4;
   s.bar_off = round_up(s.a_off + kMaxAgents * 4, 16);
-  s.total = s.bar_off + 2 * stages * 8 + 64;
+  s.total = s.bar_off + 2 * stages * 8 + stages * 4 + 64;
   return s;
 }
 
 inline size_t decode_record_floats(int NT, int D, int RK) { return (size_t)NT * 8 * (D + RK + 2); }
-
-// Consumer warps of the decode kernel form owner groups (pairs of warps);
-// tile n of a CTA goes to group n % groups and to ring stage n % stages.
-// The stage count must be a multiple of the group count so that every stage
-// always has the same owner: an mbarrier parity wait can only tell a phase
-// from the one just before it, so a group must never wait for use u+1 of a
-// stage while another group still holds use u.
-__host__ __device__ inline int decode_owner_groups(int NT) { return (NT <= 3 ? 2 : 1) * 2; }
 
 // Owner CTA of flattened tile t when W tiles are split evenly over C CTAs:
 // CTA c covers [c*W/C, (c+1)*W/C).
