@@ -311,6 +311,21 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   uint32_t phase = 0;
   int ntile = 0;  // tiles seen by this CTA so far (all groups)
 
+  // Per-lane byte offsets of the ldmatrix rows inside a 128B-swizzled K/V
+  // tile (64 keys x 64 dims per half): 16-byte chunk c of key row k sits at
+  // chunk c ^ (k & 7).  koff[i] serves k-steps with (2 ks) & 7 == 2 i (K
+  // operand), voff[i] serves m-tiles with (2 mt) & 7 == 2 i (V^T operand);
+  // the key block (2048 B) and the 64-dim half (8192 B) are added as constants.
+  uint32_t koff[4], voff[4];
+  {
+    const int j = lane >> 3, r8 = lane & 7;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      koff[i] = ((j & 1) * 8 + r8) * 128 + ((((2 * i) + (j >> 1)) ^ r8) << 4);
+      voff[i] = ((j >> 1) * 8 + r8) * 128 + ((((2 * i) + (j & 1)) ^ r8) << 4);
+    }
+  }
+
   for (long long t = t_begin; t < t_end;) {
     Seg sg = make_seg(p, t, t_end, tid == 0);
     t += sg.hi - sg.lo;
@@ -394,14 +409,11 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
         for (int e = 0; e < 4; ++e) sacc[kb][e] = 0.f;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
+        const uint32_t kb_base = Ks + koff[ks & 3] + (ks >> 2) * (KT * 128);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
-          const int j = lane >> 3;
-          const int key = 16 * kb + (j & 1) * 8 + (lane & 7);
-          const int ch = ks * 2 + (j >> 1);
-          const uint32_t addr = Ks + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
           uint32_t a0, a1, a2, a3;
-          ldsm_x4(a0, a1, a2, a3, addr);
+          ldsm_x4(a0, a1, a2, a3, kb_base + kb * (16 * 128));
           mma_bf16_16816(sacc[kb], a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
         }
       }
@@ -411,15 +423,20 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       // more than 2^8 (log2 units): probabilities then stay <= 2^8 and the
       // accumulators need rescaling only on those rare tiles.  The result is
       // exact either way, since numerator and denominator share the reference.
+      const bool boundary = tile_key0 + KT > sl;
       float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
-        const bool va = tile_key0 + 16 * kb + g8 < sl;
-        const bool vb = tile_key0 + 16 * kb + g8 + 8 < sl;
-        sacc[kb][0] = va ? sacc[kb][0] * p.scale_log2 : NEG_INF;
-        sacc[kb][1] = va ? sacc[kb][1] * p.scale_log2 : NEG_INF;
-        sacc[kb][2] = vb ? sacc[kb][2] * p.scale_log2 : NEG_INF;
-        sacc[kb][3] = vb ? sacc[kb][3] * p.scale_log2 : NEG_INF;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[kb][e] *= p.scale_log2;
+        if (boundary) {  // keys at or past seq_len are selected out
+          const bool va = tile_key0 + 16 * kb + g8 < sl;
+          const bool vb = tile_key0 + 16 * kb + g8 + 8 < sl;
+          sacc[kb][0] = va ? sacc[kb][0] : NEG_INF;
+          sacc[kb][1] = va ? sacc[kb][1] : NEG_INF;
+          sacc[kb][2] = vb ? sacc[kb][2] : NEG_INF;
+          sacc[kb][3] = vb ? sacc[kb][3] : NEG_INF;
+        }
         mx0 = fmaxf(mx0, fmaxf(sacc[kb][0], sacc[kb][2]));
         mx1 = fmaxf(mx1, fmaxf(sacc[kb][1], sacc[kb][3]));
       }
@@ -468,7 +485,6 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       }
 
       // ---- O^T += V^T P^T ; V rows past seq_len are selected out
-      const bool boundary = tile_key0 + KT > sl;
       uint32_t vm[4][2];
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
@@ -481,14 +497,11 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
+        const uint32_t mt_base = Vs + voff[mt & 3] + (mt >> 2) * (KT * 128);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
-          const int j = lane >> 3;
-          const int key = 16 * kb + (j >> 1) * 8 + (lane & 7);
-          const int ch = 2 * mt + (j & 1);
-          const uint32_t addr = Vs + (ch >> 3) * (KT * 128) + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(a0, a1, a2, a3, addr);
+          ldsm_x4_t(a0, a1, a2, a3, mt_base + kb * (16 * 128));
           if (boundary) {
             a0 &= vm[kb][0];
             a1 &= vm[kb][0];
