@@ -478,10 +478,12 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       for (int kb = 0; kb < 4; ++kb) {
         const float p0 = fast_exp2(sacc[kb][0] - mu0), p1 = fast_exp2(sacc[kb][1] - mu1);
         const float p2 = fast_exp2(sacc[kb][2] - mu0), p3 = fast_exp2(sacc[kb][3] - mu1);
-        st.l[0] += p0 + p2;
-        st.l[1] += p1 + p3;
-        pb[kb][0] = movmatrix_t(pack_bf16x2(p0, p1));
-        pb[kb][1] = movmatrix_t(pack_bf16x2(p2, p3));
+        const uint32_t w01 = pack_bf16x2(p0, p1), w23 = pack_bf16x2(p2, p3);
+        // the row sums of exactly the bf16 weights the value MMA uses
+        st.l[0] += __uint_as_float(w01 << 16) + __uint_as_float(w23 << 16);
+        st.l[1] += __uint_as_float(w01 & 0xffff0000u) + __uint_as_float(w23 & 0xffff0000u);
+        pb[kb][0] = movmatrix_t(w01);
+        pb[kb][1] = movmatrix_t(w23);
       }
 
       // ---- O^T += V^T P^T ; V rows past seq_len are selected out

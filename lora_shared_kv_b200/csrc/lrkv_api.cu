@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "lrkv_internal.h"
+#include "prefill.h"
 
 namespace {
 
@@ -376,19 +377,95 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
 }
 
 size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T) {
-  (void)p;
-  (void)ctx_len;
-  (void)T;
-  return 0;
+  if (check_problem(p) != LRKV_OK || ctx_len < 0 || T < 0) return 0;
+  return lrkv::kWsHeaderBytes;  // device-side flags only
 }
 
 lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv, int32_t session,
                                     int32_t ctx_len, int32_t T, const lrkv_u_view* u, const void* b,
                                     const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
                                     size_t workspace_bytes, lrkv_stream_t stream) {
-  (void)p; (void)q; (void)kv; (void)session; (void)ctx_len; (void)T; (void)u; (void)b;
-  (void)alora_offsets; (void)out; (void)out_dtype; (void)workspace; (void)workspace_bytes; (void)stream;
-  return fail(LRKV_ERR_UNSUPPORTED, "prefill chunk not built yet");
+  lrkv_status s = check_problem(p);
+  if (s != LRKV_OK) return s;
+  if (!q || !b || !out || !workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "q, b, out and workspace must not be NULL");
+  if (!aligned16(q) || !aligned16(b) || !aligned16(out) || !aligned16(workspace))
+    return fail(LRKV_ERR_MISALIGNED, "q, b, out and workspace must be 16-byte aligned");
+  if (out_dtype != LRKV_BF16 && out_dtype != LRKV_F32) return fail(LRKV_ERR_INVALID_ARGUMENT, "out_dtype %d", out_dtype);
+  if (ctx_len < 0 || T < 0 || session < 0 || session >= p->num_sessions)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "need ctx_len >= 0, T >= 0 and 0 <= session < num_sessions");
+  const int G = p->num_q_heads / p->num_kv_heads;
+  if (128 % G != 0) return fail(LRKV_ERR_UNSUPPORTED, "prefill needs Hq/Hkv to divide 128 (got %d)", G);
+  if (p->rank == 8) return fail(LRKV_ERR_UNSUPPORTED, "prefill supports rank 16 and 32");
+  const long long Ltot = (long long)ctx_len + T;
+  if (Ltot > 0x7fffffffLL) return fail(LRKV_ERR_INVALID_ARGUMENT, "ctx_len + T overflows");
+  if ((s = check_kv(kv, p)) != LRKV_OK) return s;
+  if ((s = check_u(u, p, (int)Ltot)) != LRKV_OK) return s;
+  if (workspace_bytes < (size_t)lrkv::kWsHeaderBytes) return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %d bytes", workspace_bytes, lrkv::kWsHeaderBytes);
+  if (T == 0) return LRKV_OK;
+  DeviceInfo dev;
+  if ((s = device_info(&dev)) != LRKV_OK) return s;
+  const int D = p->head_dim, RK = p->rank;
+  if (lrkv::prefill_smem_bytes(D, RK) > dev.smem_optin) return fail(LRKV_ERR_UNSUPPORTED, "prefill tiles do not fit in shared memory");
+
+  alignas(64) CUtensorMap maps[5];
+  const int TM = 128 / G;
+  {  // Q [N, T, Hq, d]: box = 64 dims x G heads x TM tokens of one agent
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p->num_q_heads, (uint64_t)T, (uint64_t)p->num_agents};
+    const int64_t str[3] = {D, (int64_t)p->num_q_heads * D, (int64_t)T * p->num_q_heads * D};
+    const uint32_t box[4] = {64, (uint32_t)G, (uint32_t)TM, 1};
+    if ((s = make_map4(&maps[0], q, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "Q")) != LRKV_OK) return s;
+  }
+  if (kv->page_table) {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)kv->page_size, (uint64_t)p->num_kv_heads, (uint64_t)kv->num_pages};
+    const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_page};
+    const uint32_t box[4] = {64, 64, 1, 1};
+    if ((s = make_map4(&maps[1], kv->k, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "K pages")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[2], kv->v, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "V pages")) != LRKV_OK) return s;
+  } else {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Ltot, (uint64_t)p->num_kv_heads, (uint64_t)p->num_sessions};
+    const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_session};
+    const uint32_t box[4] = {64, 128, 1, 1};
+    if ((s = make_map4(&maps[1], kv->k, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "K")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[2], kv->v, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "V")) != LRKV_OK) return s;
+  }
+  {
+    const int slots = p->mode == LRKV_BASE_SHARED ? p->num_agents : 1;
+    const uint64_t dims[4] = {(uint64_t)RK, (uint64_t)Ltot, (uint64_t)slots, (uint64_t)p->num_sessions};
+    const int64_t str[3] = {u->stride_token, u->stride_agent, u->stride_session};
+    const uint32_t box[4] = {(uint32_t)RK, 128, 1, 1};
+    const CUtensorMapSwizzle sw = RK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    if ((s = make_map4(&maps[3], u->u, dims, str, box, sw, "U")) != LRKV_OK) return s;
+  }
+  {  // B [N, r, Hkv*d]: box = d dims of one KV head x r ranks of one agent
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p->num_kv_heads, (uint64_t)RK, (uint64_t)p->num_agents};
+    const int64_t str[3] = {D, (int64_t)p->num_kv_heads * D, (int64_t)RK * p->num_kv_heads * D};
+    const uint32_t box[4] = {(uint32_t)D, 1, (uint32_t)RK, 1};
+    if ((s = make_map4(&maps[4], b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE, "B")) != LRKV_OK) return s;
+  }
+  lrkv::PrefillParams pp = {};
+  pp.offsets = alora_offsets;
+  pp.page_table = kv->page_table;
+  pp.pt_stride = kv->page_table_stride;
+  pp.num_pages = kv->page_table ? kv->num_pages : 0;
+  pp.out = out;
+  pp.out_f32 = out_dtype == LRKV_F32;
+  pp.N = p->num_agents;
+  pp.Hq = p->num_q_heads;
+  pp.Hkv = p->num_kv_heads;
+  pp.G = G;
+  pp.T = T;
+  pp.L0 = ctx_len;
+  pp.session = session;
+  pp.mode = p->mode;
+  pp.n_tb = (T + TM - 1) / TM;
+  pp.scale_log2 = scale_of(p) * 1.4426950408889634f;
+  pp.flags = static_cast<unsigned*>(workspace);
+  const long long grid = (long long)p->num_kv_heads * p->num_agents * pp.n_tb;
+  if (grid > 0x7fffffffLL) return fail(LRKV_ERR_UNSUPPORTED, "too many prefill tiles");
+  lrkv::PrefillMaps pm = {maps};
+  s = lrkv::launch_prefill(pp, pm, D, RK, (int)grid, stream);
+  if (s != LRKV_OK) return fail(s, "prefill launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+  return LRKV_OK;
 }
 
 }  // extern "C"

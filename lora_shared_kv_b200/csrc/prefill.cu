@@ -1,0 +1,464 @@
+// Prefill-chunk attention over the shared base cache with per-agent low-rank
+// value caches, on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+// For agent i, query head h (KV head g = h / G) and chunk row j at absolute
+// position L0 + j:
+//     o = ( P V_base,g + (P Umask_i) B_i,g ) / l,   P = exp(q K_base,g^T * scale - m),  keys t <= L0 + j
+// Eq. 12 of "LRAgent: Efficient KV Cache Sharing for Multi-LoRA LLM Agents"
+// (Pith review, "What carries the argument"): the rank-r values are
+// accumulated next to O as Z = P Umask_i and B_i is applied once per row in
+// the epilogue.  Umask_i drops U rows before the agent's aLoRA offset ("RoleKV",
+// "What it does").
+//
+// One CTA computes one 128-row tile: one agent, one KV head, 128/G chunk
+// tokens x the G query heads that share the KV head, so every K/V block
+// loaded serves all of them.  Roles:
+//   warp 0        TMA producer: Q tile and B_i,g once, then K, V and U blocks
+//                 of 128 keys into a two-stage ring.
+//   warp 1        TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into a
+//                 double-buffered S in TMEM; then O += P_j V_j and
+//                 Z += P_j U_j with P_j read from TMEM (it overwrites S_j).
+//   warps 4..7    softmax and epilogue, one row per thread (TMEM lane = row):
+//                 row max/sum need no shuffles; the reference max moves only
+//                 when a block exceeds it by 2^8, and only then is O rescaled
+//                 in TMEM.
+#include <float.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "prefill.h"
+
+namespace lrkv {
+
+namespace {
+
+constexpr int BM = 128;   // rows per tile (TMEM lanes)
+constexpr int BN = 128;   // keys per block
+constexpr int STAGES = 2;
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 512;
+
+template <int D, int RK>
+struct PrefillLayout {
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int B_BYTES = RK * D * 2;
+  static constexpr int K_BYTES = BN * D * 2;
+  static constexpr int U_BYTES = BN * RK * 2;
+  static constexpr int STAGE_BYTES = 2 * K_BYTES + U_BYTES;
+  static constexpr int Q_OFF = 0;
+  static constexpr int B_OFF = Q_OFF + Q_BYTES;
+  static constexpr int RING_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
+  static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE_BYTES;
+  static constexpr int TOTAL = BAR_OFF + 256;
+  // TMEM columns
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_Z = 2 * BN + D;
+  static_assert(2 * BN + D + RK <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t kv_full[STAGES];
+  uint64_t kv_empty[STAGES];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_ready;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  uintptr_t v = reinterpret_cast<uintptr_t>(p);
+  return reinterpret_cast<uint8_t*>((v + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+template <int D, int RK>
+__global__ void __launch_bounds__(THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmU,
+                   const __grid_constant__ CUtensorMap tmB, const PrefillParams p) {
+  using Lay = PrefillLayout<D, RK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  Bars* bars = reinterpret_cast<Bars*>(smem + Lay::BAR_OFF);
+  volatile int* abort_flag = &bars->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- tile coordinates: blockIdx.x = (g * N + agent) * n_tb + tb
+  const int n_tb = p.n_tb;
+  const int tb = blockIdx.x % n_tb;
+  const int ga = blockIdx.x / n_tb;
+  const int agent = ga % p.N;
+  const int g = ga / p.N;
+  const int TM = BM / p.G;                // chunk tokens per tile
+  const int j0 = tb * TM;                 // first chunk row of the tile
+  const int rows_tok = min(TM, p.T - j0); // valid chunk tokens in the tile
+  const int key_end = p.L0 + j0 + rows_tok;         // keys [0, key_end) are visible to some row
+  const int nb = (key_end + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->p_full[b], 4);
+    }
+    mbar_init(&bars->o_ready, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmU);
+    tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  pdl_launch_dependents();
+  const uint32_t tmem = bars->tmem_base;
+
+  int a_i = 0;
+  if (p.offsets) {
+    a_i = __ldg(p.offsets + agent);
+    if (a_i < 0) {
+      if (threadIdx.x == 0) atomicOr(p.flags, LRKV_DEVFLAG_OFFSET);
+      a_i = 0;
+    }
+  }
+  const int u_slot = p.mode == LRKV_BASE_SHARED ? agent : 0;
+
+  if (warp == 0) {
+    // ======================= producer =======================
+    if (lane == 0) {
+      const uint64_t pol_kv = policy_evict_last();  // K/V blocks are reused by the other tiles of the KV head
+      const uint64_t pol_q = policy_evict_first();
+      mbar_arrive_expect_tx(&bars->q_full, Lay::Q_BYTES + Lay::B_BYTES);
+#pragma unroll
+      for (int hh = 0; hh < D / 64; ++hh)
+        tma_load_4d(smem + Lay::Q_OFF + hh * (BM * 128), &tmQ, &bars->q_full, hh * 64, g * p.G, j0, agent, pol_q);
+      tma_load_4d(smem + Lay::B_OFF, &tmB, &bars->q_full, 0, g, 0, agent, pol_q);
+      int n_pages = 0;
+      if (p.page_table) n_pages = (p.L0 + p.T + 63) / 64;
+      int issued = 0;
+      for (int jb = 0; jb < nb; ++jb) {
+        const int st = jb % STAGES;
+        const uint32_t ph = (jb / STAGES) & 1;
+        if (!mbar_wait_bounded(&bars->kv_empty[st], ph ^ 1, abort_flag, p.flags)) break;
+        issued = jb + 1;
+        const bool need_u = jb * BN + BN > a_i;
+        uint8_t* Ks = smem + Lay::RING_OFF + st * Lay::STAGE_BYTES;
+        uint8_t* Vs = Ks + Lay::K_BYTES;
+        uint8_t* Us = Vs + Lay::K_BYTES;
+        mbar_arrive_expect_tx(&bars->kv_full[st], 2 * Lay::K_BYTES + (need_u ? Lay::U_BYTES : 0));
+        if (!p.page_table) {
+#pragma unroll
+          for (int hh = 0; hh < D / 64; ++hh) {
+            tma_load_4d(Ks + hh * (BN * 128), &tmK, &bars->kv_full[st], hh * 64, jb * BN, g, p.session, pol_kv);
+            tma_load_4d(Vs + hh * (BN * 128), &tmV, &bars->kv_full[st], hh * 64, jb * BN, g, p.session, pol_kv);
+          }
+        } else {
+#pragma unroll
+          for (int pg = 0; pg < BN / 64; ++pg) {
+            int lp = jb * (BN / 64) + pg;
+            if (lp >= n_pages) lp = 0;  // past the chunk: any valid page (masked out below)
+            int phys = __ldg(p.page_table + (size_t)p.session * p.pt_stride + lp);
+            if (phys < 0 || phys >= p.num_pages) {
+              atomicOr(p.flags, LRKV_DEVFLAG_PAGE);
+              phys = 0;
+            }
+#pragma unroll
+            for (int hh = 0; hh < D / 64; ++hh) {
+              tma_load_4d(Ks + hh * (BN * 128) + pg * (64 * 128), &tmK, &bars->kv_full[st], hh * 64, 0, g, phys,
+                          pol_kv);
+              tma_load_4d(Vs + hh * (BN * 128) + pg * (64 * 128), &tmV, &bars->kv_full[st], hh * 64, 0, g, phys,
+                          pol_kv);
+            }
+          }
+        }
+        if (need_u) tma_load_4d(Us, &tmU, &bars->kv_full[st], 0, jb * BN, u_slot, p.session, pol_kv);
+      }
+      if (*abort_flag) {
+        // let every copy this CTA issued land before the CTA can exit
+        uint32_t spins = 0;
+        while (!mbar_try_wait(&bars->q_full, 0) && ++spins < kSpinCap) {
+        }
+        for (int blk = issued > STAGES ? issued - STAGES : 0; blk < issued; ++blk) {
+          spins = 0;
+          while (!mbar_try_wait(&bars->kv_full[blk % STAGES], (blk / STAGES) & 1) && ++spins < kSpinCap) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    constexpr uint32_t ID_QK = umma_idesc_bf16(BM, BN, 0, 0);
+    constexpr uint32_t ID_PV = umma_idesc_bf16(BM, D, 0, 1);
+    constexpr uint32_t ID_PZ = umma_idesc_bf16(BM, RK, 0, 1);
+    constexpr uint32_t U_LAYOUT = RK == 32 ? 4u : 6u;       // 64B / 32B swizzle, rows of RK bf16
+    constexpr uint32_t U_SBO = 8 * RK * 2;                  // eight key rows
+    const uint32_t q_base = smem_u32(smem + Lay::Q_OFF);
+    bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, p.flags);
+    bool z_started = false;
+    for (int jb = 0; jb <= nb && ok; ++jb) {
+      if (jb < nb) {
+        const int st = jb % STAGES;
+        ok = mbar_wait_bounded(&bars->kv_full[st], (jb / STAGES) & 1, abort_flag, p.flags);
+        if (!ok) break;
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(smem + Lay::RING_OFF + st * Lay::STAGE_BYTES);
+          const uint32_t d_s = tmem + (jb & 1 ? Lay::COL_S1 : Lay::COL_S0);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
+            const uint64_t a = umma_desc(q_base + off, 16, 1024, 2);
+            const uint64_t b = umma_desc(k_base + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024, 2);
+            umma_ss(d_s, a, b, ID_QK, ks > 0);
+          }
+          umma_commit(&bars->s_full[jb & 1]);
+        }
+        __syncwarp();
+      }
+      if (jb >= 1) {
+        const int j = jb - 1;
+        const int st = j % STAGES;
+        ok = mbar_wait_bounded(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag, p.flags);
+        if (!ok) break;
+        const bool u_used = j * BN + BN > a_i;
+        uint8_t* Us = smem + Lay::RING_OFF + st * Lay::STAGE_BYTES + 2 * Lay::K_BYTES;
+        if (u_used && j * BN < a_i) {
+          // the block holding a_i: rows before the offset are removed (zero-filled) before the MMA reads them
+          const int nz = a_i - j * BN;  // rows [0, nz)
+          uint4* z4 = reinterpret_cast<uint4*>(Us);
+          const int n16 = nz * RK * 2 / 16;
+          for (int x = lane; x < n16; x += 32) z4[x] = make_uint4(0, 0, 0, 0);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(smem + Lay::RING_OFF + st * Lay::STAGE_BYTES + Lay::K_BYTES);
+          const uint32_t u_base = smem_u32(Us);
+          const uint32_t a_p = tmem + (j & 1 ? Lay::COL_S1 : Lay::COL_S0);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t b = umma_desc(v_base + kk * 2048, BN * 128, 1024, 2);
+            umma_ts(tmem + Lay::COL_O, a_p + kk * 8, b, ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (u_used) {
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              const uint64_t b = umma_desc(u_base + kk * (16 * RK * 2), 16, U_SBO, U_LAYOUT);
+              umma_ts(tmem + Lay::COL_Z, a_p + kk * 8, b, ID_PZ, (z_started || kk > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&bars->kv_empty[st]);
+          umma_commit(&bars->o_ready);
+        }
+        if (u_used) z_started = true;
+        __syncwarp();
+      }
+    }
+  } else if (warp >= 4) {
+    // ======================= softmax + epilogue =======================
+    const int row = threadIdx.x - 128;         // TMEM lane and S/O row
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    const int jj = row / p.G, hh = row % p.G;
+    const int token = j0 + jj;
+    const int limit = p.L0 + token;            // last visible key of this row
+    const float NEG_INF = -INFINITY;
+    float m_ref = NEG_INF, l = 0.f;
+    bool ok = true;
+    for (int jb = 0; jb < nb && ok; ++jb) {
+      ok = mbar_wait_bounded(&bars->s_full[jb & 1], (jb >> 1) & 1, abort_flag, p.flags);
+      tc_fence_after();
+      const uint32_t s_col = jb & 1 ? Lay::COL_S1 : Lay::COL_S0;
+      float x[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tmem + lane_addr + s_col + c * 32, reinterpret_cast<uint32_t*>(x) + c * 32);
+      tmem_wait_ld();
+      const int key0 = jb * BN;
+      const bool diag = key0 + BN - 1 > p.L0 + j0;  // some key of the block is past some row's limit
+      float mx = NEG_INF;
+#pragma unroll
+      for (int cc = 0; cc < BN; ++cc) {
+        float v = x[cc] * p.scale_log2;
+        if (diag) v = key0 + cc <= limit ? v : NEG_INF;
+        x[cc] = v;
+        mx = fmaxf(mx, v);
+      }
+      const bool need = mx > m_ref + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = fmaxf(m_ref, mx);
+        const float alpha = m_new == NEG_INF ? 1.f : fast_exp2(m_ref - m_new);
+        if (jb > 0) {
+          // O and Z hold the blocks before this one: rescale them in TMEM once PV_{jb-1} is done
+          ok = mbar_wait_bounded(&bars->o_ready, (jb - 1) & 1, abort_flag, p.flags);
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < (D + RK) / 32; ++c) {
+            uint32_t r[32];
+            const uint32_t col = Lay::COL_O + c * 32;
+            tmem_ld32(tmem + lane_addr + col, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tmem + lane_addr + col, r);
+          }
+          if (RK % 32 != 0) {  // RK = 16: the last 16 columns (the load overlaps the chunk just stored)
+            tmem_wait_st();
+            uint32_t r[32];
+            const uint32_t col = Lay::COL_O + ((D + RK) / 32) * 32 - 16;
+            tmem_ld32(tmem + lane_addr + col, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 16; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tmem + lane_addr + col, r);
+          }
+          tmem_wait_st();
+        }
+        l *= alpha;
+        m_ref = m_new;
+      }
+      const float mu = m_ref == NEG_INF ? 0.f : m_ref;
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int cc = 0; cc < BN / 2; ++cc) {
+        const float p0 = fast_exp2(x[2 * cc] - mu), p1 = fast_exp2(x[2 * cc + 1] - mu);
+        pk[cc] = pack_bf16x2(p0, p1);
+        l += bf16_lo(pk[cc]) + bf16_hi(pk[cc]);  // the row sum of exactly the weights the MMA uses
+      }
+#pragma unroll
+      for (int c = 0; c < BN / 64; ++c) tmem_st32(tmem + lane_addr + s_col + c * 32, pk + c * 32);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[jb & 1]);
+    }
+    // ---- epilogue: out = (O + Z B_i,g) / l
+    if (ok) ok = mbar_wait_bounded(&bars->o_ready, (nb - 1) & 1, abort_flag, p.flags);
+    tc_fence_after();
+    const bool z_used = a_i < key_end;  // some block accumulated Z
+    float z[RK];
+    {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_addr + Lay::COL_Z - (RK == 16 ? 16 : 0), r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < RK; ++k) z[k] = z_used ? __uint_as_float(r[(RK == 16 ? 16 : 0) + k]) : 0.f;
+    }
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    const bool write = token < p.T && ok;
+    const int h = g * p.G + hh;
+    const uint16_t* bs = reinterpret_cast<const uint16_t*>(smem + Lay::B_OFF);
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_addr + Lay::COL_O + c * 32, r);
+      tmem_wait_ld();
+      float acc[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) acc[e] = __uint_as_float(r[e]);
+#pragma unroll
+      for (int k = 0; k < RK; ++k) {
+        const uint4* brow = reinterpret_cast<const uint4*>(bs + k * D + c * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 bv = brow[q4];
+          const uint32_t w4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            acc[q4 * 8 + 2 * u] = fmaf(z[k], bf16_lo(w4[u]), acc[q4 * 8 + 2 * u]);
+            acc[q4 * 8 + 2 * u + 1] = fmaf(z[k], bf16_hi(w4[u]), acc[q4 * 8 + 2 * u + 1]);
+          }
+        }
+      }
+      if (write) {
+        const size_t oi = (((size_t)agent * p.T + token) * p.Hq + h) * D + c * 32;
+        if (p.out_f32) {
+          float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(p.out) + oi);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            o4[q4] = make_float4(acc[4 * q4] * inv_l, acc[4 * q4 + 1] * inv_l, acc[4 * q4 + 2] * inv_l,
+                                 acc[4 * q4 + 3] * inv_l);
+        } else {
+          uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + oi);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            o4[q4] = make_uint4(pack_bf16x2(acc[8 * q4] * inv_l, acc[8 * q4 + 1] * inv_l),
+                                pack_bf16x2(acc[8 * q4 + 2] * inv_l, acc[8 * q4 + 3] * inv_l),
+                                pack_bf16x2(acc[8 * q4 + 4] * inv_l, acc[8 * q4 + 5] * inv_l),
+                                pack_bf16x2(acc[8 * q4 + 6] * inv_l, acc[8 * q4 + 7] * inv_l));
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  // ---- teardown: every TMEM reader is done before the owner frees it
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int D, int RK>
+lrkv_status launch_t(const PrefillParams& p, const PrefillMaps& m, int grid, cudaStream_t stream) {
+  using Lay = PrefillLayout<D, RK>;
+  auto kern = prefill_kernel<D, RK>;
+  const int smem = Lay::TOTAL + 1024;
+  static int configured = 0;
+  if (configured < smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return LRKV_ERR_CUDA;
+    configured = smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const CUtensorMap* t = static_cast<const CUtensorMap*>(m.maps);
+  if (cudaLaunchKernelEx(&cfg, kern, t[0], t[1], t[2], t[3], t[4], p) != cudaSuccess) return LRKV_ERR_CUDA;
+  return LRKV_OK;
+}
+
+}  // namespace
+
+int prefill_smem_bytes(int D, int RK) {
+  if (D == 128 && RK == 32) return PrefillLayout<128, 32>::TOTAL + 1024;
+  if (D == 128 && RK == 16) return PrefillLayout<128, 16>::TOTAL + 1024;
+  if (D == 64 && RK == 32) return PrefillLayout<64, 32>::TOTAL + 1024;
+  if (D == 64 && RK == 16) return PrefillLayout<64, 16>::TOTAL + 1024;
+  return -1;
+}
+
+lrkv_status launch_prefill(const PrefillParams& p, const PrefillMaps& m, int D, int RK, int grid, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 128 && RK == 32) return launch_t<128, 32>(p, m, grid, st);
+  if (D == 128 && RK == 16) return launch_t<128, 16>(p, m, grid, st);
+  if (D == 64 && RK == 32) return launch_t<64, 32>(p, m, grid, st);
+  if (D == 64 && RK == 16) return launch_t<64, 16>(p, m, grid, st);
+  return LRKV_ERR_UNSUPPORTED;
+}
+
+}  // namespace lrkv

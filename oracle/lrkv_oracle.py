@@ -216,14 +216,15 @@ def decode(q, k, v, u, b, offsets, seq_lens, mode=BASE_SHARED, scale=None,
     return out
 
 
-def prefill_chunk(q, k, v, u, b, offsets, ctx_len, mode=BASE_SHARED, scale=None):
+def prefill_chunk(q, k, v, u, b, offsets, ctx_len, mode=BASE_SHARED, scale=None, rows=None):
     """Causal attention of a chunk of T new rows per agent over one session.
 
     q [N, T, Hq, d]; k, v [Hkv, L0 + T, d] (the chunk's own base K/V already at
     rows [L0, L0 + T)); u [N_U, L0 + T, r] (chunk rows already appended);
     b [N, r, Hkv * d]; offsets [N] (or None); ctx_len = L0.
     Row j of agent i sits at absolute position L0 + j and sees keys t <= L0 + j.
-    Returns float64 [N, T, Hq, d].
+    Returns float64 [N, T, Hq, d]; with ``rows`` (chunk row indices) only those
+    rows are computed and the others are NaN.
     """
     q = to_f64(q)
     kk = to_f64(k)
@@ -237,15 +238,16 @@ def prefill_chunk(q, k, v, u, b, offsets, ctx_len, mode=BASE_SHARED, scale=None)
     Ltot = L0 + T
     sc = _scale(d, scale)
     offs = np.zeros(N, dtype=np.int64) if offsets is None else np.asarray(to_f64(offsets), dtype=np.int64)
-    visible = L0 + np.arange(T) + 1
-    out = np.empty((N, T, Hq, d), dtype=np.float64)
+    sel = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    visible = L0 + sel + 1
+    out = np.full((N, T, Hq, d), np.nan)
     for i in range(N):
         u_i = uu[i if mode == BASE_SHARED else 0, :Ltot]
         umask = masked_lr_cache(u_i, offs[i])
         v_i = agent_value_cache(vv[:, :Ltot], umask, b[i])
         for h in range(Hq):
             g = h // G
-            out[i, :, h] = attention_rows(q[i, :, h], kk[g, :Ltot], v_i[g], visible, sc)
+            out[i, sel, h] = attention_rows(q[i, sel, h], kk[g, :Ltot], v_i[g], visible, sc)
     return out
 
 
