@@ -184,6 +184,30 @@ class DecodeRunner:
         return decode_layer_bytes(self.cfg, self.inp.offsets.cpu())
 
 
+# ---------------------------------------------------------------------------
+# ranks: one process per GPU, each with its own sessions (weak scaling)
+# ---------------------------------------------------------------------------
+
+def rank_seed_offset(rank: int) -> int:
+    """Every rank draws its own sessions: the seed moves by a prime per rank."""
+    return 7919 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """The slowest rank's time (a timing reduction only, never on the data path)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job units per second: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
 def _timed(fn, steps, warmup, sync_all):
     for _ in range(warmup):
         fn()
@@ -337,21 +361,16 @@ def main():
         def sync_all():
             torch.cuda.synchronize()
 
-    runner = DecodeRunner(cfg, dev, seed_offset=7919 * rank)
+    runner = DecodeRunner(cfg, dev, seed_offset=rank_seed_offset(rank))
     runner.capture()
     clocks = ClockSampler(local)
     clocks.start()
     sync_all()
     ms = _timed(runner.step, args.steps, args.warmup, sync_all)
     ck = clocks.stop()
-    ms_step = ms / args.steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(ms / args.steps, dev)
     queries = cfg.queries_per_step * world
-    value = queries / (ms_step * 1e-3)
+    value = job_throughput(cfg.queries_per_step, world, ms_step)
 
     hbm, _, _, peak_src = _peaks()
     lb = runner.layer_bytes()
@@ -365,13 +384,9 @@ def main():
     e2e = None
     if not args.no_e2e:
         e_ms, hb, db = run_e2e(runner, max(10, args.steps // 10), args.warmup, sync_all)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": queries / (e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db,
-               "ms_per_step": e_ms}
+        e_ms = max_over_ranks(e_ms, dev)
+        e2e = {"value": job_throughput(cfg.queries_per_step, world, e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "ms_per_step": e_ms}
 
     prefill = None
     if not args.no_prefill and rank == 0:

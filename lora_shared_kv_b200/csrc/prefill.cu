@@ -13,8 +13,9 @@
 // One CTA computes one 128-row tile: one agent, one KV head, 128/G chunk
 // tokens x the G query heads that share the KV head, so every K/V block
 // loaded serves all of them.  Roles:
-//   warp 0        TMA producer: Q tile and B_i,g once, then K, V and U blocks
-//                 of 128 keys into a two-stage ring.
+//   warp 0        TMA producer: Q tile and B_i,g once, then 128-key blocks of
+//                 K into a 3-stage ring (a stage frees as soon as its S is
+//                 computed) and of V and U into a 2-stage ring.
 //   warp 1        TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into a
 //                 double-buffered S in TMEM; then O += P_j V_j and
 //                 Z += P_j U_j with P_j read from TMEM (it overwrites S_j).
@@ -34,7 +35,8 @@ namespace {
 
 constexpr int BM = 128;   // rows per tile (TMEM lanes)
 constexpr int BN = 128;   // keys per block
-constexpr int STAGES = 2;
+constexpr int KST = 3;    // K ring: a stage is free once S = Q K^T has been computed
+constexpr int VST = 2;    // V/U ring: a stage is free once O += P V and Z += P U are done
 constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -44,25 +46,31 @@ struct PrefillLayout {
   static constexpr int B_BYTES = RK * D * 2;
   static constexpr int K_BYTES = BN * D * 2;
   static constexpr int U_BYTES = BN * RK * 2;
-  static constexpr int STAGE_BYTES = 2 * K_BYTES + U_BYTES;
+  static constexpr int V_STAGE = K_BYTES + U_BYTES;   // V block then U block
   static constexpr int Q_OFF = 0;
   static constexpr int B_OFF = Q_OFF + Q_BYTES;
-  static constexpr int RING_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
-  static constexpr int BAR_OFF = RING_OFF + STAGES * STAGE_BYTES;
+  static constexpr int K_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
+  static constexpr int V_OFF = K_OFF + KST * K_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VST * V_STAGE;
   static constexpr int TOTAL = BAR_OFF + 256;
   // TMEM columns
   static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_Z = 2 * BN + D;
   static_assert(2 * BN + D + RK <= (int)TMEM_COLS, "TMEM budget");
-  static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+  static_assert(K_BYTES % 1024 == 0 && V_STAGE % 1024 == 0, "stage alignment");
 };
 
 struct Bars {
   uint64_t q_full;
-  uint64_t kv_full[STAGES];
-  uint64_t kv_empty[STAGES];
+  uint64_t k_full[KST];
+  uint64_t k_empty[KST];
+  uint64_t v_full[VST];
+  uint64_t v_empty[VST];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_ready;
+  // O/Z accumulation of block j completes phase j >> 1 of o_ready[j & 1].  With
+  // two barriers the block before any awaited one is always already complete,
+  // so a parity wait can never be satisfied by a stale phase.
+  uint64_t o_ready[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -101,15 +109,20 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
       mbar_init(&bars->p_full[b], 4);
     }
-    mbar_init(&bars->o_ready, 1);
+    mbar_init(&bars->o_ready[0], 1);
+    mbar_init(&bars->o_ready[1], 1);
     bars->abort_flag = 0;
     fence_barrier_init();
   }
@@ -153,52 +166,73 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_4d(smem + Lay::B_OFF, &tmB, &bars->q_full, 0, g, 0, agent, pol_q);
       int n_pages = 0;
       if (p.page_table) n_pages = (p.L0 + p.T + 63) / 64;
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int jb = 0; jb < nb; ++jb) {
-        const int st = jb % STAGES;
-        const uint32_t ph = (jb / STAGES) & 1;
-        if (!mbar_wait_bounded(&bars->kv_empty[st], ph ^ 1, abort_flag, p.flags)) break;
-        issued = jb + 1;
-        const bool need_u = jb * BN + BN > a_i;
-        uint8_t* Ks = smem + Lay::RING_OFF + st * Lay::STAGE_BYTES;
-        uint8_t* Vs = Ks + Lay::K_BYTES;
-        uint8_t* Us = Vs + Lay::K_BYTES;
-        mbar_arrive_expect_tx(&bars->kv_full[st], 2 * Lay::K_BYTES + (need_u ? Lay::U_BYTES : 0));
-        if (!p.page_table) {
-#pragma unroll
-          for (int hh = 0; hh < D / 64; ++hh) {
-            tma_load_4d(Ks + hh * (BN * 128), &tmK, &bars->kv_full[st], hh * 64, jb * BN, g, p.session, pol_kv);
-            tma_load_4d(Vs + hh * (BN * 128), &tmV, &bars->kv_full[st], hh * 64, jb * BN, g, p.session, pol_kv);
-          }
-        } else {
+        // ---- K block jb
+        const int ks_ = jb % KST;
+        if (!mbar_wait_bounded(&bars->k_empty[ks_], ((jb / KST) & 1) ^ 1, abort_flag, p.flags)) break;
+        k_issued = jb + 1;
+        uint8_t* Ks = smem + Lay::K_OFF + ks_ * Lay::K_BYTES;
+        mbar_arrive_expect_tx(&bars->k_full[ks_], Lay::K_BYTES);
+        int phys[BN / 64];
+        if (p.page_table) {
 #pragma unroll
           for (int pg = 0; pg < BN / 64; ++pg) {
             int lp = jb * (BN / 64) + pg;
-            if (lp >= n_pages) lp = 0;  // past the chunk: any valid page (masked out below)
-            int phys = __ldg(p.page_table + (size_t)p.session * p.pt_stride + lp);
-            if (phys < 0 || phys >= p.num_pages) {
+            if (lp >= n_pages) lp = 0;  // past the chunk: any valid page (masked out in the softmax)
+            int ph_ = __ldg(p.page_table + (size_t)p.session * p.pt_stride + lp);
+            if (ph_ < 0 || ph_ >= p.num_pages) {
               atomicOr(p.flags, LRKV_DEVFLAG_PAGE);
-              phys = 0;
+              ph_ = 0;
             }
-#pragma unroll
-            for (int hh = 0; hh < D / 64; ++hh) {
-              tma_load_4d(Ks + hh * (BN * 128) + pg * (64 * 128), &tmK, &bars->kv_full[st], hh * 64, 0, g, phys,
-                          pol_kv);
-              tma_load_4d(Vs + hh * (BN * 128) + pg * (64 * 128), &tmV, &bars->kv_full[st], hh * 64, 0, g, phys,
-                          pol_kv);
-            }
+            phys[pg] = ph_;
           }
         }
-        if (need_u) tma_load_4d(Us, &tmU, &bars->kv_full[st], 0, jb * BN, u_slot, p.session, pol_kv);
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+          if (!p.page_table) {
+            tma_load_4d(Ks + hh * (BN * 128), &tmK, &bars->k_full[ks_], hh * 64, jb * BN, g, p.session, pol_kv);
+          } else {
+#pragma unroll
+            for (int pg = 0; pg < BN / 64; ++pg)
+              tma_load_4d(Ks + hh * (BN * 128) + pg * (64 * 128), &tmK, &bars->k_full[ks_], hh * 64, 0, g, phys[pg],
+                          pol_kv);
+          }
+        }
+        // ---- V (and U) block jb
+        const int vs_ = jb % VST;
+        if (!mbar_wait_bounded(&bars->v_empty[vs_], ((jb / VST) & 1) ^ 1, abort_flag, p.flags)) break;
+        v_issued = jb + 1;
+        const bool need_u = jb * BN + BN > a_i;
+        uint8_t* Vs = smem + Lay::V_OFF + vs_ * Lay::V_STAGE;
+        uint8_t* Us = Vs + Lay::K_BYTES;
+        mbar_arrive_expect_tx(&bars->v_full[vs_], Lay::K_BYTES + (need_u ? Lay::U_BYTES : 0));
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+          if (!p.page_table) {
+            tma_load_4d(Vs + hh * (BN * 128), &tmV, &bars->v_full[vs_], hh * 64, jb * BN, g, p.session, pol_kv);
+          } else {
+#pragma unroll
+            for (int pg = 0; pg < BN / 64; ++pg)
+              tma_load_4d(Vs + hh * (BN * 128) + pg * (64 * 128), &tmV, &bars->v_full[vs_], hh * 64, 0, g, phys[pg],
+                          pol_kv);
+          }
+        }
+        if (need_u) tma_load_4d(Us, &tmU, &bars->v_full[vs_], 0, jb * BN, u_slot, p.session, pol_kv);
       }
       if (*abort_flag) {
         // let every copy this CTA issued land before the CTA can exit
         uint32_t spins = 0;
         while (!mbar_try_wait(&bars->q_full, 0) && ++spins < kSpinCap) {
         }
-        for (int blk = issued > STAGES ? issued - STAGES : 0; blk < issued; ++blk) {
+        for (int blk = k_issued > KST ? k_issued - KST : 0; blk < k_issued; ++blk) {
           spins = 0;
-          while (!mbar_try_wait(&bars->kv_full[blk % STAGES], (blk / STAGES) & 1) && ++spins < kSpinCap) {
+          while (!mbar_try_wait(&bars->k_full[blk % KST], (blk / KST) & 1) && ++spins < kSpinCap) {
+          }
+        }
+        for (int blk = v_issued > VST ? v_issued - VST : 0; blk < v_issued; ++blk) {
+          spins = 0;
+          while (!mbar_try_wait(&bars->v_full[blk % VST], (blk / VST) & 1) && ++spins < kSpinCap) {
           }
         }
       }
@@ -215,12 +249,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool z_started = false;
     for (int jb = 0; jb <= nb && ok; ++jb) {
       if (jb < nb) {
-        const int st = jb % STAGES;
-        ok = mbar_wait_bounded(&bars->kv_full[st], (jb / STAGES) & 1, abort_flag, p.flags);
+        const int st = jb % KST;
+        ok = mbar_wait_bounded(&bars->k_full[st], (jb / KST) & 1, abort_flag, p.flags);
         if (!ok) break;
         if (lane == 0) {
           tc_fence_after();
-          const uint32_t k_base = smem_u32(smem + Lay::RING_OFF + st * Lay::STAGE_BYTES);
+          const uint32_t k_base = smem_u32(smem + Lay::K_OFF + st * Lay::K_BYTES);
           const uint32_t d_s = tmem + (jb & 1 ? Lay::COL_S1 : Lay::COL_S0);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
@@ -230,16 +264,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             umma_ss(d_s, a, b, ID_QK, ks > 0);
           }
           umma_commit(&bars->s_full[jb & 1]);
+          umma_commit(&bars->k_empty[st]);
         }
         __syncwarp();
       }
       if (jb >= 1) {
         const int j = jb - 1;
-        const int st = j % STAGES;
+        const int st = j % VST;
         ok = mbar_wait_bounded(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag, p.flags);
+        if (ok) ok = mbar_wait_bounded(&bars->v_full[st], (j / VST) & 1, abort_flag, p.flags);
         if (!ok) break;
         const bool u_used = j * BN + BN > a_i;
-        uint8_t* Us = smem + Lay::RING_OFF + st * Lay::STAGE_BYTES + 2 * Lay::K_BYTES;
+        uint8_t* Us = smem + Lay::V_OFF + st * Lay::V_STAGE + Lay::K_BYTES;
         if (u_used && j * BN < a_i) {
           // the block holding a_i: rows before the offset are removed (zero-filled) before the MMA reads them
           const int nz = a_i - j * BN;  // rows [0, nz)
@@ -251,7 +287,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) {
           tc_fence_after();
-          const uint32_t v_base = smem_u32(smem + Lay::RING_OFF + st * Lay::STAGE_BYTES + Lay::K_BYTES);
+          const uint32_t v_base = smem_u32(smem + Lay::V_OFF + st * Lay::V_STAGE);
           const uint32_t u_base = smem_u32(Us);
           const uint32_t a_p = tmem + (j & 1 ? Lay::COL_S1 : Lay::COL_S0);
 #pragma unroll
@@ -266,8 +302,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               umma_ts(tmem + Lay::COL_Z, a_p + kk * 8, b, ID_PZ, (z_started || kk > 0) ? 1u : 0u);
             }
           }
-          umma_commit(&bars->kv_empty[st]);
-          umma_commit(&bars->o_ready);
+          umma_commit(&bars->v_empty[st]);
+          umma_commit(&bars->o_ready[j & 1]);
         }
         if (u_used) z_started = true;
         __syncwarp();
@@ -293,21 +329,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_wait_ld();
       const int key0 = jb * BN;
       const bool diag = key0 + BN - 1 > p.L0 + j0;  // some key of the block is past some row's limit
+      if (diag) {
+#pragma unroll
+        for (int cc = 0; cc < BN; ++cc) x[cc] = key0 + cc <= limit ? x[cc] : NEG_INF;
+      }
       float mx = NEG_INF;
 #pragma unroll
-      for (int cc = 0; cc < BN; ++cc) {
-        float v = x[cc] * p.scale_log2;
-        if (diag) v = key0 + cc <= limit ? v : NEG_INF;
-        x[cc] = v;
-        mx = fmaxf(mx, v);
-      }
+      for (int cc = 0; cc < BN; ++cc) mx = fmaxf(mx, x[cc]);
+      mx *= p.scale_log2;  // the scale is positive: the max commutes with it
       const bool need = mx > m_ref + 8.f;
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = fmaxf(m_ref, mx);
         const float alpha = m_new == NEG_INF ? 1.f : fast_exp2(m_ref - m_new);
         if (jb > 0) {
           // O and Z hold the blocks before this one: rescale them in TMEM once PV_{jb-1} is done
-          ok = mbar_wait_bounded(&bars->o_ready, (jb - 1) & 1, abort_flag, p.flags);
+          ok = mbar_wait_bounded(&bars->o_ready[(jb - 1) & 1], ((jb - 1) >> 1) & 1, abort_flag, p.flags);
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < (D + RK) / 32; ++c) {
@@ -338,7 +374,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int cc = 0; cc < BN / 2; ++cc) {
-        const float p0 = fast_exp2(x[2 * cc] - mu), p1 = fast_exp2(x[2 * cc + 1] - mu);
+        const float p0 = fast_exp2(fmaf(x[2 * cc], p.scale_log2, -mu));
+        const float p1 = fast_exp2(fmaf(x[2 * cc + 1], p.scale_log2, -mu));
         pk[cc] = pack_bf16x2(p0, p1);
         l += bf16_lo(pk[cc]) + bf16_hi(pk[cc]);  // the row sum of exactly the weights the MMA uses
       }
@@ -350,7 +387,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(&bars->p_full[jb & 1]);
     }
     // ---- epilogue: out = (O + Z B_i,g) / l
-    if (ok) ok = mbar_wait_bounded(&bars->o_ready, (nb - 1) & 1, abort_flag, p.flags);
+    if (ok) ok = mbar_wait_bounded(&bars->o_ready[(nb - 1) & 1], ((nb - 1) >> 1) & 1, abort_flag, p.flags);
     tc_fence_after();
     const bool z_used = a_i < key_end;  // some block accumulated Z
     float z[RK];
