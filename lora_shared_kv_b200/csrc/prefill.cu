@@ -333,9 +333,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int cc = 0; cc < BN; ++cc) x[cc] = key0 + cc <= limit ? x[cc] : NEG_INF;
       }
-      float mx = NEG_INF;
+      // row max over the block: eight independent chains, then a tree
+      float mx8[8];
 #pragma unroll
-      for (int cc = 0; cc < BN; ++cc) mx = fmaxf(mx, x[cc]);
+      for (int e = 0; e < 8; ++e) mx8[e] = x[e];
+#pragma unroll
+      for (int cc = 8; cc < BN; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], x[cc]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= p.scale_log2;  // the scale is positive: the max commutes with it
       const bool need = mx > m_ref + 8.f;
       if (__any_sync(0xffffffffu, need)) {
@@ -372,13 +377,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const float mu = m_ref == NEG_INF ? 0.f : m_ref;
       uint32_t pk[BN / 2];
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int cc = 0; cc < BN / 2; ++cc) {
         const float p0 = fast_exp2(fmaf(x[2 * cc], p.scale_log2, -mu));
         const float p1 = fast_exp2(fmaf(x[2 * cc + 1], p.scale_log2, -mu));
         pk[cc] = pack_bf16x2(p0, p1);
-        l += bf16_lo(pk[cc]) + bf16_hi(pk[cc]);  // the row sum of exactly the weights the MMA uses
+        // the row sum of exactly the bf16 weights the MMA uses, in eight chains
+        ls[cc & 7] += bf16_lo(pk[cc]) + bf16_hi(pk[cc]);
       }
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) tmem_st32(tmem + lane_addr + s_col + c * 32, pk + c * 32);
       tmem_wait_st();
