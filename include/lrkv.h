@@ -184,6 +184,40 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
                              const int32_t* alora_offsets, void* out, int32_t out_dtype,
                              void* workspace, size_t workspace_bytes, lrkv_stream_t stream);
 
+/*
+ * Decode with the library's own scratch, for callers that cannot allocate
+ * device memory.  The pages have no counterpart: this is a convenience of the
+ * library, not part of the method.
+ *
+ * Who needs it: code whose device memory belongs to someone else's allocator
+ * (a serving engine that hands its plug-ins only tensors), and code for which a
+ * cudaMalloc is not acceptable at call time - cudaMalloc synchronises the whole
+ * device, and on a long-running server with a fragmented heap it can fail even
+ * when enough memory is free in total.
+ *
+ * Same arguments and result as lrkv_attn_decode, minus the workspace.  The
+ * scratch is one file-scope device array of LRKV_STATIC_SCRATCH_BYTES that
+ * every GPU which loads the library keeps until the process exits.  The call
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *  - Shapes whose lrkv_decode_workspace_bytes() exceeds the scratch size return
+ *    LRKV_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *  - The first call on a device looks up the scratch's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call clears the scratch's flag and ticket words on `stream`, then
+ *    runs the same kernel as lrkv_attn_decode.  All calls share the one array
+ *    and it keeps the last call's contents, so calls that can overlap on the GPU
+ *    (different streams, or different host threads on one device) race and
+ *    give wrong results: order them.  Device-side flags of these calls are not
+ *    reported (the scratch is not visible to the caller).
+ */
+#define LRKV_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv,
+                                            const int32_t* seq_lens, int32_t max_seq_len,
+                                            const lrkv_u_view* u, const void* b,
+                                            const int32_t* alora_offsets, void* out, int32_t out_dtype,
+                                            lrkv_stream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* Prefill chunk: T new rows per agent, causal, over one session.          */
 /* ---------------------------------------------------------------------- */

@@ -44,6 +44,7 @@ EXPORTS = (
     "lrkv_append_lr_cache",
     "lrkv_decode_workspace_bytes",
     "lrkv_attn_decode",
+    "lrkv_attn_decode_static_scratch",
     "lrkv_prefill_workspace_bytes",
     "lrkv_attn_prefill_chunk",
     "lrkv_workspace_reset",
@@ -98,6 +99,8 @@ def lib():
         L.lrkv_decode_workspace_bytes.argtypes = [P(Problem), i32]
         L.lrkv_decode_workspace_bytes.restype = sz
         L.lrkv_attn_decode.argtypes = [P(Problem), vp, P(KVView), vp, i32, P(UView), vp, vp, vp, i32, vp, sz, vp]
+        L.lrkv_attn_decode_static_scratch.argtypes = [P(Problem), vp, P(KVView), vp, i32, P(UView), vp, vp, vp,
+                                                      i32, vp]
         L.lrkv_prefill_workspace_bytes.argtypes = [P(Problem), i32, i32]
         L.lrkv_prefill_workspace_bytes.restype = sz
         L.lrkv_attn_prefill_chunk.argtypes = [P(Problem), vp, P(KVView), i32, i32, i32, P(UView), vp, vp, vp,
@@ -109,7 +112,8 @@ def lib():
         L.lrkv_last_error_detail.argtypes = []
         L.lrkv_last_error_detail.restype = ctypes.c_char_p
         L.lrkv_version.restype = i32
-        for name in ("lrkv_append_lr_cache", "lrkv_attn_decode", "lrkv_attn_prefill_chunk",
+        for name in ("lrkv_append_lr_cache", "lrkv_attn_decode", "lrkv_attn_decode_static_scratch",
+                     "lrkv_attn_prefill_chunk",
                      "lrkv_workspace_reset", "lrkv_query_device_status"):
             getattr(L, name).restype = i32
         _lib = L
@@ -191,6 +195,20 @@ def lrkv_attn_decode(problem, q, kv, seq_lens, max_seq_len, u, b, offsets, out, 
                                   int(max_seq_len), ctypes.byref(uv), _ptr(b), _ptr(offsets), _ptr(out), odt,
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)))
+
+
+def lrkv_attn_decode_static_scratch(problem, q, kv, seq_lens, max_seq_len, u, b, offsets, out, stream=None):
+    """lrkv_attn_decode without a workspace argument, for callers that may not allocate device memory.
+
+    The library keeps one fixed scratch array per GPU (LRKV_STATIC_SCRATCH_BYTES); shapes that need more
+    are rejected with LRKV_ERR_WORKSPACE_TOO_SMALL.  Calls share that array: keep them ordered on one stream.
+    """
+    assert q.is_contiguous() and b.is_contiguous() and out.is_contiguous()
+    odt = F32 if out.dtype == torch.float32 else BF16
+    uv = u if isinstance(u, UView) else u_view(u)
+    _check(lib().lrkv_attn_decode_static_scratch(ctypes.byref(problem), _ptr(q), ctypes.byref(kv), _ptr(seq_lens),
+                                                 int(max_seq_len), ctypes.byref(uv), _ptr(b), _ptr(offsets),
+                                                 _ptr(out), odt, _stream(stream)))
 
 
 def lrkv_prefill_workspace_bytes(problem, ctx_len, T):

@@ -376,6 +376,67 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
   return LRKV_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Decode with library-owned scratch: for callers that may not allocate device
+// memory.  The scratch is one file-scope device array (every GPU that loads the
+// library holds it until the process exits).
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;  // LRKV_STATIC_SCRATCH_BYTES in lrkv.h
+static_assert(kStaticScratchBytes == LRKV_STATIC_SCRATCH_BYTES, "header and library disagree on the scratch size");
+
+__device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+// Device address of g_decode_scratch on the current device, looked up once per
+// device (the host-side name of the array is not a device address).
+lrkv_status static_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LRKV_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess || ptr == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
+    addr[dev] = ptr;
+  }
+  *out = addr[dev];
+  return LRKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv,
+                                            const int32_t* seq_lens, int32_t max_seq_len, const lrkv_u_view* u,
+                                            const void* b, const int32_t* alora_offsets, void* out,
+                                            int32_t out_dtype, lrkv_stream_t stream) {
+  lrkv_status s = check_problem(p);
+  if (s != LRKV_OK) return s;
+  DeviceInfo dev;
+  if ((s = device_info(&dev)) != LRKV_OK) return s;
+  DecodePlan pl;
+  if ((s = plan_decode(p, max_seq_len, dev, &pl)) != LRKV_OK) return s;
+  if (pl.bytes > kStaticScratchBytes)
+    return fail(LRKV_ERR_WORKSPACE_TOO_SMALL,
+                "this shape needs %zu bytes of decode scratch; the library's fixed scratch holds %zu "
+                "(use lrkv_attn_decode with a caller-owned workspace)", pl.bytes, kStaticScratchBytes);
+  void* scratch = nullptr;
+  if ((s = static_scratch_address(&scratch)) != LRKV_OK) return s;
+  // flags and per-item tickets must start at zero; the partial records need no clearing
+  cudaError_t e = cudaMemsetAsync(scratch, 0, pl.partials_off, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(decode scratch header)");
+  return lrkv_attn_decode(p, q, kv, seq_lens, max_seq_len, u, b, alora_offsets, out, out_dtype, scratch,
+                          kStaticScratchBytes, stream);
+}
+
 size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T) {
   if (check_problem(p) != LRKV_OK || ctx_len < 0 || T < 0) return 0;
   return lrkv::kWsHeaderBytes;  // device-side flags only
