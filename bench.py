@@ -331,6 +331,10 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small profiling cases only; not a bench line)")
+    ap.add_argument("--context", type=int, default=None,
+                    help="override the context length (profiling sweeps only; not a bench line)")
+    ap.add_argument("--sessions", type=int, default=None,
+                    help="override the session count (profiling sweeps only; not a bench line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -338,9 +342,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = CONFIGS[args.workload]
+    import dataclasses
     if args.layers is not None:
-        import dataclasses
         cfg = dataclasses.replace(cfg, layers=args.layers)
+    if args.context is not None:
+        cfg = dataclasses.replace(cfg, L=args.context)
+    if args.sessions is not None:
+        cfg = dataclasses.replace(cfg, S=args.sessions)
 
     if args.impl == "reference":
         if rank != 0:

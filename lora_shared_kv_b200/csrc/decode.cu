@@ -83,9 +83,50 @@ __device__ __forceinline__ void seg_rows(const DecodeParams& p, Seg& sg) {
   sg.n_ag = (row_hi - 1) / p.G - sg.i_lo + 1;
 }
 
-__device__ __forceinline__ int seg_tiles_end(const Seg& sg) {
-  const int nts = (sg.sl + KT - 1) / KT;
-  return sg.hi < nts ? sg.hi : nts;
+__device__ __forceinline__ int seg_tiles_valid(const Seg& sg) { return (sg.sl + KT - 1) / KT; }
+
+// Visiting order of an item's tiles.  Tiles go in runs of kTileRun
+// (contiguous in HBM); the full runs are visited in the order
+// (j * stride) mod runs with a stride coprime to the run count (near 0.618 of
+// it), and a partial last run stays in place.  Every contiguous range of k then
+// covers the item evenly, so the tiles past the agents' offsets (which carry
+// the low-rank work) spread evenly over the CTAs that share an item.  The
+// softmax result does not depend on the order.  The iterator steps with one
+// add and one compare; the modulo runs once per segment.
+struct TileOrder {
+  int runs, stride, r, w;
+  __device__ __forceinline__ void start(const DecodeParams& p, int k0) {
+    runs = p.nt / kTileRun;
+    stride = p.tile_stride;
+    const int j = k0 / kTileRun;
+    w = k0 % kTileRun;
+    r = j < runs ? (int)(((long long)j * stride) % runs) : -1 - j;
+  }
+  __device__ __forceinline__ int tile() const { return r >= 0 ? r * kTileRun + w : (-1 - r) * kTileRun + w; }
+  __device__ __forceinline__ void next() {
+    if (++w == kTileRun) {
+      w = 0;
+      if (r >= 0) {
+        ++run_index;
+        if (run_index < runs) {
+          r += stride;
+          if (r >= runs) r -= runs;
+        } else {
+          r = -1 - run_index;
+        }
+      } else {
+        --r;
+      }
+    }
+  }
+  int run_index;
+};
+
+__device__ __forceinline__ TileOrder tile_order(const DecodeParams& p, int k0) {
+  TileOrder o;
+  o.start(p, k0);
+  o.run_index = k0 / kTileRun;
+  return o;
 }
 
 __device__ __forceinline__ int load_offset(const DecodeParams& p, int s, int agent, bool flag_errors) {
@@ -126,17 +167,22 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
     Seg sg = make_seg(p, t, t_end, false);
     t += sg.hi - sg.lo;
     seg_rows(p, sg);
-    const int hi_e = seg_tiles_end(sg);
+    const int nts = seg_tiles_valid(sg);
     // lane j < n_ag holds the offset of agent i_lo + j
     const int my_a = lane < sg.n_ag ? load_offset(p, sg.s, sg.i_lo + lane, false) : 0x7fffffff;
     int pid_reg = 0;
-    for (int tile = sg.lo; tile < hi_e; ++tile, ++n) {
-      const int k = tile - sg.lo;
-      if (p.paged && (k & 31) == 0) {
-        const int tt = tile + lane;
-        pid_reg = tt < hi_e ? __ldg(p.page_table + (size_t)sg.s * p.pt_stride + tt) : 0;
+    TileOrder ord = tile_order(p, sg.lo);
+    for (int kk = sg.lo; kk < sg.hi; ++kk, ord.next()) {
+      const int tile = ord.tile();
+      const int k = kk - sg.lo;
+      if (p.paged && (k & 31) == 0) {  // page ids of the next 32 tiles, one per lane
+        const int k2 = kk + lane;
+        const int t2 = k2 < sg.hi ? tile_order(p, k2).tile() : nts;
+        pid_reg = t2 < nts ? __ldg(p.page_table + (size_t)sg.s * p.pt_stride + t2) : 0;
       }
       const int phys = p.paged ? __shfl_sync(0xffffffffu, pid_reg, k & 31) : 0;
+      if (tile >= nts) continue;  // past the session's length (consumers skip it too)
+      ++n;
       const int tile_end_key = tile * KT + KT;
       const unsigned need = __ballot_sync(0xffffffffu, lane < sg.n_ag && tile_end_key > my_a);
       const unsigned umask = p.mode == LRKV_BASE_SHARED ? need : (need ? 1u : 0u);
@@ -145,7 +191,7 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
       mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.flags);
       if (lane == 0) {
         if (!page_ok) atomicOr(p.flags, LRKV_DEVFLAG_PAGE);
-        seq[stage] = n;
+        seq[stage] = n - 1;
         uint8_t* st = ring + (size_t)stage * stage_bytes;
         if (bytes == 0) {
           mbar_arrive(&full[stage]);
@@ -330,7 +376,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     Seg sg = make_seg(p, t, t_end, tid == 0);
     t += sg.hi - sg.lo;
     seg_rows(p, sg);
-    const int hi_e = seg_tiles_end(sg);
+    const int nts = seg_tiles_valid(sg);
     const int sl = sg.sl;
 
     if (tid < sg.n_ag) a_sm[tid] = load_offset(p, sg.s, sg.i_lo + tid, true);
@@ -371,7 +417,10 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
 #pragma unroll
       for (int e = 0; e < 4; ++e) st.z[mz][e] = 0.f;
 
-    for (int tile = sg.lo; tile < hi_e; ++tile) {
+    TileOrder ord = tile_order(p, sg.lo);
+    for (int kk = sg.lo; kk < sg.hi; ++kk, ord.next()) {
+      const int tile = ord.tile();
+      if (tile >= nts) continue;  // past the session's length (the producer skips it too)
       const int my_n = ntile;
       const bool mine = (ntile % NOG) == og;
       const int my_stage = stage;
@@ -514,7 +563,8 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
         }
       }
 
-      // ---- Z^T += U_i^T P^T over this warp's rows of agent i; U rows < a_i or >= seq_len selected out
+      // ---- Z^T += U_i^T P^T over this warp's rows of agent i; U rows < a_i or >= seq_len selected out.
+      // Tiles wholly inside [a_i, seq_len) need no masks: one ldmatrix and one MMA per key block.
       const bool lr_full = p.mode == LRKV_BASE_LR_SHARED && !boundary && a_max <= tile_key0;
       const int pass_lo = lr_full ? 0 : ag_lo;
       const int pass_hi = lr_full ? 0 : ag_hi;
@@ -524,6 +574,31 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
         const int slot = p.mode == LRKV_BASE_SHARED ? ag : 0;
         const uint32_t ub = Us + slot * U_BYTES;
         const bool use = lr_full ? (my_agent >= 0) : (my_agent == ag);
+        const bool clean = !boundary && a_i <= tile_key0;  // warp-uniform
+        uint32_t bz[4][2];
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          bz[kb][0] = use ? pb[kb][0] : 0u;
+          bz[kb][1] = use ? pb[kb][1] : 0u;
+        }
+        if (clean) {
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+#pragma unroll
+            for (int mz = 0; mz < MTZ; ++mz) {
+              uint32_t a0, a1 = 0, a2, a3 = 0;
+              if constexpr (RK == 8) {
+                ldsm_x2_t(a0, a2, ub + (16 * kb + ((lane >> 3) & 1) * 8 + (lane & 7)) * (RK * 2));
+              } else {
+                const int j = lane >> 3;
+                ldsm_x4_t(a0, a1, a2, a3,
+                          ub + (16 * kb + (j >> 1) * 8 + (lane & 7)) * (RK * 2) + (2 * mz + (j & 1)) * 16);
+              }
+              mma_bf16_16816(st.z[mz], a0, a1, a2, a3, bz[kb][0], bz[kb][1]);
+            }
+          }
+          continue;
+        }
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
           const int k16 = tile_key0 + 16 * kb;
@@ -533,30 +608,45 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           const bool ok8 = k0 + 8 >= a_i && k0 + 8 < sl, ok9 = k0 + 9 >= a_i && k0 + 9 < sl;
           const uint32_t um_lo = (ok0 ? 0x0000ffffu : 0u) | (ok1 ? 0xffff0000u : 0u);
           const uint32_t um_hi = (ok8 ? 0x0000ffffu : 0u) | (ok9 ? 0xffff0000u : 0u);
-          const uint32_t b0 = use ? pb[kb][0] : 0u, b1 = use ? pb[kb][1] : 0u;
 #pragma unroll
           for (int mz = 0; mz < MTZ; ++mz) {
             uint32_t a0, a1 = 0, a2, a3 = 0;
             if constexpr (RK == 8) {
-              const int key = 16 * kb + ((lane >> 3) & 1) * 8 + (lane & 7);
-              ldsm_x2_t(a0, a2, ub + key * (RK * 2));
+              ldsm_x2_t(a0, a2, ub + (16 * kb + ((lane >> 3) & 1) * 8 + (lane & 7)) * (RK * 2));
             } else {
               const int j = lane >> 3;
-              const int key = 16 * kb + (j >> 1) * 8 + (lane & 7);
-              const int ch = 2 * mz + (j & 1);
-              ldsm_x4_t(a0, a1, a2, a3, ub + key * (RK * 2) + ch * 16);
+              ldsm_x4_t(a0, a1, a2, a3,
+                        ub + (16 * kb + (j >> 1) * 8 + (lane & 7)) * (RK * 2) + (2 * mz + (j & 1)) * 16);
             }
             a0 &= um_lo;
             a1 &= um_lo;
             a2 &= um_hi;
             a3 &= um_hi;
-            mma_bf16_16816(st.z[mz], a0, a1, a2, a3, b0, b1);
+            mma_bf16_16816(st.z[mz], a0, a1, a2, a3, bz[kb][0], bz[kb][1]);
           }
         }
       }
 
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[my_stage]);
+    }
+
+    // ---- the finishing epilogue needs, per (agent, dim) pair, the agent's B
+    // column B_i[:, g d + dim]; fetch this thread's first pairs now so the loads
+    // overlap the merge and the ticket round trip (B is small and L2-resident)
+    constexpr int PB = RK >= 32 ? 2 : 4;  // pairs per thread kept in registers
+    const int HD = p.Hkv * D;
+    const int n_pairs = sg.n_ag * D;
+    float bk[PB][RK];
+#pragma unroll
+    for (int k = 0; k < PB; ++k) {
+      const int e = tid + k * CT;
+      if (e < n_pairs) {
+        const uint16_t* bcol = static_cast<const uint16_t*>(p.b) + ((size_t)(sg.i_lo + e / D) * RK) * HD +
+                               (size_t)sg.g * D + e % D;
+#pragma unroll
+        for (int r = 0; r < RK; ++r) bk[k][r] = bf16_to_f32(__ldg(bcol + (size_t)r * HD));
+      }
     }
 
     // ---- reduce l over the lanes that share a row; chain the groups into record 0
@@ -600,90 +690,110 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       if (finish) {
         __threadfence();
         const float* base = p.partials + (size_t)sg.item * p.max_segs * REC;
-        if (tid < RP) {
-          float M = NEG_INF;
-          for (int j = 0; j < segs; ++j) M = fmaxf(M, __ldcg(base + (size_t)j * REC + tid));
-          float L = 0.f;
-          for (int j = 0; j < segs; ++j) {
-            const float mj = __ldcg(base + (size_t)j * REC + tid);
-            L += mj == NEG_INF ? 0.f : __ldcg(base + (size_t)j * REC + RP + tid) * fast_exp2(mj - M);
-          }
-          merge[tid] = M;
-          merge[RP + tid] = L;
-        }
-        named_bar_sync(1, CT);
+        constexpr int E4 = RP * (D + RK) / 4;
+        constexpr int PER = (E4 + CT - 1) / CT;  // float4 elements of the record per thread
+        float4 acc[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j0 = 0; j0 < segs; j0 += SEG_CHUNK) {
           const int nj = min(SEG_CHUNK, segs - j0);
+          // row maxima and sums of every record of the chunk: one round of loads
           if (tid < RP) {
-            const float M = merge[tid];
-            for (int jj = 0; jj < nj; ++jj) {
-              const float mj = __ldcg(base + (size_t)(j0 + jj) * REC + tid);
-              scw[jj * RP + tid] = mj == NEG_INF ? 0.f : fast_exp2(mj - M);
+            float mj[SEG_CHUNK], lj[SEG_CHUNK];
+#pragma unroll
+            for (int jj = 0; jj < SEG_CHUNK; ++jj) {
+              mj[jj] = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + tid) : NEG_INF;
+              lj[jj] = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + RP + tid) : 0.f;
             }
+            if (j0 == 0) {
+              // the global maximum needs every record: this chunk's, then any further ones
+              float M = NEG_INF;
+#pragma unroll
+              for (int jj = 0; jj < SEG_CHUNK; ++jj) M = fmaxf(M, mj[jj]);
+              for (int j = SEG_CHUNK; j < segs; ++j) M = fmaxf(M, __ldcg(base + (size_t)j * REC + tid));
+              merge[tid] = M;
+              merge[RP + tid] = 0.f;
+            }
+            const float M = merge[tid];
+            float L = merge[RP + tid];
+#pragma unroll
+            for (int jj = 0; jj < SEG_CHUNK; ++jj) {
+              const float sc = (jj < nj && mj[jj] != NEG_INF) ? fast_exp2(mj[jj] - M) : 0.f;
+              scw[jj * RP + tid] = sc;
+              L += lj[jj] * sc;
+            }
+            merge[RP + tid] = L;
           }
           named_bar_sync(1, CT);
-          constexpr int E4 = RP * (D + RK) / 4;
-          for (int e4 = tid; e4 < E4; e4 += 2 * CT) {
-            float4 acc[2];
-            int rows2[2];
+          // O and Z of every record of the chunk: PER float4 loads per record, issued together
+          for (int jj = 0; jj < nj; ++jj) {
+            const float* rj = base + (size_t)(j0 + jj) * REC + 2 * RP;
+            float4 v[PER];
 #pragma unroll
-            for (int u2 = 0; u2 < 2; ++u2) {
-              const int e = (e4 + u2 * CT) * 4;
-              rows2[u2] = e < RP * D ? e / D : (e - RP * D) / RK;
-              acc[u2] = (j0 == 0 || e4 + u2 * CT >= E4) ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                                          : *reinterpret_cast<const float4*>(merge + 2 * RP + e);
-            }
-            for (int jj = 0; jj < nj; ++jj) {
-              const float* rj = base + (size_t)(j0 + jj) * REC + 2 * RP;
-#pragma unroll
-              for (int u2 = 0; u2 < 2; ++u2) {
-                if (e4 + u2 * CT >= E4) continue;
-                const float4 x = __ldcg(reinterpret_cast<const float4*>(rj + (e4 + u2 * CT) * 4));
-                const float sc = scw[jj * RP + rows2[u2]];
-                acc[u2].x += x.x * sc;
-                acc[u2].y += x.y * sc;
-                acc[u2].z += x.z * sc;
-                acc[u2].w += x.w * sc;
-              }
+            for (int u = 0; u < PER; ++u) {
+              const int e4 = tid + u * CT;
+              v[u] = e4 < E4 ? __ldcg(reinterpret_cast<const float4*>(rj) + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
 #pragma unroll
-            for (int u2 = 0; u2 < 2; ++u2)
-              if (e4 + u2 * CT < E4) *reinterpret_cast<float4*>(merge + 2 * RP + (e4 + u2 * CT) * 4) = acc[u2];
+            for (int u = 0; u < PER; ++u) {
+              const int e = (tid + u * CT) * 4;
+              if (e >= E4 * 4) continue;
+              const int row = e < RP * D ? e / D : (e - RP * D) / RK;
+              const float sc = scw[jj * RP + row];
+              acc[u].x += v[u].x * sc;
+              acc[u].y += v[u].y * sc;
+              acc[u].z += v[u].z * sc;
+              acc[u].w += v[u].w * sc;
+            }
           }
           named_bar_sync(1, CT);
         }
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+          const int e4 = tid + u * CT;
+          if (e4 < E4) *reinterpret_cast<float4*>(merge + 2 * RP + e4 * 4) = acc[u];
+        }
+        named_bar_sync(1, CT);
       }
     }
 
     if (finish) {
       // out = (O + Z B_i,g) / l, once per row: the up-projection of Eq. 12.
-      // One thread per (agent, dim): the agent's B column is loaded once and
-      // reused by every GQA row of that agent.
+      // One thread per (agent, dim); the agent's B column serves all its GQA rows.
       const float* mL = merge + RP;
       const float* mO = merge + 2 * RP;
       const float* mZ = mO + RP * D;
-      const int HD = p.Hkv * D;
-      for (int e = tid; e < sg.n_ag * D; e += CT) {
-        const int a_loc = e / D, dim = e % D;
-        const int agent = sg.i_lo + a_loc;
-        const uint16_t* bcol = static_cast<const uint16_t*>(p.b) + ((size_t)agent * RK) * HD + (size_t)sg.g * D + dim;
-        float bk[RK];
+      for (int e0 = tid; e0 < n_pairs; e0 += PB * CT) {
 #pragma unroll
-        for (int k = 0; k < RK; ++k) bk[k] = bf16_to_f32(__ldg(bcol + (size_t)k * HD));
-        int r_begin = agent * p.G - sg.row_lo, r_end = r_begin + p.G;
-        r_begin = r_begin < 0 ? 0 : r_begin;
-        r_end = r_end > sg.rows ? sg.rows : r_end;
-        for (int row = r_begin; row < r_end; ++row) {
-          float acc = mO[row * D + dim];
+        for (int k = 0; k < PB; ++k) {
+          const int e = e0 + k * CT;
+          if (e >= n_pairs) continue;
+          const int dim = e % D;
+          const int agent = sg.i_lo + e / D;
+          float bcol[RK];
+          if (e0 == tid) {
 #pragma unroll
-          for (int k = 0; k < RK; ++k) acc = fmaf(mZ[row * RK + k], bk[k], acc);
-          const float L = mL[row];
-          const float o = L > 0.f ? acc / L : 0.f;
-          const int grow = sg.row_lo + row;
-          const int h = sg.g * p.G + grow % p.G;
-          const size_t oi = (((size_t)sg.s * p.N + agent) * p.Hq + h) * D + dim;
-          if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
-          else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+            for (int r = 0; r < RK; ++r) bcol[r] = bk[k][r];
+          } else {  // pairs beyond the prefetched ones (many agents per KV head)
+            const uint16_t* bp = static_cast<const uint16_t*>(p.b) + ((size_t)agent * RK) * HD + (size_t)sg.g * D + dim;
+#pragma unroll
+            for (int r = 0; r < RK; ++r) bcol[r] = bf16_to_f32(__ldg(bp + (size_t)r * HD));
+          }
+          int r_begin = agent * p.G - sg.row_lo, r_end = r_begin + p.G;
+          r_begin = r_begin < 0 ? 0 : r_begin;
+          r_end = r_end > sg.rows ? sg.rows : r_end;
+          for (int row = r_begin; row < r_end; ++row) {
+            float acc = mO[row * D + dim];
+#pragma unroll
+            for (int r = 0; r < RK; ++r) acc = fmaf(mZ[row * RK + r], bcol[r], acc);
+            const float L = mL[row];
+            const float o = L > 0.f ? acc / L : 0.f;
+            const int grow = sg.row_lo + row;
+            const int h = sg.g * p.G + grow % p.G;
+            const size_t oi = (((size_t)sg.s * p.N + agent) * p.Hq + h) * D + dim;
+            if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
+            else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+          }
         }
       }
     }

@@ -362,6 +362,25 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
   dp.num_pages = kv->page_table ? kv->num_pages : 0;
   dp.paged = kv->page_table != nullptr;
   dp.nt = pl.nt;
+  {
+    // Visiting order of an item's tiles.  Tiles past an agent's offset carry
+    // its U tile and low-rank MMAs; when those are a large share of a tile's
+    // work (BaseShared with n_agents * r >= d / 2, i.e. U bytes >= a quarter of
+    // the K+V bytes) they must be spread evenly over the CTAs sharing an item,
+    // so runs of tiles are visited in a low-discrepancy order (stride coprime
+    // to the run count, near 0.618 of it).  Otherwise plain ascending order
+    // streams HBM best (stride 1).
+    const int runs = pl.nt / lrkv::kTileRun;
+    const bool balance = p->mode == LRKV_BASE_SHARED && pl.n_u_slots * p->rank * 2 >= p->head_dim;
+    int stride = 1;
+    if (balance && runs > 1) {
+      stride = (int)(0.618 * runs) | 1;
+      auto gcd = [](long long x, long long y) { while (y) { long long t = x % y; x = y; y = t; } return x; };
+      while (gcd(stride, runs) != 1) stride += 2;
+      if (stride % runs == 0) stride = 1;
+    }
+    dp.tile_stride = stride;
+  }
   dp.items = pl.items;
   dp.W = pl.W;
   dp.max_segs = pl.max_segs;

@@ -18,6 +18,7 @@ constexpr int kWsHeaderBytes = 256;     // flags word + padding at the start of 
 constexpr int kKeysPerTile = 64;        // keys per K/V tile (one TMA box, one page)
 constexpr int kMaxRowsPerItem = 32;     // query rows (agents x GQA heads) per decode work item
 constexpr int kMaxAgents = 16;
+constexpr int kTileRun = 4;             // decode tiles visited contiguously (see tile_of in decode.cu)
 
 // ---------------------------------------------------------------------------
 // decode
@@ -42,6 +43,7 @@ struct DecodeParams {
   int num_pages;
   int paged;
   int nt;                    // key tiles per work item
+  int tile_stride;           // runs of kTileRun tiles of an item are visited in the order (j * tile_stride) mod runs
   int items;                 // S * Hkv * n_rg
   long long W;               // items * nt (flattened tile count)
   int max_segs;              // partial slots per item
