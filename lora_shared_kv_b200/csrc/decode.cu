@@ -326,6 +326,188 @@ __device__ __forceinline__ void absorb_rows(RowState<D, RK>& st, const float* re
   }
 }
 
+// This warp's query rows as the B operand of S^T = K Q^T: row `qrow` of the
+// item, dims 16 ks + 2 t4 (+1, +8, +9).
+template <int D>
+__device__ __forceinline__ void load_q_frags(const DecodeParams& p, const Seg& sg, int qrow, int t4,
+                                             uint32_t (*qf)[2]) {
+  const bool qvalid = qrow < sg.rows;
+  const __nv_bfloat16* qptr = nullptr;
+  if (qvalid) {
+    const int grow = sg.row_lo + qrow;
+    qptr = static_cast<const __nv_bfloat16*>(p.q) + (((size_t)sg.s * p.N + grow / p.G) * p.Hq + sg.g * p.G + grow % p.G) * D;
+  }
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    qf[ks][0] = qvalid ? __ldg(reinterpret_cast<const unsigned int*>(qptr + ks * 16 + 2 * t4)) : 0u;
+    qf[ks][1] = qvalid ? __ldg(reinterpret_cast<const unsigned int*>(qptr + ks * 16 + 8 + 2 * t4)) : 0u;
+  }
+}
+
+// Facts of one segment's merged record, enough to publish or finish it.
+struct SegInfo {
+  int item, s, g, row_lo, rows, i_lo, n_ag;
+  int segs;  // CTAs sharing the item
+  int slot;  // this CTA's partial-record slot among them
+};
+
+__device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Seg& sg) {
+  SegInfo si;
+  si.item = sg.item;
+  si.s = sg.s;
+  si.g = sg.g;
+  si.row_lo = sg.row_lo;
+  si.rows = sg.rows;
+  si.i_lo = sg.i_lo;
+  si.n_ag = sg.n_ag;
+  const long long C = gridDim.x;
+  const long long c_first = owner_cta((long long)sg.item * p.nt, p.W, C);
+  const long long c_last = owner_cta((long long)(sg.item + 1) * p.nt - 1, p.W, C);
+  si.segs = (int)(c_last - c_first + 1);
+  si.slot = (int)((long long)blockIdx.x - c_first);
+  return si;
+}
+
+// Publish a segment's merged record `rec` (shared memory, [m | l | O | Z] per
+// row), or, when this CTA is the last of the item's CTAs to get there (atomic
+// ticket), combine every partial record of the item and write
+// out = (O + Z B_i,g) / l: the up-projection of Eq. 12, once per row.  Run by a
+// team of NTH threads (tid in [0, NTH)) that `sync` synchronises; each thread
+// holds the B columns of PB (agent, dim) pairs at a time.
+template <int D, int NT, int RK, int NTH, int PB, typename Sync>
+__device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegInfo& si, float* rec, float* scw,
+                                               int* bcast, int tid, Sync sync) {
+  constexpr int RP = NT * 8;
+  constexpr int REC = RP * (D + RK + 2);
+  constexpr int E4 = RP * (D + RK) / 4;
+  constexpr int PERC = 6;  // float4 elements per thread per combine pass
+  const float NEG_INF = -INFINITY;
+  bool finish = true;
+  if (si.segs > 1) {
+    float* grec = p.partials + ((size_t)si.item * p.max_segs + (size_t)si.slot) * REC;
+    for (int e = tid * 4; e < REC; e += NTH * 4)
+      __stcg(reinterpret_cast<float4*>(grec + e), *reinterpret_cast<const float4*>(rec + e));
+    sync();
+    if (tid == 0) {
+      __threadfence();
+      const int prev = atomicAdd(p.tickets + si.item, 1);
+      const int last = prev == si.segs - 1;
+      if (last) p.tickets[si.item] = 0;
+      *bcast = last;
+    }
+    sync();
+    finish = *bcast != 0;
+    if (!finish) return;
+    __threadfence();
+    const float* base = p.partials + (size_t)si.item * p.max_segs * REC;
+    // maxima and sums of every record (chunks of SEG_CHUNK records); rows <= 32 <= NTH
+    if (tid < RP) {
+      float M = NEG_INF;
+      for (int j0 = 0; j0 < si.segs; j0 += SEG_CHUNK) {
+        float mj[SEG_CHUNK];
+#pragma unroll
+        for (int jj = 0; jj < SEG_CHUNK; ++jj)
+          mj[jj] = j0 + jj < si.segs ? __ldcg(base + (size_t)(j0 + jj) * REC + tid) : NEG_INF;
+#pragma unroll
+        for (int jj = 0; jj < SEG_CHUNK; ++jj) M = fmaxf(M, mj[jj]);
+      }
+      rec[tid] = M;
+    }
+    sync();
+    // O and Z: PERC float4 per thread per pass, all records' loads of a pass issued together
+    for (int e0 = 0; e0 < E4; e0 += NTH * PERC) {
+      float4 acc[PERC];
+#pragma unroll
+      for (int u = 0; u < PERC; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      float L = 0.f;
+      for (int j0 = 0; j0 < si.segs; j0 += SEG_CHUNK) {
+        const int nj = min(SEG_CHUNK, si.segs - j0);
+        if (tid < RP) {
+          const float M = rec[tid];
+#pragma unroll
+          for (int jj = 0; jj < SEG_CHUNK; ++jj) {
+            const float mj = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + tid) : NEG_INF;
+            const float lj = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + RP + tid) : 0.f;
+            const float sc = mj == NEG_INF ? 0.f : fast_exp2(mj - M);
+            scw[jj * RP + tid] = sc;
+            L += lj * sc;
+          }
+        }
+        sync();
+        for (int jj = 0; jj < nj; ++jj) {
+          const float4* rj = reinterpret_cast<const float4*>(base + (size_t)(j0 + jj) * REC + 2 * RP);
+          float4 v[PERC];
+#pragma unroll
+          for (int u = 0; u < PERC; ++u) {
+            const int e4 = e0 + tid + u * NTH;
+            v[u] = e4 < E4 ? __ldcg(rj + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < PERC; ++u) {
+            const int e4 = e0 + tid + u * NTH;
+            if (e4 >= E4) continue;
+            const int e = e4 * 4;
+            const int row = e < RP * D ? e / D : (e - RP * D) / RK;
+            const float sc = scw[jj * RP + row];
+            acc[u].x += v[u].x * sc;
+            acc[u].y += v[u].y * sc;
+            acc[u].z += v[u].z * sc;
+            acc[u].w += v[u].w * sc;
+          }
+        }
+        sync();
+      }
+#pragma unroll
+      for (int u = 0; u < PERC; ++u) {
+        const int e4 = e0 + tid + u * NTH;
+        if (e4 < E4) *reinterpret_cast<float4*>(rec + 2 * RP + e4 * 4) = acc[u];
+      }
+      if (e0 == 0 && tid < RP) rec[RP + tid] = L;
+    }
+    sync();
+  }
+  // out = (O + Z B_i,g) / l; one thread per (agent, dim), the agent's B column serves its GQA rows
+  const int HD = p.Hkv * D;
+  const int n_pairs = si.n_ag * D;
+  const float* mL = rec + RP;
+  const float* mO = rec + 2 * RP;
+  const float* mZ = mO + RP * D;
+  for (int e0 = tid; e0 < n_pairs; e0 += PB * NTH) {
+    float bb[PB][RK];
+#pragma unroll
+    for (int k = 0; k < PB; ++k) {
+      const int e = e0 + k * NTH;
+      if (e >= n_pairs) continue;
+      const uint16_t* bp =
+          static_cast<const uint16_t*>(p.b) + ((size_t)(si.i_lo + e / D) * RK) * HD + (size_t)si.g * D + e % D;
+#pragma unroll
+      for (int r = 0; r < RK; ++r) bb[k][r] = bf16_to_f32(__ldg(bp + (size_t)r * HD));
+    }
+#pragma unroll
+    for (int k = 0; k < PB; ++k) {
+      const int e = e0 + k * NTH;
+      if (e >= n_pairs) continue;
+      const int dim = e % D;
+      const int agent = si.i_lo + e / D;
+      int r_begin = agent * p.G - si.row_lo, r_end = r_begin + p.G;
+      r_begin = r_begin < 0 ? 0 : r_begin;
+      r_end = r_end > si.rows ? si.rows : r_end;
+      for (int row = r_begin; row < r_end; ++row) {
+        float acc = mO[row * D + dim];
+#pragma unroll
+        for (int r = 0; r < RK; ++r) acc = fmaf(mZ[row * RK + r], bb[k][r], acc);
+        const float L = mL[row];
+        const float o = L > 0.f ? acc / L : 0.f;
+        const int grow = si.row_lo + row;
+        const int h = si.g * p.G + grow % p.G;
+        const size_t oi = (((size_t)si.s * p.N + agent) * p.Hq + h) * D + dim;
+        if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
+        else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+      }
+    }
+  }
+}
+
 template <int D, int NT, int RK>
 __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const DecodeSmem& lay, uint64_t* full,
                                  uint64_t* empty, volatile int* seq, volatile int* abort_flag, int* bcast,
@@ -346,16 +528,13 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   const int rbase = nw * 8;
   const int g8 = lane >> 2, t4 = lane & 3;
   const uint32_t ring_s = smem_u32(smem);
-  float* merge = reinterpret_cast<float*>(smem + lay.merge_off);
-  float* scw = reinterpret_cast<float*>(smem + lay.scw_off);
   int* a_sm = reinterpret_cast<int*>(smem + lay.a_off);
   const float NEG_INF = -INFINITY;
-  const long long C = gridDim.x;
-  const long long c = blockIdx.x;
 
   int stage = 0;
   uint32_t phase = 0;
   int ntile = 0;  // tiles seen by this CTA so far (all groups)
+  int sn = 0;     // segments of this CTA so far
 
   // Per-lane byte offsets of the ldmatrix rows inside a 128B-swizzled K/V
   // tile (64 keys x 64 dims per half): 16-byte chunk c of key row k sits at
@@ -372,6 +551,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     }
   }
 
+  uint32_t qf[KS][2];
   for (long long t = t_begin; t < t_end;) {
     Seg sg = make_seg(p, t, t_end, tid == 0);
     t += sg.hi - sg.lo;
@@ -380,21 +560,11 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     const int sl = sg.sl;
 
     if (tid < sg.n_ag) a_sm[tid] = load_offset(p, sg.s, sg.i_lo + tid, true);
-    // this warp's query rows as the B operand of S^T = K Q^T (kept in registers)
+    // this warp's query rows as the B operand of S^T = K Q^T (kept in registers;
+    // from the second segment on they were fetched during the previous merge)
     const int qrow = rbase + g8;  // row of this lane's B fragment
     const bool qvalid = qrow < sg.rows;
-    const __nv_bfloat16* qptr = nullptr;
-    if (qvalid) {
-      const int grow = sg.row_lo + qrow;
-      qptr = static_cast<const __nv_bfloat16*>(p.q) +
-             (((size_t)sg.s * p.N + grow / p.G) * p.Hq + sg.g * p.G + grow % p.G) * D;
-    }
-    uint32_t qf[KS][2];
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      qf[ks][0] = qvalid ? __ldg(reinterpret_cast<const unsigned int*>(qptr + ks * 16 + 2 * t4)) : 0u;
-      qf[ks][1] = qvalid ? __ldg(reinterpret_cast<const unsigned int*>(qptr + ks * 16 + 8 + 2 * t4)) : 0u;
-    }
+    if (sn == 0) load_q_frags<D>(p, sg, qrow, t4, qf);
     named_bar_sync(1, CT);
     int a_max = 0;
     for (int j = 0; j < sg.n_ag; ++j) a_max = max(a_max, a_sm[j]);
@@ -631,25 +801,22 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       if (lane == 0) mbar_arrive(&empty[my_stage]);
     }
 
-    // ---- the finishing epilogue needs, per (agent, dim) pair, the agent's B
-    // column B_i[:, g d + dim]; fetch this thread's first pairs now so the loads
-    // overlap the merge and the ticket round trip (B is small and L2-resident)
-    constexpr int PB = RK >= 32 ? 2 : 4;  // pairs per thread kept in registers
-    const int HD = p.Hkv * D;
-    const int n_pairs = sg.n_ag * D;
-    float bk[PB][RK];
-#pragma unroll
-    for (int k = 0; k < PB; ++k) {
-      const int e = tid + k * CT;
-      if (e < n_pairs) {
-        const uint16_t* bcol = static_cast<const uint16_t*>(p.b) + ((size_t)(sg.i_lo + e / D) * RK) * HD +
-                               (size_t)sg.g * D + e % D;
-#pragma unroll
-        for (int r = 0; r < RK; ++r) bk[k][r] = bf16_to_f32(__ldg(bcol + (size_t)r * HD));
-      }
+    // ---- segment end.  The next segment's query fragments are fetched now so
+    // that their latency overlaps the merge.  The addresses used here are
+    // formed here rather than kept live through the tile loop, and the last
+    // segment's B columns are loaded inside the finish rather than held in
+    // registers across the merge: the tile loop needs every register.
+    const bool last_seg = t >= t_end;
+    const int buf = sn & 1;
+    float* merge = reinterpret_cast<float*>(smem + lay.merge_off) + buf * REC;  // records alternate
+    uint64_t* rec_full = full + 2 * p.stages;
+    uint64_t* rec_free = rec_full + 2;
+    if (!last_seg) {
+      Seg nx = make_seg(p, t, t_end, false);
+      seg_rows(p, nx);
+      load_q_frags<D>(p, nx, rbase + g8, t4, qf);
     }
-
-    // ---- reduce l over the lanes that share a row; chain the groups into record 0
+    // reduce l over the lanes that share a row
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       float v = st.l[e];
@@ -658,6 +825,9 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       v += __shfl_xor_sync(0xffffffffu, v, 16);
       st.l[e] = v;
     }
+    // the record buffer of segment sn - 2 must have been released by the epilogue warp
+    if (sn >= 2) mbar_wait_bounded(&rec_free[buf], ((sn >> 1) - 1) & 1, abort_flag, p.flags);
+    // chain the owner groups into the record (same rows, different tiles)
     for (int src = NOG - 1; src >= 1; --src) {
       if (og == src) store_rows<D, RK>(st, merge, RP, rbase, g8, t4);
       named_bar_sync(1, CT);
@@ -666,146 +836,53 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     }
     if (og == 0) store_rows<D, RK>(st, merge, RP, rbase, g8, t4);
     named_bar_sync(1, CT);
-
-    // ---- publish or finish this item
-    const long long W = p.W;
-    const long long c_first = owner_cta((long long)sg.item * p.nt, W, C);
-    const long long c_last = owner_cta((long long)(sg.item + 1) * p.nt - 1, W, C);
-    const int segs = (int)(c_last - c_first + 1);
-    bool finish = true;
-    if (segs > 1) {
-      float* rec = p.partials + ((size_t)sg.item * p.max_segs + (size_t)(c - c_first)) * REC;
-      for (int e = tid * 4; e < REC; e += CT * 4)
-        __stcg(reinterpret_cast<float4*>(rec + e), *reinterpret_cast<const float4*>(merge + e));
-      named_bar_sync(1, CT);
-      if (tid == 0) {
-        __threadfence();
-        const int prev = atomicAdd(p.tickets + sg.item, 1);
-        const int last = prev == segs - 1;
-        if (last) p.tickets[sg.item] = 0;
-        *bcast = last;
-      }
-      named_bar_sync(1, CT);
-      finish = *bcast != 0;
-      if (finish) {
-        __threadfence();
-        const float* base = p.partials + (size_t)sg.item * p.max_segs * REC;
-        constexpr int E4 = RP * (D + RK) / 4;
-        constexpr int PER = (E4 + CT - 1) / CT;  // float4 elements of the record per thread
-        float4 acc[PER];
-#pragma unroll
-        for (int u = 0; u < PER; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j0 = 0; j0 < segs; j0 += SEG_CHUNK) {
-          const int nj = min(SEG_CHUNK, segs - j0);
-          // row maxima and sums of every record of the chunk: one round of loads
-          if (tid < RP) {
-            float mj[SEG_CHUNK], lj[SEG_CHUNK];
-#pragma unroll
-            for (int jj = 0; jj < SEG_CHUNK; ++jj) {
-              mj[jj] = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + tid) : NEG_INF;
-              lj[jj] = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + RP + tid) : 0.f;
-            }
-            if (j0 == 0) {
-              // the global maximum needs every record: this chunk's, then any further ones
-              float M = NEG_INF;
-#pragma unroll
-              for (int jj = 0; jj < SEG_CHUNK; ++jj) M = fmaxf(M, mj[jj]);
-              for (int j = SEG_CHUNK; j < segs; ++j) M = fmaxf(M, __ldcg(base + (size_t)j * REC + tid));
-              merge[tid] = M;
-              merge[RP + tid] = 0.f;
-            }
-            const float M = merge[tid];
-            float L = merge[RP + tid];
-#pragma unroll
-            for (int jj = 0; jj < SEG_CHUNK; ++jj) {
-              const float sc = (jj < nj && mj[jj] != NEG_INF) ? fast_exp2(mj[jj] - M) : 0.f;
-              scw[jj * RP + tid] = sc;
-              L += lj[jj] * sc;
-            }
-            merge[RP + tid] = L;
-          }
-          named_bar_sync(1, CT);
-          // O and Z of every record of the chunk: PER float4 loads per record, issued together
-          for (int jj = 0; jj < nj; ++jj) {
-            const float* rj = base + (size_t)(j0 + jj) * REC + 2 * RP;
-            float4 v[PER];
-#pragma unroll
-            for (int u = 0; u < PER; ++u) {
-              const int e4 = tid + u * CT;
-              v[u] = e4 < E4 ? __ldcg(reinterpret_cast<const float4*>(rj) + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < PER; ++u) {
-              const int e = (tid + u * CT) * 4;
-              if (e >= E4 * 4) continue;
-              const int row = e < RP * D ? e / D : (e - RP * D) / RK;
-              const float sc = scw[jj * RP + row];
-              acc[u].x += v[u].x * sc;
-              acc[u].y += v[u].y * sc;
-              acc[u].z += v[u].z * sc;
-              acc[u].w += v[u].w * sc;
-            }
-          }
-          named_bar_sync(1, CT);
-        }
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-          const int e4 = tid + u * CT;
-          if (e4 < E4) *reinterpret_cast<float4*>(merge + 2 * RP + e4 * 4) = acc[u];
-        }
-        named_bar_sync(1, CT);
-      }
+    if (!last_seg) {
+      // hand the record to the epilogue warp and go on streaming
+      if (tid == 0) mbar_arrive(&rec_full[buf]);
+    } else {
+      const SegInfo si = seg_info(p, sg);
+      float* scw = reinterpret_cast<float*>(smem + lay.scw_off);  // the consumers' half
+      finish_segment<D, NT, RK, CT, (RK >= 32 ? 2 : 4)>(p, si, merge, scw, bcast, tid, [] { named_bar_sync(1, CT); });
     }
-
-    if (finish) {
-      // out = (O + Z B_i,g) / l, once per row: the up-projection of Eq. 12.
-      // One thread per (agent, dim); the agent's B column serves all its GQA rows.
-      const float* mL = merge + RP;
-      const float* mO = merge + 2 * RP;
-      const float* mZ = mO + RP * D;
-      for (int e0 = tid; e0 < n_pairs; e0 += PB * CT) {
-#pragma unroll
-        for (int k = 0; k < PB; ++k) {
-          const int e = e0 + k * CT;
-          if (e >= n_pairs) continue;
-          const int dim = e % D;
-          const int agent = sg.i_lo + e / D;
-          float bcol[RK];
-          if (e0 == tid) {
-#pragma unroll
-            for (int r = 0; r < RK; ++r) bcol[r] = bk[k][r];
-          } else {  // pairs beyond the prefetched ones (many agents per KV head)
-            const uint16_t* bp = static_cast<const uint16_t*>(p.b) + ((size_t)agent * RK) * HD + (size_t)sg.g * D + dim;
-#pragma unroll
-            for (int r = 0; r < RK; ++r) bcol[r] = bf16_to_f32(__ldg(bp + (size_t)r * HD));
-          }
-          int r_begin = agent * p.G - sg.row_lo, r_end = r_begin + p.G;
-          r_begin = r_begin < 0 ? 0 : r_begin;
-          r_end = r_end > sg.rows ? sg.rows : r_end;
-          for (int row = r_begin; row < r_end; ++row) {
-            float acc = mO[row * D + dim];
-#pragma unroll
-            for (int r = 0; r < RK; ++r) acc = fmaf(mZ[row * RK + r], bcol[r], acc);
-            const float L = mL[row];
-            const float o = L > 0.f ? acc / L : 0.f;
-            const int grow = sg.row_lo + row;
-            const int h = sg.g * p.G + grow % p.G;
-            const size_t oi = (((size_t)sg.s * p.N + agent) * p.Hq + h) * D + dim;
-            if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
-            else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
-          }
-        }
-      }
-    }
-    named_bar_sync(1, CT);
+    ++sn;
   }
 }
 
-// Warp roles: warps 0 .. kDecodeGroups*NT-1 consume, the last warp produces.
+// The epilogue warp: publishes (and, as the last CTA of an item, combines and
+// finishes) the records of every segment of this CTA but the last, while the
+// consumer warps stream the next segment's tiles.
+template <int D, int NT, int RK>
+__device__ void decode_epilogue(const DecodeParams& p, uint8_t* smem, const DecodeSmem& lay, uint64_t* rec_full,
+                                uint64_t* rec_free, volatile int* abort_flag, int* bcast, long long t_begin,
+                                long long t_end) {
+  constexpr int RP = NT * 8;
+  constexpr int REC = RP * (D + RK + 2);
+  const int lane = threadIdx.x & 31;
+  float* merge0 = reinterpret_cast<float*>(smem + lay.merge_off);
+  float* scw = reinterpret_cast<float*>(smem + lay.scw_off) + 8 * RP;  // the epilogue warp's half
+  int sn = 0;
+  for (long long t = t_begin; t < t_end;) {
+    Seg sg = make_seg(p, t, t_end, false);
+    t += sg.hi - sg.lo;
+    seg_rows(p, sg);
+    if (t >= t_end) break;  // the consumers finish the last segment
+    const int buf = sn & 1;
+    if (!mbar_wait_bounded(&rec_full[buf], (sn >> 1) & 1, abort_flag, p.flags)) break;
+    const SegInfo si = seg_info(p, sg);
+    finish_segment<D, NT, RK, 32, (RK >= 32 ? 1 : 2)>(p, si, merge0 + buf * REC, scw, bcast, lane,
+                                                      [] { __syncwarp(); });
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&rec_free[buf]);
+    ++sn;
+  }
+}
+
+// Warp roles: warps 0 .. kDecodeGroups*NT-1 consume, then one producer warp
+// and one epilogue warp.
 template <int NT>
 struct Roles {
   static constexpr int CONSUMER_WARPS = kDecodeGroups * NT;
-  static constexpr int THREADS = (CONSUMER_WARPS + 1) * 32;
+  static constexpr int THREADS = (CONSUMER_WARPS + 2) * 32;
 };
 
 template <int D, int NT, int RK>
@@ -817,19 +894,26 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
   const DecodeSmem lay = decode_smem_plan(D, NT, RK, p.n_u_slots, p.stages);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bar_off);
   uint64_t* empty = full + p.stages;
-  volatile int* seq = reinterpret_cast<volatile int*>(empty + p.stages);
+  uint64_t* rec_full = empty + p.stages;
+  uint64_t* rec_free = rec_full + 2;
+  volatile int* seq = reinterpret_cast<volatile int*>(rec_free + 2);
   volatile int* abort_flag = seq + p.stages;
-  int* bcast = const_cast<int*>(abort_flag) + 1;
+  int* bcast = const_cast<int*>(abort_flag) + 1;  // [0] consumers, [1] epilogue warp
   const int warp = threadIdx.x >> 5;
   constexpr int PRODUCER = Roles<NT>::CONSUMER_WARPS;
+  constexpr int EPILOGUE = PRODUCER + 1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NT);  // the NT warps of the group that owns the tile
       seq[s] = -1;
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&rec_full[b], 1);
+      mbar_init(&rec_free[b], 1);
+    }
     *abort_flag = 0;
-    *bcast = 0;
+    bcast[0] = bcast[1] = 0;
     fence_barrier_init();
   }
   if (warp == PRODUCER && (threadIdx.x & 31) == 0) {
@@ -846,6 +930,8 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
   if (warp == PRODUCER) {
     decode_producer<D, RK>(p, &tmK, &tmV, &tmU, smem, lay.stage_bytes, full, empty, seq, abort_flag, t_begin,
                            t_end);
+  } else if (warp == EPILOGUE) {
+    decode_epilogue<D, NT, RK>(p, smem, lay, rec_full, rec_free, abort_flag, bcast + 1, t_begin, t_end);
   } else {
     decode_consumers<D, NT, RK>(p, smem, lay, full, empty, seq, abort_flag, bcast, t_begin, t_end);
   }

@@ -73,10 +73,10 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int D, int NT, int RK, in
   s.ring_bytes = stages * s.stage_bytes;
   s.merge_off = s.ring_bytes;
   const int rec = RP * (D + RK + 2) * 4;
-  s.scw_off = s.merge_off + rec;
-  s.a_off = s.scw_off + 8 * RP * 4;
+  s.scw_off = s.merge_off + 2 * rec;      // two records: segments alternate
+  s.a_off = s.scw_off + 2 * 8 * RP * 4;   // scale tables of the consumers and of the epilogue warp
   s.bar_off = round_up(s.a_off + kMaxAgents * 4, 16);
-  s.total = s.bar_off + 2 * stages * 8 + stages * 4 + 64;
+  s.total = s.bar_off + (2 * stages + 4) * 8 + stages * 4 + 64;
   return s;
 }
 
