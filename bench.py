@@ -53,6 +53,52 @@ def _peaks():
 
 
 # ---------------------------------------------------------------------------
+# DRAM traffic from the committed ncu summaries
+# ---------------------------------------------------------------------------
+
+# Sources that decide what a kernel reads and writes.  A summary under
+# profiles/ records their sha256 at capture time; its DRAM bytes are reported
+# only while the sources still hash the same (else the counters are stale).
+KERNEL_SOURCES = {
+    "decode_kernel": ["decode.cu", "common.cuh", "lrkv_internal.h", "lrkv_api.cu"],
+    "prefill_kernel": ["prefill.cu", "prefill.h", "common.cuh", "lrkv_internal.h", "lrkv_api.cu"],
+}
+
+
+def kernel_sources_sha256(kernel):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "lora_shared_kv_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from
+    profiles/<kernel>__<workload>.md, or None when there is no summary or the
+    kernel's sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.md")
+    try:
+        with open(path) as f:
+            text = f.read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        line = line.strip().lstrip("-* ").strip()
+        if ":" in line:
+            k, v = line.split(":", 1)
+            fields[k.strip().strip("`")] = v.strip().strip("`")
+    try:
+        if fields.get("sources_sha256") != kernel_sources_sha256(kernel):
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError, OSError):
+        return None
+
+
+# ---------------------------------------------------------------------------
 # algorithmic bytes
 # ---------------------------------------------------------------------------
 
@@ -316,6 +362,7 @@ def bench_prefill(device, steps=20, warmup=5):
     tf = flops / (ms * 1e-3) / 1e12
     return {"workload": cfg.name, "ms_per_step": ms, "tflops": tf, "flops_per_step": flops,
             "peak_tflops": bf16_peak, "frac": tf / bf16_peak, "peak_source": src,
+            "prefill_kernel_traffic": profiled_traffic("prefill_kernel", cfg.name),
             "l2": "256 MB flush before each step"}
 
 
@@ -385,7 +432,7 @@ def main():
     per_launch_ms = ms_step / runner.launches_per_step
     achieved = lb / (per_launch_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-            "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+            "traffic": profiled_traffic("decode_kernel", cfg.name), "peak_source": f"{peak_src} copy bandwidth",
             "kernel": "decode_kernel", "algorithmic_bytes_per_launch": lb,
             "launch_ms": per_launch_ms, "launch_ms_note": "step time / launches per step (gaps included)"}
 

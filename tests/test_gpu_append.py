@@ -23,6 +23,8 @@ def _bits(t):
     (37, 1536, 16, 3, 100, 200),
     (512, 2048, 32, 4, 16384, 16896),
     (5, 65, 16, 1, 3, 8),
+    (70, 100, 8, 2, 0, 100),
+    (17, 300, 32, 1, 40, 64),
 ])
 def test_append_bit_exact(T, Dm, r, n_a, start, cap):
     g = torch.Generator(device=DEV)
