@@ -15,23 +15,25 @@ namespace lrkv {
 
 namespace {
 
-// A block owns TB tokens x all r columns of one agent; a thread owns one token
-// and 4 adjacent columns (4 independent fmaf chains).  X and A are staged in
-// shared memory as fp32 one k-chunk at a time; the next chunk's global loads
-// are issued into registers before the current chunk's FMAs, so their latency
-// hides behind the arithmetic.  Each output still sums k = 0 .. Dm-1 in order.
+// A warp owns 32 consecutive tokens (one per lane) and a group of 8 columns:
+// each thread runs 8 independent fmaf chains.  Per k a lane reads its own
+// x[t, k] (a conflict-free 32-bit load) and the group's 8 A values (two
+// 128-bit loads every lane shares: broadcasts), so shared memory serves 8
+// FMAs per lane with 3 loads.  A block of 4 warps covers TB tokens x all r
+// columns of one agent; X (transposed, k-major) and A are staged as fp32 one
+// k-chunk at a time, the next chunk's global loads held in registers while the
+// current chunk is consumed.  Each output still sums k = 0 .. Dm-1 in order.
 constexpr int APP_THREADS = 128;
-constexpr int X_PER_CHUNK = 2048;  // X elements staged per chunk (TB x KC)
+constexpr int KC = 64;  // k per chunk
 
 template <int R>
 struct AppShape {
-  static constexpr int CG = R / 4;                    // column groups of 4
-  static constexpr int TB = APP_THREADS / CG;         // tokens per block
-  static constexpr int KC = X_PER_CHUNK / TB;         // k per chunk
-  static constexpr int XL = X_PER_CHUNK / APP_THREADS;  // X loads per thread per chunk
+  static constexpr int CG = R / 8;                      // column groups of 8
+  static constexpr int TB = (APP_THREADS / 32) / CG * 32;  // tokens per block
+  static constexpr int XS = TB + 1;                     // padded k-row of the transposed X chunk
+  static constexpr int XL = TB * KC / APP_THREADS;      // X loads per thread per chunk
   static constexpr int AL = KC * R / APP_THREADS;       // A loads per thread per chunk
-  static constexpr int XS = KC + 1;                   // padded X row (conflict-free column reads)
-  static_assert(APP_THREADS % KC == 0 && X_PER_CHUNK % APP_THREADS == 0 && (KC * R) % APP_THREADS == 0, "shape");
+  static_assert(APP_THREADS % KC == 0 && (TB * KC) % APP_THREADS == 0 && (KC * R) % APP_THREADS == 0, "shape");
 };
 
 template <int R>
@@ -40,20 +42,19 @@ __global__ void __launch_bounds__(APP_THREADS)
                   __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st, int session,
                   int start_row) {
   using S = AppShape<R>;
-  __shared__ float xs[S::TB * S::XS];
-  __shared__ __align__(16) float as[S::KC * R];
-  const int tid = threadIdx.x;
-  const int tok = tid / S::CG;       // token within the block
-  const int col = (tid % S::CG) * 4;  // first of this thread's 4 columns
+  __shared__ float xs[KC * S::XS];                // xs[k * XS + token]
+  __shared__ __align__(16) float as[KC * R];      // as[k * R + column]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cg = warp % S::CG;                    // this warp's 8 columns: [8 cg, 8 cg + 8)
+  const int tl = (warp / S::CG) * 32 + lane;      // this thread's token within the block
   const int agent = blockIdx.y;
   const int t0 = blockIdx.x * S::TB;
   const uint16_t* a_ag = a + (size_t)agent * Dm * R;
 
-  // chunk element e = tid + i * APP_THREADS sits at row e / KC, k e % KC; as
-  // APP_THREADS is a multiple of KC, a thread's k is fixed and its rows step by
-  // APP_THREADS / KC
-  constexpr int RSTEP = APP_THREADS / S::KC;
-  const int my_kk = tid % S::KC, my_row = tid / S::KC;
+  // staging: chunk element e = tid + i * APP_THREADS of X sits at token e / KC,
+  // k e % KC; as APP_THREADS is a multiple of KC a thread's k is fixed
+  constexpr int RSTEP = APP_THREADS / KC;
+  const int my_kk = tid % KC, my_row = tid / KC;
   const uint16_t* xp = x + (size_t)(t0 + my_row) * Dm + my_kk;
   uint16_t xr[S::XL], ar[S::AL];
   auto load_chunk = [&](int k0) {
@@ -67,46 +68,55 @@ __global__ void __launch_bounds__(APP_THREADS)
       ar[i] = (k0 + e / R < Dm) ? __ldg(a_ag + (size_t)k0 * R + e) : (uint16_t)0;
     }
   };
-  float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.0f;
+  const float* xcol = xs + tl;
+  const float4* acol = reinterpret_cast<const float4*>(as + cg * 8);
   load_chunk(0);
-  for (int k0 = 0; k0 < Dm; k0 += S::KC) {
+  for (int k0 = 0; k0 < Dm; k0 += KC) {
     __syncthreads();  // the previous chunk's reads are done
 #pragma unroll
-    for (int i = 0; i < S::XL; ++i) xs[(my_row + i * RSTEP) * S::XS + my_kk] = __uint_as_float((uint32_t)xr[i] << 16);
+    for (int i = 0; i < S::XL; ++i) xs[my_kk * S::XS + my_row + i * RSTEP] = __uint_as_float((uint32_t)xr[i] << 16);
 #pragma unroll
     for (int i = 0; i < S::AL; ++i) as[tid + i * APP_THREADS] = __uint_as_float((uint32_t)ar[i] << 16);
     __syncthreads();
-    if (k0 + S::KC < Dm) load_chunk(k0 + S::KC);
-    const int kc = min(S::KC, Dm - k0);
-    const float* xrow = xs + tok * S::XS;
-    if (kc == S::KC) {
-#pragma unroll 8
-      for (int kk = 0; kk < S::KC; ++kk) {
-        const float xv = xrow[kk];
-        const float4 av = *reinterpret_cast<const float4*>(as + kk * R + col);
-        acc0 = fmaf(xv, av.x, acc0);
-        acc1 = fmaf(xv, av.y, acc1);
-        acc2 = fmaf(xv, av.z, acc2);
-        acc3 = fmaf(xv, av.w, acc3);
+    if (k0 + KC < Dm) load_chunk(k0 + KC);
+    const int kc = min(KC, Dm - k0);
+    if (kc == KC) {
+#pragma unroll
+      for (int kk = 0; kk < KC; ++kk) {
+        const float xv = xcol[kk * S::XS];
+        const float4 a0 = acol[kk * (R / 4)], a1 = acol[kk * (R / 4) + 1];
+        acc[0] = fmaf(xv, a0.x, acc[0]);
+        acc[1] = fmaf(xv, a0.y, acc[1]);
+        acc[2] = fmaf(xv, a0.z, acc[2]);
+        acc[3] = fmaf(xv, a0.w, acc[3]);
+        acc[4] = fmaf(xv, a1.x, acc[4]);
+        acc[5] = fmaf(xv, a1.y, acc[5]);
+        acc[6] = fmaf(xv, a1.z, acc[6]);
+        acc[7] = fmaf(xv, a1.w, acc[7]);
       }
     } else {
       for (int kk = 0; kk < kc; ++kk) {
-        const float xv = xrow[kk];
-        const float4 av = *reinterpret_cast<const float4*>(as + kk * R + col);
-        acc0 = fmaf(xv, av.x, acc0);
-        acc1 = fmaf(xv, av.y, acc1);
-        acc2 = fmaf(xv, av.z, acc2);
-        acc3 = fmaf(xv, av.w, acc3);
+        const float xv = xcol[kk * S::XS];
+        const float4 a0 = acol[kk * (R / 4)], a1 = acol[kk * (R / 4) + 1];
+        acc[0] = fmaf(xv, a0.x, acc[0]);
+        acc[1] = fmaf(xv, a0.y, acc[1]);
+        acc[2] = fmaf(xv, a0.z, acc[2]);
+        acc[3] = fmaf(xv, a0.w, acc[3]);
+        acc[4] = fmaf(xv, a1.x, acc[4]);
+        acc[5] = fmaf(xv, a1.y, acc[5]);
+        acc[6] = fmaf(xv, a1.z, acc[6]);
+        acc[7] = fmaf(xv, a1.w, acc[7]);
       }
     }
   }
-  const int t = t0 + tok;
+  const int t = t0 + tl;
   if (t < T) {
-    __nv_bfloat16* dst = u + (size_t)session * u_ss + (size_t)agent * u_sa + (size_t)(start_row + t) * u_st + col;
-    dst[0] = __float2bfloat16_rn(acc0);
-    dst[1] = __float2bfloat16_rn(acc1);
-    dst[2] = __float2bfloat16_rn(acc2);
-    dst[3] = __float2bfloat16_rn(acc3);
+    __nv_bfloat16* dst = u + (size_t)session * u_ss + (size_t)agent * u_sa + (size_t)(start_row + t) * u_st + cg * 8;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) dst[c] = __float2bfloat16_rn(acc[c]);
   }
 }
 

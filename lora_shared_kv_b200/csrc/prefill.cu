@@ -17,12 +17,18 @@
 //                 K into a 3-stage ring (a stage frees as soon as its S is
 //                 computed) and of V and U into a 2-stage ring.
 //   warp 1        TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into a
-//                 double-buffered S in TMEM; then O += P_j V_j and
-//                 Z += P_j U_j with P_j read from TMEM (it overwrites S_j).
-//   warps 4..7    softmax and epilogue, one row per thread (TMEM lane = row):
-//                 row max/sum need no shuffles; the reference max moves only
-//                 when a block exceeds it by 2^8, and only then is O rescaled
-//                 in TMEM.
+//                 double-buffered S in TMEM; then [O | Z] += P_j [V_j | U_j]
+//                 with P_j read from TMEM (it overwrites S_j): V_j and U_j lie
+//                 side by side in shared memory as one operand of d + r
+//                 columns, so a k-step is one MMA of N = d + r (N = d for the
+//                 blocks wholly before the aLoRA offset, whose U is not read).
+//   warps 4..11   softmax and epilogue in two warpgroups, one per half of the
+//                 block's 128 keys; a thread owns one row (TMEM lane) of its
+//                 half.  The halves agree on each row's reference max through
+//                 shared memory and keep separate partial sums.  The reference
+//                 max moves only when a block exceeds it by 2^8, and only then
+//                 are O and Z rescaled in TMEM (each half rescales its share of
+//                 the columns).  The epilogue splits the output columns.
 #include <float.h>
 #include <math.h>
 
@@ -37,7 +43,8 @@ constexpr int BM = 128;   // rows per tile (TMEM lanes)
 constexpr int BN = 128;   // keys per block
 constexpr int KST = 3;    // K ring: a stage is free once S = Q K^T has been computed
 constexpr int VST = 2;    // V/U ring: a stage is free once O += P V and Z += P U are done
-constexpr int THREADS = 256;
+constexpr int THREADS = 384;  // producer, MMA, 2 idle, 2 softmax warpgroups
+constexpr int SMX_THREADS = 256;  // the two softmax warpgroups (named barrier 1)
 constexpr uint32_t TMEM_COLS = 512;
 
 template <int D, int RK>
@@ -52,7 +59,8 @@ struct PrefillLayout {
   static constexpr int K_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int V_OFF = K_OFF + KST * K_BYTES;
   static constexpr int BAR_OFF = V_OFF + VST * V_STAGE;
-  static constexpr int TOTAL = BAR_OFF + 256;
+  static constexpr int XCH_OFF = BAR_OFF + 256;  // row max [2 blocks][2 halves][BM], row sum [2 halves][BM]
+  static constexpr int TOTAL = XCH_OFF + 6 * BM * 4;
   // TMEM columns
   static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_Z = 2 * BN + D;
   static_assert(2 * BN + D + RK <= (int)TMEM_COLS, "TMEM budget");
@@ -119,7 +127,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], 4);
+      mbar_init(&bars->p_full[b], 8);  // every softmax warp
     }
     mbar_init(&bars->o_ready[0], 1);
     mbar_init(&bars->o_ready[1], 1);
@@ -208,14 +216,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t* Us = Vs + Lay::K_BYTES;
         mbar_arrive_expect_tx(&bars->v_full[vs_], Lay::K_BYTES + (need_u ? Lay::U_BYTES : 0));
 #pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh) {
+        for (int at = 0; at < D / RK; ++at) {  // RK-wide atoms of V, each [BN keys][RK dims]
           if (!p.page_table) {
-            tma_load_4d(Vs + hh * (BN * 128), &tmV, &bars->v_full[vs_], hh * 64, jb * BN, g, p.session, pol_kv);
+            tma_load_4d(Vs + at * Lay::U_BYTES, &tmV, &bars->v_full[vs_], at * RK, jb * BN, g, p.session, pol_kv);
           } else {
 #pragma unroll
             for (int pg = 0; pg < BN / 64; ++pg)
-              tma_load_4d(Vs + hh * (BN * 128) + pg * (64 * 128), &tmV, &bars->v_full[vs_], hh * 64, 0, g, phys[pg],
-                          pol_kv);
+              tma_load_4d(Vs + at * Lay::U_BYTES + pg * (64 * RK * 2), &tmV, &bars->v_full[vs_], at * RK, 0, g,
+                          phys[pg], pol_kv);
           }
         }
         if (need_u) tma_load_4d(Us, &tmU, &bars->v_full[vs_], 0, jb * BN, u_slot, p.session, pol_kv);
@@ -240,13 +248,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     constexpr uint32_t ID_QK = umma_idesc_bf16(BM, BN, 0, 0);
-    constexpr uint32_t ID_PV = umma_idesc_bf16(BM, D, 0, 1);
-    constexpr uint32_t ID_PZ = umma_idesc_bf16(BM, RK, 0, 1);
-    constexpr uint32_t U_LAYOUT = RK == 32 ? 4u : 6u;       // 64B / 32B swizzle, rows of RK bf16
-    constexpr uint32_t U_SBO = 8 * RK * 2;                  // eight key rows
+    constexpr uint32_t ID_PV = umma_idesc_bf16(BM, D, 0, 1);        // [O] += P V
+    constexpr uint32_t ID_PVU = umma_idesc_bf16(BM, D + RK, 0, 1);  // [O | Z] += P [V | U]
+    constexpr uint32_t VU_LAYOUT = RK == 32 ? 4u : 6u;  // 64B / 32B swizzle: atoms of RK bf16 per key row
+    constexpr uint32_t VU_LBO = Lay::U_BYTES;           // next atom along d + r
+    constexpr uint32_t VU_SBO = 8 * RK * 2;             // next eight key rows
     const uint32_t q_base = smem_u32(smem + Lay::Q_OFF);
     bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, p.flags);
-    bool z_started = false;
     for (int jb = 0; jb <= nb && ok; ++jb) {
       if (jb < nb) {
         const int st = jb % KST;
@@ -288,87 +296,99 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
           tc_fence_after();
           const uint32_t v_base = smem_u32(smem + Lay::V_OFF + st * Lay::V_STAGE);
-          const uint32_t u_base = smem_u32(Us);
           const uint32_t a_p = tmem + (j & 1 ? Lay::COL_S1 : Lay::COL_S0);
+          const uint32_t id = u_used ? ID_PVU : ID_PV;  // Z (zeroed at the start) accumulates from its first block on
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t b = umma_desc(v_base + kk * 2048, BN * 128, 1024, 2);
-            umma_ts(tmem + Lay::COL_O, a_p + kk * 8, b, ID_PV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          if (u_used) {
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              const uint64_t b = umma_desc(u_base + kk * (16 * RK * 2), 16, U_SBO, U_LAYOUT);
-              umma_ts(tmem + Lay::COL_Z, a_p + kk * 8, b, ID_PZ, (z_started || kk > 0) ? 1u : 0u);
-            }
+            const uint64_t b = umma_desc(v_base + kk * (16 * RK * 2), VU_LBO, VU_SBO, VU_LAYOUT);
+            umma_ts(tmem + Lay::COL_O, a_p + kk * 8, b, id, (j > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bars->v_empty[st]);
           umma_commit(&bars->o_ready[j & 1]);
         }
-        if (u_used) z_started = true;
         __syncwarp();
       }
     }
   } else if (warp >= 4) {
-    // ======================= softmax + epilogue =======================
-    const int row = threadIdx.x - 128;         // TMEM lane and S/O row
+    // ======================= softmax + epilogue (two warpgroups) =======================
+    const int wg = (warp - 4) >> 2;           // key half of every block
+    const int row = (warp & 3) * 32 + lane;   // TMEM lane and S/O row
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+    constexpr int HB = BN / 2;                // keys per half
+    const int c0 = wg * HB;
+    float* xmax = reinterpret_cast<float*>(smem + Lay::XCH_OFF);  // [blk & 1][half][row]
+    float* xsum = xmax + 4 * BM;                                  // [half][row]
     const int jj = row / p.G, hh = row % p.G;
     const int token = j0 + jj;
     const int limit = p.L0 + token;            // last visible key of this row
     const float NEG_INF = -INFINITY;
     float m_ref = NEG_INF, l = 0.f;
     bool ok = true;
-    for (int jb = 0; jb < nb && ok; ++jb) {
-      ok = mbar_wait_bounded(&bars->s_full[jb & 1], (jb >> 1) & 1, abort_flag, p.flags);
+    if (wg == 1) {
+      // Z starts at zero: the MMA of the first block that reads U accumulates into it
+      // (a P [V | U] MMA has one accumulate flag for O and Z)
+      uint32_t zero[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) zero[e] = 0u;
+      if constexpr (RK == 32) tmem_st32(tmem + lane_addr + Lay::COL_Z, zero);
+      else tmem_st16(tmem + lane_addr + Lay::COL_Z, zero);
+      tmem_wait_st();
+    }
+    // Both warpgroups pass the same named barriers whatever happens: after a
+    // failed wait they skip the waits, not the barriers.
+    for (int jb = 0; jb < nb; ++jb) {
+      if (ok) ok = mbar_wait_bounded(&bars->s_full[jb & 1], (jb >> 1) & 1, abort_flag, p.flags);
       tc_fence_after();
       const uint32_t s_col = jb & 1 ? Lay::COL_S1 : Lay::COL_S0;
-      float x[BN];
+      float x[HB];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tmem + lane_addr + s_col + c * 32, reinterpret_cast<uint32_t*>(x) + c * 32);
+      for (int c = 0; c < HB / 32; ++c)
+        tmem_ld32(tmem + lane_addr + s_col + c0 + c * 32, reinterpret_cast<uint32_t*>(x) + c * 32);
       tmem_wait_ld();
-      const int key0 = jb * BN;
-      const bool diag = key0 + BN - 1 > p.L0 + j0;  // some key of the block is past some row's limit
-      if (diag) {
+      const int key0 = jb * BN + c0;
+      if (key0 + HB - 1 > p.L0 + j0) {  // some key of the half is past some row's limit
 #pragma unroll
-        for (int cc = 0; cc < BN; ++cc) x[cc] = key0 + cc <= limit ? x[cc] : NEG_INF;
+        for (int cc = 0; cc < HB; ++cc) x[cc] = key0 + cc <= limit ? x[cc] : NEG_INF;
       }
-      // row max over the block: eight independent chains, then a tree
+      // row max over the half: eight independent chains, then a tree; then the other half's
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = x[e];
 #pragma unroll
-      for (int cc = 8; cc < BN; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], x[cc]);
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int cc = 8; cc < HB; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], x[cc]);
+      float* xm = xmax + (jb & 1) * 2 * BM;
+      xm[wg * BM + row] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      named_bar_sync(1, SMX_THREADS);  // also: both halves have read their S columns
+      float mx = fmaxf(xm[row], xm[BM + row]);
       mx *= p.scale_log2;  // the scale is positive: the max commutes with it
       const bool need = mx > m_ref + 8.f;
-      if (__any_sync(0xffffffffu, need)) {
+      if (__any_sync(0xffffffffu, need)) {  // the same vote in both halves (same rows, same values)
         const float m_new = fmaxf(m_ref, mx);
         const float alpha = m_new == NEG_INF ? 1.f : fast_exp2(m_ref - m_new);
         if (jb > 0) {
-          // O and Z hold the blocks before this one: rescale them in TMEM once PV_{jb-1} is done
-          ok = mbar_wait_bounded(&bars->o_ready[(jb - 1) & 1], ((jb - 1) >> 1) & 1, abort_flag, p.flags);
+          // O and Z hold the blocks before this one: rescale this half's share of
+          // their columns in TMEM once PV_{jb-1} is done
+          if (ok) ok = mbar_wait_bounded(&bars->o_ready[(jb - 1) & 1], ((jb - 1) >> 1) & 1, abort_flag, p.flags);
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < (D + RK) / 32; ++c) {
+          for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
             uint32_t r[32];
-            const uint32_t col = Lay::COL_O + c * 32;
-            tmem_ld32(tmem + lane_addr + col, r);
+            tmem_ld32(tmem + lane_addr + Lay::COL_O + c * 32, r);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(tmem + lane_addr + col, r);
+            tmem_st32(tmem + lane_addr + Lay::COL_O + c * 32, r);
           }
-          if (RK % 32 != 0) {  // RK = 16: the last 16 columns (the load overlaps the chunk just stored)
-            tmem_wait_st();
-            uint32_t r[32];
-            const uint32_t col = Lay::COL_O + ((D + RK) / 32) * 32 - 16;
-            tmem_ld32(tmem + lane_addr + col, r);
+          if (wg == 1) {  // Z
+            uint32_t r[RK];
+            if constexpr (RK == 32) tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);
+            else tmem_ld16(tmem + lane_addr + Lay::COL_Z, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 16; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(tmem + lane_addr + col, r);
+            for (int e = 0; e < RK; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            if constexpr (RK == 32) tmem_st32(tmem + lane_addr + Lay::COL_Z, r);
+            else tmem_st16(tmem + lane_addr + Lay::COL_Z, r);
           }
           tmem_wait_st();
         }
@@ -376,10 +396,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_ref = m_new;
       }
       const float mu = m_ref == NEG_INF ? 0.f : m_ref;
-      uint32_t pk[BN / 2];
+      uint32_t pk[HB / 2];
       float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int cc = 0; cc < BN / 2; ++cc) {
+      for (int cc = 0; cc < HB / 2; ++cc) {
         const float p0 = fast_exp2(fmaf(x[2 * cc], p.scale_log2, -mu));
         const float p1 = fast_exp2(fmaf(x[2 * cc + 1], p.scale_log2, -mu));
         pk[cc] = pack_bf16x2(p0, p1);
@@ -387,31 +407,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         ls[cc & 7] += bf16_lo(pk[cc]) + bf16_hi(pk[cc]);
       }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-#pragma unroll
-      for (int c = 0; c < BN / 64; ++c) tmem_st32(tmem + lane_addr + s_col + c * 32, pk + c * 32);
+      // P of keys [c0, c0 + 64) as bf16 pairs: TMEM columns s_col + c0 / 2 + [0, 32)
+      tmem_st32(tmem + lane_addr + s_col + c0 / 2, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[jb & 1]);
     }
-    // ---- epilogue: out = (O + Z B_i,g) / l
+    // ---- epilogue: out = (O + Z B_i,g) / l, each half writes half of the columns
+    xsum[wg * BM + row] = l;
     if (ok) ok = mbar_wait_bounded(&bars->o_ready[(nb - 1) & 1], ((nb - 1) >> 1) & 1, abort_flag, p.flags);
+    named_bar_sync(1, SMX_THREADS);
+    l = xsum[row] + xsum[BM + row];
     tc_fence_after();
-    const bool z_used = a_i < key_end;  // some block accumulated Z
     float z[RK];
     {
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_addr + Lay::COL_Z - (RK == 16 ? 16 : 0), r);
+      uint32_t r[RK];
+      if constexpr (RK == 32) tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);
+      else tmem_ld16(tmem + lane_addr + Lay::COL_Z, r);
       tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < RK; ++k) z[k] = z_used ? __uint_as_float(r[(RK == 16 ? 16 : 0) + k]) : 0.f;
+      for (int k = 0; k < RK; ++k) z[k] = __uint_as_float(r[k]);
     }
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const bool write = token < p.T && ok;
     const int h = g * p.G + hh;
     const uint16_t* bs = reinterpret_cast<const uint16_t*>(smem + Lay::B_OFF);
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
       uint32_t r[32];
       tmem_ld32(tmem + lane_addr + Lay::COL_O + c * 32, r);
       tmem_wait_ld();
