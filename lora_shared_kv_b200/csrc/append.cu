@@ -38,7 +38,7 @@ struct AppShape {
 
 template <int R>
 __global__ void __launch_bounds__(APP_THREADS)
-    append_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int T, int Dm,
+    append_kernel_generic(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int T, int Dm,
                   __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st, int session,
                   int start_row) {
   using S = AppShape<R>;
@@ -121,12 +121,135 @@ __global__ void __launch_bounds__(APP_THREADS)
 }
 
 template <int R>
-void launch_r(const void* x, const void* a, int n_a, int T, int Dm, void* u, long long u_ss, long long u_sa,
+void launch_generic(const void* x, const void* a, int n_a, int T, int Dm, void* u, long long u_ss, long long u_sa,
               long long u_st, int session, int start_row, cudaStream_t stream) {
   dim3 grid((T + AppShape<R>::TB - 1) / AppShape<R>::TB, n_a);
-  append_kernel<R><<<grid, APP_THREADS, 0, stream>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(a),
+  append_kernel_generic<R><<<grid, APP_THREADS, 0, stream>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(a),
                                                      T, Dm, static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st,
                                                      session, start_row);
+}
+
+// ---------------------------------------------------------------------------
+// Fast path (Dm a multiple of 8, x and a 16-byte aligned): a warp owns 32
+// tokens (one per lane) x 4 columns, so a lane runs 4 fmaf chains and a block
+// of 4 warps covers 32 tokens x 16 columns (64 x 8 when r = 8).  X and A
+// k-chunks stream through a 4-stage cp.async ring, so three chunks are in
+// flight while one is consumed; a lane reads 8 k of its token's X row with one
+// 128-bit load (rows padded to 144 B: conflict-free) and each k's 4 A values
+// (converted to fp32 once per chunk) with one broadcast load.
+// ---------------------------------------------------------------------------
+constexpr int F_NS = 4;   // ring stages
+constexpr int F_KC = 64;  // k per chunk
+constexpr int F_XP = F_KC + 8;  // X row pitch in bf16 (144 B)
+
+template <int R>
+struct FastShape {
+  static constexpr int CGB = R / 4 < 4 ? R / 4 : 4;  // 4-column groups per block
+  static constexpr int TGB = 4 / CGB;                 // 32-token groups per block
+  static constexpr int TB = 32 * TGB;                 // tokens per block
+  static constexpr int CB = 4 * CGB;                  // columns per block
+  static constexpr int NCB = R / CB;                  // column blocks
+  static constexpr int XCP = TB * (F_KC / 8);         // 16-byte X copies per chunk
+  static constexpr int ACP = F_KC * CB / 8;           // 16-byte A copies per chunk
+  static_assert(XCP % APP_THREADS == 0 && ACP <= APP_THREADS && (F_KC * CB) % APP_THREADS == 0, "shape");
+};
+
+template <int R>
+__global__ void __launch_bounds__(APP_THREADS)
+    append_kernel_fast(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int T, int Dm,
+                       __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st, int session,
+                       int start_row) {
+  using S = FastShape<R>;
+  __shared__ __align__(16) uint16_t xr[F_NS][S::TB * F_XP];
+  __shared__ __align__(16) uint16_t ar[F_NS][F_KC * S::CB];
+  __shared__ __align__(16) float af[F_KC * S::CB];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cg = warp % S::CGB;
+  const int tl = (warp / S::CGB) * 32 + lane;  // token within the block
+  const int agent = blockIdx.y;
+  const int t0 = blockIdx.x * S::TB;
+  const int c0 = blockIdx.z * S::CB;           // first column of the block
+  const uint16_t* a_ag = a + (size_t)agent * Dm * R;
+  const int n_chunks = (Dm + F_KC - 1) / F_KC;
+
+  auto issue = [&](int c) {
+    if (c < n_chunks) {
+      const int k0 = c * F_KC, st = c % F_NS;
+#pragma unroll
+      for (int i = 0; i < S::XCP / APP_THREADS; ++i) {
+        const int e = tid + i * APP_THREADS;
+        const int row = e / (F_KC / 8), seg = e % (F_KC / 8);
+        const bool ok = t0 + row < T && k0 + seg * 8 < Dm;
+        const uint16_t* src = ok ? x + (size_t)(t0 + row) * Dm + k0 + seg * 8 : x;
+        cp_async16(&xr[st][row * F_XP + seg * 8], src, ok ? 16u : 0u);
+      }
+      if (tid < S::ACP) {
+        const int row = tid / (S::CB / 8), seg = tid % (S::CB / 8);
+        const bool ok = k0 + row < Dm;
+        const uint16_t* src = ok ? a_ag + (size_t)(k0 + row) * R + c0 + seg * 8 : a_ag;
+        cp_async16(&ar[st][row * S::CB + seg * 8], src, ok ? 16u : 0u);
+      }
+    }
+    cp_async_commit();  // one group per chunk index, empty past the end
+  };
+
+  float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+#pragma unroll
+  for (int c = 0; c < F_NS - 1; ++c) issue(c);
+  for (int c = 0; c < n_chunks; ++c) {
+    cp_async_wait<F_NS - 2>();  // this thread's copies of chunk c have landed
+    __syncthreads();            // everyone's; and chunk c - 1 is no longer read
+    const int st = c % F_NS;
+#pragma unroll
+    for (int i = 0; i < F_KC * S::CB / APP_THREADS; ++i) {
+      const int e = tid + i * APP_THREADS;
+      af[e] = __uint_as_float((uint32_t)ar[st][e] << 16);
+    }
+    __syncthreads();
+    issue(c + F_NS - 1);  // into the stage chunk c - 1 used
+    const int kc = min(F_KC, Dm - c * F_KC);  // a multiple of 8
+    const uint4* xrow = reinterpret_cast<const uint4*>(&xr[st][tl * F_XP]);
+    const float4* acol = reinterpret_cast<const float4*>(af) + cg;
+    for (int k8 = 0; k8 < kc / 8; ++k8) {
+      const uint4 xv = xrow[k8];
+      const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float xf = __uint_as_float(q & 1 ? (w[q >> 1] & 0xffff0000u) : (w[q >> 1] << 16));
+        const float4 av = acol[(k8 * 8 + q) * (S::CB / 4)];
+        acc0 = fmaf(xf, av.x, acc0);
+        acc1 = fmaf(xf, av.y, acc1);
+        acc2 = fmaf(xf, av.z, acc2);
+        acc3 = fmaf(xf, av.w, acc3);
+      }
+    }
+  }
+  cp_async_wait<0>();
+  const int t = t0 + tl;
+  if (t < T) {
+    __nv_bfloat16* dst =
+        u + (size_t)session * u_ss + (size_t)agent * u_sa + (size_t)(start_row + t) * u_st + c0 + cg * 4;
+    dst[0] = __float2bfloat16_rn(acc0);
+    dst[1] = __float2bfloat16_rn(acc1);
+    dst[2] = __float2bfloat16_rn(acc2);
+    dst[3] = __float2bfloat16_rn(acc3);
+  }
+}
+
+template <int R>
+void launch_r(const void* x, const void* a, int n_a, int T, int Dm, void* u, long long u_ss, long long u_sa,
+              long long u_st, int session, int start_row, cudaStream_t stream) {
+  const bool fast = Dm % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 && (reinterpret_cast<uintptr_t>(a) & 15) == 0;
+  if (!fast) {
+    launch_generic<R>(x, a, n_a, T, Dm, u, u_ss, u_sa, u_st, session, start_row, stream);
+    return;
+  }
+  using S = FastShape<R>;
+  dim3 grid((T + S::TB - 1) / S::TB, n_a, S::NCB);
+  append_kernel_fast<R><<<grid, APP_THREADS, 0, stream>>>(static_cast<const uint16_t*>(x),
+                                                          static_cast<const uint16_t*>(a), T, Dm,
+                                                          static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st,
+                                                          session, start_row);
 }
 
 }  // namespace

@@ -487,46 +487,41 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
   const int D = p->head_dim, RK = p->rank;
   if (lrkv::prefill_smem_bytes(D, RK) > dev.smem_optin) return fail(LRKV_ERR_UNSUPPORTED, "prefill tiles do not fit in shared memory");
 
-  alignas(64) CUtensorMap maps[5];
+  alignas(64) CUtensorMap maps[4];
   // V and U blocks sit side by side in shared memory as one [keys, d + r]
   // operand of RK-element swizzle atoms, so that P [V | U] is one MMA per k-step
   const CUtensorMapSwizzle vu_swizzle = RK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   const int TM = 128 / G;
-  {  // Q [N, T, Hq, d]: box = 64 dims x G heads x TM tokens of one agent
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p->num_q_heads, (uint64_t)T, (uint64_t)p->num_agents};
-    const int64_t str[3] = {D, (int64_t)p->num_q_heads * D, (int64_t)T * p->num_q_heads * D};
-    const uint32_t box[4] = {64, (uint32_t)G, (uint32_t)TM, 1};
-    if ((s = make_map4(&maps[0], q, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "Q")) != LRKV_OK) return s;
-  }
   if (kv->page_table) {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)kv->page_size, (uint64_t)p->num_kv_heads, (uint64_t)kv->num_pages};
     const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_page};
     const uint32_t box[4] = {64, 64, 1, 1};
     const uint32_t vbox[4] = {(uint32_t)RK, 64, 1, 1};  // V in the same RK-wide swizzle atoms as U
-    if ((s = make_map4(&maps[1], kv->k, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "K pages")) != LRKV_OK) return s;
-    if ((s = make_map4(&maps[2], kv->v, dims, str, vbox, vu_swizzle, "V pages")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[0], kv->k, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "K pages")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[1], kv->v, dims, str, vbox, vu_swizzle, "V pages")) != LRKV_OK) return s;
   } else {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Ltot, (uint64_t)p->num_kv_heads, (uint64_t)p->num_sessions};
     const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_session};
     const uint32_t box[4] = {64, 128, 1, 1};
     const uint32_t vbox[4] = {(uint32_t)RK, 128, 1, 1};
-    if ((s = make_map4(&maps[1], kv->k, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "K")) != LRKV_OK) return s;
-    if ((s = make_map4(&maps[2], kv->v, dims, str, vbox, vu_swizzle, "V")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[0], kv->k, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "K")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[1], kv->v, dims, str, vbox, vu_swizzle, "V")) != LRKV_OK) return s;
   }
   {
     const int slots = p->mode == LRKV_BASE_SHARED ? p->num_agents : 1;
     const uint64_t dims[4] = {(uint64_t)RK, (uint64_t)Ltot, (uint64_t)slots, (uint64_t)p->num_sessions};
     const int64_t str[3] = {u->stride_token, u->stride_agent, u->stride_session};
     const uint32_t box[4] = {(uint32_t)RK, 128, 1, 1};
-    if ((s = make_map4(&maps[3], u->u, dims, str, box, vu_swizzle, "U")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[2], u->u, dims, str, box, vu_swizzle, "U")) != LRKV_OK) return s;
   }
   {  // B [N, r, Hkv*d]: box = d dims of one KV head x r ranks of one agent
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p->num_kv_heads, (uint64_t)RK, (uint64_t)p->num_agents};
     const int64_t str[3] = {D, (int64_t)p->num_kv_heads * D, (int64_t)RK * p->num_kv_heads * D};
     const uint32_t box[4] = {(uint32_t)D, 1, (uint32_t)RK, 1};
-    if ((s = make_map4(&maps[4], b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE, "B")) != LRKV_OK) return s;
+    if ((s = make_map4(&maps[3], b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE, "B")) != LRKV_OK) return s;
   }
   lrkv::PrefillParams pp = {};
+  pp.q = q;
   pp.offsets = alora_offsets;
   pp.page_table = kv->page_table;
   pp.pt_stride = kv->page_table_stride;

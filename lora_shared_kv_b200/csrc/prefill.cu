@@ -15,7 +15,8 @@
 // loaded serves all of them.  Roles:
 //   warp 0        TMA producer: Q tile and B_i,g once, then 128-key blocks of
 //                 K into a 3-stage ring (a stage frees as soon as its S is
-//                 computed) and of V and U into a 2-stage ring.
+//                 computed).
+//   warp 2        TMA producer of the V and U blocks (2-stage ring).
 //   warp 1        TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into a
 //                 double-buffered S in TMEM; then [O | Z] += P_j [V_j | U_j]
 //                 with P_j read from TMEM (it overwrites S_j): V_j and U_j lie
@@ -43,19 +44,17 @@ constexpr int BM = 128;   // rows per tile (TMEM lanes)
 constexpr int BN = 128;   // keys per block
 constexpr int KST = 3;    // K ring: a stage is free once S = Q K^T has been computed
 constexpr int VST = 2;    // V/U ring: a stage is free once O += P V and Z += P U are done
-constexpr int THREADS = 384;  // producer, MMA, 2 idle, 2 softmax warpgroups
+constexpr int THREADS = 384;  // K producer, MMA, V/U producer, idle, 2 softmax warpgroups
 constexpr int SMX_THREADS = 256;  // the two softmax warpgroups (named barrier 1)
 constexpr uint32_t TMEM_COLS = 512;
 
 template <int D, int RK>
 struct PrefillLayout {
-  static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int B_BYTES = RK * D * 2;
   static constexpr int K_BYTES = BN * D * 2;
   static constexpr int U_BYTES = BN * RK * 2;
   static constexpr int V_STAGE = K_BYTES + U_BYTES;   // V block then U block
-  static constexpr int Q_OFF = 0;
-  static constexpr int B_OFF = Q_OFF + Q_BYTES;
+  static constexpr int B_OFF = 0;
   static constexpr int K_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int V_OFF = K_OFF + KST * K_BYTES;
   static constexpr int BAR_OFF = V_OFF + VST * V_STAGE;
@@ -63,12 +62,14 @@ struct PrefillLayout {
   static constexpr int TOTAL = XCH_OFF + 6 * BM * 4;
   // TMEM columns
   static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_Z = 2 * BN + D;
-  static_assert(2 * BN + D + RK <= (int)TMEM_COLS, "TMEM budget");
+  static constexpr uint32_t COL_Q = 448;  // the Q tile, bf16 pairs: the A operand of S = Q K^T
+  static_assert(2 * BN + D + RK <= (int)COL_Q && COL_Q + D / 2 <= TMEM_COLS, "TMEM budget");
   static_assert(K_BYTES % 1024 == 0 && V_STAGE % 1024 == 0, "stage alignment");
 };
 
 struct Bars {
-  uint64_t q_full;
+  uint64_t q_full;  // the Q tile is in TMEM (one arrival per softmax warp)
+  uint64_t b_full;  // B_i,g has landed in shared memory
   uint64_t k_full[KST];
   uint64_t k_empty[KST];
   uint64_t v_full[VST];
@@ -93,7 +94,7 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 
 template <int D, int RK>
 __global__ void __launch_bounds__(THREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    prefill_kernel(const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmU,
                    const __grid_constant__ CUtensorMap tmB, const PrefillParams p) {
   using Lay = PrefillLayout<D, RK>;
@@ -116,7 +117,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nb = (key_end + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_full, 8);
+    mbar_init(&bars->b_full, 1);
     for (int s = 0; s < KST; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
@@ -139,7 +141,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmU);
@@ -162,26 +163,26 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   const int u_slot = p.mode == LRKV_BASE_SHARED ? agent : 0;
 
-  if (warp == 0) {
-    // ======================= producer =======================
+  if (warp == 0 || warp == 2) {
+    // ======================= producers: K (warp 0), V and U (warp 2) =======================
+    // Separate issuers, so that K blocks run ahead by their own ring depth and
+    // never wait behind a V stage that the PV of two blocks back still holds.
     if (lane == 0) {
+      const bool k_role = warp == 0;
       const uint64_t pol_kv = policy_evict_last();  // K/V blocks are reused by the other tiles of the KV head
-      const uint64_t pol_q = policy_evict_first();
-      mbar_arrive_expect_tx(&bars->q_full, Lay::Q_BYTES + Lay::B_BYTES);
-#pragma unroll
-      for (int hh = 0; hh < D / 64; ++hh)
-        tma_load_4d(smem + Lay::Q_OFF + hh * (BM * 128), &tmQ, &bars->q_full, hh * 64, g * p.G, j0, agent, pol_q);
-      tma_load_4d(smem + Lay::B_OFF, &tmB, &bars->q_full, 0, g, 0, agent, pol_q);
-      int n_pages = 0;
-      if (p.page_table) n_pages = (p.L0 + p.T + 63) / 64;
-      int k_issued = 0, v_issued = 0;
+      if (k_role) {
+        mbar_arrive_expect_tx(&bars->b_full, Lay::B_BYTES);
+        tma_load_4d(smem + Lay::B_OFF, &tmB, &bars->b_full, 0, g, 0, agent, policy_evict_first());
+      }
+      const int n_pages = p.page_table ? (p.L0 + p.T + 63) / 64 : 0;
+      const int NS = k_role ? KST : VST;
+      uint64_t* full = k_role ? bars->k_full : bars->v_full;
+      uint64_t* empty = k_role ? bars->k_empty : bars->v_empty;
+      int issued = 0;
       for (int jb = 0; jb < nb; ++jb) {
-        // ---- K block jb
-        const int ks_ = jb % KST;
-        if (!mbar_wait_bounded(&bars->k_empty[ks_], ((jb / KST) & 1) ^ 1, abort_flag, p.flags)) break;
-        k_issued = jb + 1;
-        uint8_t* Ks = smem + Lay::K_OFF + ks_ * Lay::K_BYTES;
-        mbar_arrive_expect_tx(&bars->k_full[ks_], Lay::K_BYTES);
+        const int st = jb % NS;
+        if (!mbar_wait_bounded(&empty[st], ((jb / NS) & 1) ^ 1, abort_flag, p.flags)) break;
+        issued = jb + 1;
         int phys[BN / 64];
         if (p.page_table) {
 #pragma unroll
@@ -196,51 +197,47 @@ __global__ void __launch_bounds__(THREADS, 1)
             phys[pg] = ph_;
           }
         }
+        if (k_role) {
+          uint8_t* Ks = smem + Lay::K_OFF + st * Lay::K_BYTES;
+          mbar_arrive_expect_tx(&full[st], Lay::K_BYTES);
 #pragma unroll
-        for (int hh = 0; hh < D / 64; ++hh) {
-          if (!p.page_table) {
-            tma_load_4d(Ks + hh * (BN * 128), &tmK, &bars->k_full[ks_], hh * 64, jb * BN, g, p.session, pol_kv);
-          } else {
+          for (int hh = 0; hh < D / 64; ++hh) {
+            if (!p.page_table) {
+              tma_load_4d(Ks + hh * (BN * 128), &tmK, &full[st], hh * 64, jb * BN, g, p.session, pol_kv);
+            } else {
 #pragma unroll
-            for (int pg = 0; pg < BN / 64; ++pg)
-              tma_load_4d(Ks + hh * (BN * 128) + pg * (64 * 128), &tmK, &bars->k_full[ks_], hh * 64, 0, g, phys[pg],
-                          pol_kv);
+              for (int pg = 0; pg < BN / 64; ++pg)
+                tma_load_4d(Ks + hh * (BN * 128) + pg * (64 * 128), &tmK, &full[st], hh * 64, 0, g, phys[pg], pol_kv);
+            }
           }
-        }
-        // ---- V (and U) block jb
-        const int vs_ = jb % VST;
-        if (!mbar_wait_bounded(&bars->v_empty[vs_], ((jb / VST) & 1) ^ 1, abort_flag, p.flags)) break;
-        v_issued = jb + 1;
-        const bool need_u = jb * BN + BN > a_i;
-        uint8_t* Vs = smem + Lay::V_OFF + vs_ * Lay::V_STAGE;
-        uint8_t* Us = Vs + Lay::K_BYTES;
-        mbar_arrive_expect_tx(&bars->v_full[vs_], Lay::K_BYTES + (need_u ? Lay::U_BYTES : 0));
+        } else {
+          const bool need_u = jb * BN + BN > a_i;
+          uint8_t* Vs = smem + Lay::V_OFF + st * Lay::V_STAGE;
+          uint8_t* Us = Vs + Lay::K_BYTES;
+          mbar_arrive_expect_tx(&full[st], Lay::K_BYTES + (need_u ? Lay::U_BYTES : 0));
 #pragma unroll
-        for (int at = 0; at < D / RK; ++at) {  // RK-wide atoms of V, each [BN keys][RK dims]
-          if (!p.page_table) {
-            tma_load_4d(Vs + at * Lay::U_BYTES, &tmV, &bars->v_full[vs_], at * RK, jb * BN, g, p.session, pol_kv);
-          } else {
+          for (int at = 0; at < D / RK; ++at) {  // RK-wide atoms of V, each [BN keys][RK dims]
+            if (!p.page_table) {
+              tma_load_4d(Vs + at * Lay::U_BYTES, &tmV, &full[st], at * RK, jb * BN, g, p.session, pol_kv);
+            } else {
 #pragma unroll
-            for (int pg = 0; pg < BN / 64; ++pg)
-              tma_load_4d(Vs + at * Lay::U_BYTES + pg * (64 * RK * 2), &tmV, &bars->v_full[vs_], at * RK, 0, g,
-                          phys[pg], pol_kv);
+              for (int pg = 0; pg < BN / 64; ++pg)
+                tma_load_4d(Vs + at * Lay::U_BYTES + pg * (64 * RK * 2), &tmV, &full[st], at * RK, 0, g, phys[pg],
+                            pol_kv);
+            }
           }
+          if (need_u) tma_load_4d(Us, &tmU, &full[st], 0, jb * BN, u_slot, p.session, pol_kv);
         }
-        if (need_u) tma_load_4d(Us, &tmU, &bars->v_full[vs_], 0, jb * BN, u_slot, p.session, pol_kv);
       }
       if (*abort_flag) {
-        // let every copy this CTA issued land before the CTA can exit
+        // let every copy this issuer started land before the CTA can exit
         uint32_t spins = 0;
-        while (!mbar_try_wait(&bars->q_full, 0) && ++spins < kSpinCap) {
-        }
-        for (int blk = k_issued > KST ? k_issued - KST : 0; blk < k_issued; ++blk) {
-          spins = 0;
-          while (!mbar_try_wait(&bars->k_full[blk % KST], (blk / KST) & 1) && ++spins < kSpinCap) {
+        if (k_role)
+          while (!mbar_try_wait(&bars->b_full, 0) && ++spins < kSpinCap) {
           }
-        }
-        for (int blk = v_issued > VST ? v_issued - VST : 0; blk < v_issued; ++blk) {
+        for (int blk = issued > NS ? issued - NS : 0; blk < issued; ++blk) {
           spins = 0;
-          while (!mbar_try_wait(&bars->v_full[blk % VST], (blk / VST) & 1) && ++spins < kSpinCap) {
+          while (!mbar_try_wait(&full[blk % NS], (blk / NS) & 1) && ++spins < kSpinCap) {
           }
         }
       }
@@ -253,7 +250,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr uint32_t VU_LAYOUT = RK == 32 ? 4u : 6u;  // 64B / 32B swizzle: atoms of RK bf16 per key row
     constexpr uint32_t VU_LBO = Lay::U_BYTES;           // next atom along d + r
     constexpr uint32_t VU_SBO = 8 * RK * 2;             // next eight key rows
-    const uint32_t q_base = smem_u32(smem + Lay::Q_OFF);
     bool ok = mbar_wait_bounded(&bars->q_full, 0, abort_flag, p.flags);
     for (int jb = 0; jb <= nb && ok; ++jb) {
       if (jb < nb) {
@@ -266,10 +262,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t d_s = tmem + (jb & 1 ? Lay::COL_S1 : Lay::COL_S0);
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
-            const uint64_t a = umma_desc(q_base + off, 16, 1024, 2);
             const uint64_t b = umma_desc(k_base + (ks >> 2) * (BN * 128) + (ks & 3) * 32, 16, 1024, 2);
-            umma_ss(d_s, a, b, ID_QK, ks > 0);
+            umma_ts(d_s, tmem + Lay::COL_Q + ks * 8, b, ID_QK, ks > 0);
           }
           umma_commit(&bars->s_full[jb & 1]);
           umma_commit(&bars->k_empty[st]);
@@ -324,6 +318,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float NEG_INF = -INFINITY;
     float m_ref = NEG_INF, l = 0.f;
     bool ok = true;
+    {
+      // this row's Q into TMEM: half wg of its d dims as bf16 pairs (zeros past the chunk)
+      constexpr int QH = D / 2;  // dims per half
+      uint32_t qw[QH / 2];
+      const uint4* qsrc = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                                         (((size_t)agent * p.T + token) * p.Hq + g * p.G + hh) * D +
+                                                         wg * QH);
+#pragma unroll
+      for (int v = 0; v < QH / 8; ++v) {
+        const uint4 w = token < p.T ? __ldg(qsrc + v) : make_uint4(0, 0, 0, 0);
+        qw[4 * v] = w.x;
+        qw[4 * v + 1] = w.y;
+        qw[4 * v + 2] = w.z;
+        qw[4 * v + 3] = w.w;
+      }
+      if constexpr (QH / 2 == 32) tmem_st32(tmem + lane_addr + Lay::COL_Q + wg * (QH / 2), qw);
+      else tmem_st16(tmem + lane_addr + Lay::COL_Q + wg * (QH / 2), qw);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_full);
+    }
     if (wg == 1) {
       // Z starts at zero: the MMA of the first block that reads U accumulates into it
       // (a P [V | U] MMA has one accumulate flag for O and Z)
@@ -419,6 +435,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok) ok = mbar_wait_bounded(&bars->o_ready[(nb - 1) & 1], ((nb - 1) >> 1) & 1, abort_flag, p.flags);
     named_bar_sync(1, SMX_THREADS);
     l = xsum[row] + xsum[BM + row];
+    if (ok) ok = mbar_wait_bounded(&bars->b_full, 0, abort_flag, p.flags);
     tc_fence_after();
     float z[RK];
     {
@@ -506,7 +523,7 @@ lrkv_status launch_t(const PrefillParams& p, const PrefillMaps& m, int grid, cud
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const CUtensorMap* t = static_cast<const CUtensorMap*>(m.maps);
-  if (cudaLaunchKernelEx(&cfg, kern, t[0], t[1], t[2], t[3], t[4], p) != cudaSuccess) return LRKV_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, t[0], t[1], t[2], t[3], p) != cudaSuccess) return LRKV_ERR_CUDA;
   return LRKV_OK;
 }
 

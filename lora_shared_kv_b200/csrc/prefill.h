@@ -6,6 +6,7 @@
 namespace lrkv {
 
 struct PrefillParams {
+  const void* q;             // [N, T, Hq, d] bf16, contiguous
   const int32_t* offsets;    // [N] or null
   const int32_t* page_table; // null => dense
   long long pt_stride;
@@ -20,7 +21,7 @@ struct PrefillParams {
   unsigned* flags;
 };
 
-// Five CUtensorMap objects, in order: Q, K, V, U, B.
+// Four CUtensorMap objects, in order: K, V, U, B.
 struct PrefillMaps {
   const void* maps;
 };
