@@ -53,17 +53,23 @@ struct PrefillLayout {
   static constexpr int B_BYTES = RK * D * 2;
   static constexpr int K_BYTES = BN * D * 2;
   static constexpr int U_BYTES = BN * RK * 2;
-  static constexpr int V_STAGE = K_BYTES + U_BYTES;   // V block then U block
+  // V block (D / RK atoms), a constant atom whose column 0 is 1 (the row
+  // sums of P come out of the same MMA as O), then the U block
+  static constexpr int V_STAGE = K_BYTES + 2 * U_BYTES;
+  static constexpr int ONES_OFF = K_BYTES;
+  static constexpr int U_OFF = K_BYTES + U_BYTES;
   static constexpr int B_OFF = 0;
   static constexpr int K_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int V_OFF = K_OFF + KST * K_BYTES;
   static constexpr int BAR_OFF = V_OFF + VST * V_STAGE;
-  static constexpr int XCH_OFF = BAR_OFF + 256;  // row max [2 blocks][2 halves][BM], row sum [2 halves][BM]
-  static constexpr int TOTAL = XCH_OFF + 6 * BM * 4;
+  static constexpr int XCH_OFF = BAR_OFF + 256;  // row max [2 blocks][2 halves][BM]
+  static constexpr int TOTAL = XCH_OFF + 4 * BM * 4;
   // TMEM columns
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_Z = 2 * BN + D;
+  // TMEM columns: S double buffer; then [O | L | Z], the accumulator of
+  // P [V | ones | U] (L: column 0 of an RK-wide block is the row sum l)
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_L = 2 * BN + D, COL_Z = 2 * BN + D + RK;
   static constexpr uint32_t COL_Q = 448;  // the Q tile, bf16 pairs: the A operand of S = Q K^T
-  static_assert(2 * BN + D + RK <= (int)COL_Q && COL_Q + D / 2 <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * BN + D + 2 * RK <= (int)COL_Q && COL_Q + D / 2 <= TMEM_COLS, "TMEM budget");
   static_assert(K_BYTES % 1024 == 0 && V_STAGE % 1024 == 0, "stage alignment");
 };
 
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else {
           const bool need_u = jb * BN + BN > a_i;
           uint8_t* Vs = smem + Lay::V_OFF + st * Lay::V_STAGE;
-          uint8_t* Us = Vs + Lay::K_BYTES;
+          uint8_t* Us = Vs + Lay::U_OFF;
           mbar_arrive_expect_tx(&full[st], Lay::K_BYTES + (need_u ? Lay::U_BYTES : 0));
 #pragma unroll
           for (int at = 0; at < D / RK; ++at) {  // RK-wide atoms of V, each [BN keys][RK dims]
@@ -245,8 +251,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     constexpr uint32_t ID_QK = umma_idesc_bf16(BM, BN, 0, 0);
-    constexpr uint32_t ID_PV = umma_idesc_bf16(BM, D, 0, 1);        // [O] += P V
-    constexpr uint32_t ID_PVU = umma_idesc_bf16(BM, D + RK, 0, 1);  // [O | Z] += P [V | U]
+    constexpr uint32_t ID_PV = umma_idesc_bf16(BM, D + 16, 0, 1);       // [O | l] += P [V | 1]
+    constexpr uint32_t ID_PVU = umma_idesc_bf16(BM, D + 2 * RK, 0, 1);  // [O | l | Z] += P [V | 1 | U]
     constexpr uint32_t VU_LAYOUT = RK == 32 ? 4u : 6u;  // 64B / 32B swizzle: atoms of RK bf16 per key row
     constexpr uint32_t VU_LBO = Lay::U_BYTES;           // next atom along d + r
     constexpr uint32_t VU_SBO = 8 * RK * 2;             // next eight key rows
@@ -277,7 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ok) ok = mbar_wait_bounded(&bars->v_full[st], (j / VST) & 1, abort_flag, p.flags);
         if (!ok) break;
         const bool u_used = j * BN + BN > a_i;
-        uint8_t* Us = smem + Lay::V_OFF + st * Lay::V_STAGE + Lay::K_BYTES;
+        uint8_t* Us = smem + Lay::V_OFF + st * Lay::V_STAGE + Lay::U_OFF;
         if (u_used && j * BN < a_i) {
           // the block holding a_i: rows before the offset are removed (zero-filled) before the MMA reads them
           const int nz = a_i - j * BN;  // rows [0, nz)
@@ -292,6 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t v_base = smem_u32(smem + Lay::V_OFF + st * Lay::V_STAGE);
           const uint32_t a_p = tmem + (j & 1 ? Lay::COL_S1 : Lay::COL_S0);
           const uint32_t id = u_used ? ID_PVU : ID_PV;  // Z (zeroed at the start) accumulates from its first block on
+          // (the first MMA overwrites O and l)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint64_t b = umma_desc(v_base + kk * (16 * RK * 2), VU_LBO, VU_SBO, VU_LAYOUT);
@@ -311,12 +318,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int HB = BN / 2;                // keys per half
     const int c0 = wg * HB;
     float* xmax = reinterpret_cast<float*>(smem + Lay::XCH_OFF);  // [blk & 1][half][row]
-    float* xsum = xmax + 4 * BM;                                  // [half][row]
     const int jj = row / p.G, hh = row % p.G;
     const int token = j0 + jj;
     const int limit = p.L0 + token;            // last visible key of this row
     const float NEG_INF = -INFINITY;
-    float m_ref = NEG_INF, l = 0.f;
+    float m_ref = NEG_INF;
     bool ok = true;
     {
       // this row's Q into TMEM: half wg of its d dims as bf16 pairs (zeros past the chunk)
@@ -342,13 +348,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (wg == 1) {
       // Z starts at zero: the MMA of the first block that reads U accumulates into it
-      // (a P [V | U] MMA has one accumulate flag for O and Z)
+      // (a P [V | 1 | U] MMA has one accumulate flag for O, l and Z)
       uint32_t zero[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) zero[e] = 0u;
       if constexpr (RK == 32) tmem_st32(tmem + lane_addr + Lay::COL_Z, zero);
       else tmem_st16(tmem + lane_addr + Lay::COL_Z, zero);
       tmem_wait_st();
+      // the constant atom of every V stage: logical column 0 of each key row is
+      // bf16 1.0.  Its rows use the RK-wide swizzle of V and U: 16-byte chunk c
+      // of row r sits at chunk c ^ (r >> 1) & 3 (64-byte rows) or c ^ (r >> 2) & 1
+      // (32-byte rows).
+      constexpr int CPR = RK / 8;  // 16-byte chunks per row
+      for (int q = row; q < VST * BN * CPR; q += BM) {
+        const int stg = q / (BN * CPR), r = (q / CPR) % BN, pc = q % CPR;
+        const int swz = RK == 32 ? (r >> 1) & 3 : (r >> 2) & 1;
+        uint4* dst = reinterpret_cast<uint4*>(smem + Lay::V_OFF + stg * Lay::V_STAGE + Lay::ONES_OFF) + r * CPR + pc;
+        *dst = make_uint4((pc ^ swz) == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();  // the tensor core reads it through the async proxy
     }
     // Both warpgroups pass the same named barriers whatever happens: after a
     // failed wait they skip the waits, not the barriers.
@@ -396,33 +414,30 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
             tmem_st32(tmem + lane_addr + Lay::COL_O + c * 32, r);
           }
-          if (wg == 1) {  // Z
-            uint32_t r[RK];
-            if constexpr (RK == 32) tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);
-            else tmem_ld16(tmem + lane_addr + Lay::COL_Z, r);
-            tmem_wait_ld();
+          if (wg == 1) {  // l and Z
 #pragma unroll
-            for (int e = 0; e < RK; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            if constexpr (RK == 32) tmem_st32(tmem + lane_addr + Lay::COL_Z, r);
-            else tmem_st16(tmem + lane_addr + Lay::COL_Z, r);
+            for (int c = 0; c < 2 * RK / 32; ++c) {
+              uint32_t r[32];
+              tmem_ld32(tmem + lane_addr + Lay::COL_L + c * 32, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st32(tmem + lane_addr + Lay::COL_L + c * 32, r);
+            }
           }
           tmem_wait_st();
         }
-        l *= alpha;
         m_ref = m_new;
       }
       const float mu = m_ref == NEG_INF ? 0.f : m_ref;
+      // (the row sum l of exactly these bf16 weights is accumulated by the MMA)
       uint32_t pk[HB / 2];
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int cc = 0; cc < HB / 2; ++cc) {
         const float p0 = fast_exp2(fmaf(x[2 * cc], p.scale_log2, -mu));
         const float p1 = fast_exp2(fmaf(x[2 * cc + 1], p.scale_log2, -mu));
         pk[cc] = pack_bf16x2(p0, p1);
-        // the row sum of exactly the bf16 weights the MMA uses, in eight chains
-        ls[cc & 7] += bf16_lo(pk[cc]) + bf16_hi(pk[cc]);
       }
-      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       // P of keys [c0, c0 + 64) as bf16 pairs: TMEM columns s_col + c0 / 2 + [0, 32)
       tmem_st32(tmem + lane_addr + s_col + c0 / 2, pk);
       tmem_wait_st();
@@ -431,20 +446,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(&bars->p_full[jb & 1]);
     }
     // ---- epilogue: out = (O + Z B_i,g) / l, each half writes half of the columns
-    xsum[wg * BM + row] = l;
     if (ok) ok = mbar_wait_bounded(&bars->o_ready[(nb - 1) & 1], ((nb - 1) >> 1) & 1, abort_flag, p.flags);
-    named_bar_sync(1, SMX_THREADS);
-    l = xsum[row] + xsum[BM + row];
     if (ok) ok = mbar_wait_bounded(&bars->b_full, 0, abort_flag, p.flags);
     tc_fence_after();
-    float z[RK];
+    float z[RK], l;
     {
-      uint32_t r[RK];
-      if constexpr (RK == 32) tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);
-      else tmem_ld16(tmem + lane_addr + Lay::COL_Z, r);
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_addr + Lay::COL_L, r);  // l, then Z when RK = 16
       tmem_wait_ld();
+      l = __uint_as_float(r[0]);
+      if constexpr (RK == 16) {
 #pragma unroll
-      for (int k = 0; k < RK; ++k) z[k] = __uint_as_float(r[k]);
+        for (int k = 0; k < RK; ++k) z[k] = __uint_as_float(r[16 + k]);
+      } else {
+        tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < RK; ++k) z[k] = __uint_as_float(r[k]);
+      }
     }
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const bool write = token < p.T && ok;
