@@ -13,23 +13,25 @@
 // One CTA computes one 128-row tile: one agent, one KV head, 128/G chunk
 // tokens x the G query heads that share the KV head, so every K/V block
 // loaded serves all of them.  Roles:
-//   warp 0        TMA producer: Q tile and B_i,g once, then 128-key blocks of
-//                 K into a 3-stage ring (a stage frees as soon as its S is
-//                 computed).
+//   warp 0        TMA producer: B_i,g once, then 128-key blocks of K into a
+//                 3-stage ring (a stage frees as soon as its S is computed).
 //   warp 2        TMA producer of the V and U blocks (2-stage ring).
-//   warp 1        TMEM owner and MMA issuer (one thread): S_j = Q K_j^T into a
-//                 double-buffered S in TMEM; then [O | Z] += P_j [V_j | U_j]
-//                 with P_j read from TMEM (it overwrites S_j): V_j and U_j lie
-//                 side by side in shared memory as one operand of d + r
-//                 columns, so a k-step is one MMA of N = d + r (N = d for the
-//                 blocks wholly before the aLoRA offset, whose U is not read).
-//   warps 4..11   softmax and epilogue in two warpgroups, one per half of the
-//                 block's 128 keys; a thread owns one row (TMEM lane) of its
-//                 half.  The halves agree on each row's reference max through
-//                 shared memory and keep separate partial sums.  The reference
-//                 max moves only when a block exceeds it by 2^8, and only then
-//                 are O and Z rescaled in TMEM (each half rescales its share of
-//                 the columns).  The epilogue splits the output columns.
+//   warp 1        TMEM owner and MMA issuer (one thread): S_j = Q K_j^T with
+//                 the Q tile read from TMEM, into a double-buffered S; then
+//                 [O | Z | l] += P_j [V_j | U_j | 1] with P_j read from TMEM
+//                 (it overwrites S_j).  V_j, U_j and a constant block whose
+//                 column 0 is one lie side by side in shared memory as one
+//                 operand, so a k-step is one MMA of N = d + r + 16 and the row
+//                 sums l of exactly the bf16 weights come out with O.  U rows
+//                 before the aLoRA offset are zero-filled (the U of blocks
+//                 wholly before it is not loaded).
+//   warps 4..11   Q into TMEM, softmax and epilogue, in two warpgroups, one
+//                 per half of the block's 128 keys; a thread owns one row (TMEM
+//                 lane) of its half.  The halves agree on each row's reference
+//                 max through shared memory.  The reference max moves only when
+//                 a block exceeds it by 2^8, and only then are O, Z and l
+//                 rescaled in TMEM (each half rescales its share of the
+//                 columns).  The epilogue splits the output columns.
 #include <float.h>
 #include <math.h>
 
@@ -53,11 +55,11 @@ struct PrefillLayout {
   static constexpr int B_BYTES = RK * D * 2;
   static constexpr int K_BYTES = BN * D * 2;
   static constexpr int U_BYTES = BN * RK * 2;
-  // V block (D / RK atoms), a constant atom whose column 0 is 1 (the row
-  // sums of P come out of the same MMA as O), then the U block
+  // V block (D / RK atoms), the U block, then a constant atom whose column 0
+  // is 1, so that the row sums of P come out of the same MMA as O and Z
   static constexpr int V_STAGE = K_BYTES + 2 * U_BYTES;
-  static constexpr int ONES_OFF = K_BYTES;
-  static constexpr int U_OFF = K_BYTES + U_BYTES;
+  static constexpr int U_OFF = K_BYTES;
+  static constexpr int ONES_OFF = K_BYTES + U_BYTES;
   static constexpr int B_OFF = 0;
   static constexpr int K_OFF = (B_OFF + B_BYTES + 1023) / 1024 * 1024;
   static constexpr int V_OFF = K_OFF + KST * K_BYTES;
@@ -65,11 +67,11 @@ struct PrefillLayout {
   static constexpr int XCH_OFF = BAR_OFF + 256;  // row max [2 blocks][2 halves][BM]
   static constexpr int TOTAL = XCH_OFF + 4 * BM * 4;
   // TMEM columns
-  // TMEM columns: S double buffer; then [O | L | Z], the accumulator of
-  // P [V | ones | U] (L: column 0 of an RK-wide block is the row sum l)
-  static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_L = 2 * BN + D, COL_Z = 2 * BN + D + RK;
+  // TMEM columns: S double buffer; then [O | Z | L], the accumulator of
+  // P [V | U | ones] (column 0 of the 16 L columns is the row sum l)
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_Z = 2 * BN + D, COL_L = 2 * BN + D + RK;
   static constexpr uint32_t COL_Q = 448;  // the Q tile, bf16 pairs: the A operand of S = Q K^T
-  static_assert(2 * BN + D + 2 * RK <= (int)COL_Q && COL_Q + D / 2 <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * BN + D + RK + 16 <= (int)COL_Q && COL_Q + D / 2 <= TMEM_COLS, "TMEM budget");
   static_assert(K_BYTES % 1024 == 0 && V_STAGE % 1024 == 0, "stage alignment");
 };
 
@@ -251,8 +253,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     constexpr uint32_t ID_QK = umma_idesc_bf16(BM, BN, 0, 0);
-    constexpr uint32_t ID_PV = umma_idesc_bf16(BM, D + 16, 0, 1);       // [O | l] += P [V | 1]
-    constexpr uint32_t ID_PVU = umma_idesc_bf16(BM, D + 2 * RK, 0, 1);  // [O | l | Z] += P [V | 1 | U]
+    constexpr uint32_t ID_PVU = umma_idesc_bf16(BM, D + RK + 16, 0, 1);  // [O | Z | l] += P [V | U | 1]
     constexpr uint32_t VU_LAYOUT = RK == 32 ? 4u : 6u;  // 64B / 32B swizzle: atoms of RK bf16 per key row
     constexpr uint32_t VU_LBO = Lay::U_BYTES;           // next atom along d + r
     constexpr uint32_t VU_SBO = 8 * RK * 2;             // next eight key rows
@@ -282,11 +283,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = mbar_wait_bounded(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag, p.flags);
         if (ok) ok = mbar_wait_bounded(&bars->v_full[st], (j / VST) & 1, abort_flag, p.flags);
         if (!ok) break;
-        const bool u_used = j * BN + BN > a_i;
         uint8_t* Us = smem + Lay::V_OFF + st * Lay::V_STAGE + Lay::U_OFF;
-        if (u_used && j * BN < a_i) {
-          // the block holding a_i: rows before the offset are removed (zero-filled) before the MMA reads them
-          const int nz = a_i - j * BN;  // rows [0, nz)
+        if (j * BN < a_i) {
+          // U rows before the offset are zero-filled before the MMA reads them: all
+          // of a block wholly before it (its U was not loaded), the head of the block holding it
+          const int nz = min(a_i - j * BN, BN);  // rows [0, nz)
           uint4* z4 = reinterpret_cast<uint4*>(Us);
           const int n16 = nz * RK * 2 / 16;
           for (int x = lane; x < n16; x += 32) z4[x] = make_uint4(0, 0, 0, 0);
@@ -297,12 +298,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint32_t v_base = smem_u32(smem + Lay::V_OFF + st * Lay::V_STAGE);
           const uint32_t a_p = tmem + (j & 1 ? Lay::COL_S1 : Lay::COL_S0);
-          const uint32_t id = u_used ? ID_PVU : ID_PV;  // Z (zeroed at the start) accumulates from its first block on
-          // (the first MMA overwrites O and l)
+          // (the first MMA overwrites O, Z and l)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint64_t b = umma_desc(v_base + kk * (16 * RK * 2), VU_LBO, VU_SBO, VU_LAYOUT);
-            umma_ts(tmem + Lay::COL_O, a_p + kk * 8, b, id, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tmem + Lay::COL_O, a_p + kk * 8, b, ID_PVU, (j > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&bars->v_empty[st]);
           umma_commit(&bars->o_ready[j & 1]);
@@ -347,14 +347,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(&bars->q_full);
     }
     if (wg == 1) {
-      // Z starts at zero: the MMA of the first block that reads U accumulates into it
-      // (a P [V | 1 | U] MMA has one accumulate flag for O, l and Z)
-      uint32_t zero[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) zero[e] = 0u;
-      if constexpr (RK == 32) tmem_st32(tmem + lane_addr + Lay::COL_Z, zero);
-      else tmem_st16(tmem + lane_addr + Lay::COL_Z, zero);
-      tmem_wait_st();
       // the constant atom of every V stage: logical column 0 of each key row is
       // bf16 1.0.  Its rows use the RK-wide swizzle of V and U: 16-byte chunk c
       // of row r sits at chunk c ^ (r >> 1) & 3 (64-byte rows) or c ^ (r >> 2) & 1
@@ -414,15 +406,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
             tmem_st32(tmem + lane_addr + Lay::COL_O + c * 32, r);
           }
-          if (wg == 1) {  // l and Z
+          if (wg == 1) {  // Z and l: RK + 16 columns
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);
+            tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 2 * RK / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld32(tmem + lane_addr + Lay::COL_L + c * 32, r);
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(tmem + lane_addr + Lay::COL_Z, r);
+            if constexpr (RK == 32) {
+              tmem_ld16(tmem + lane_addr + Lay::COL_L, r);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-              tmem_st32(tmem + lane_addr + Lay::COL_L + c * 32, r);
+              for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st16(tmem + lane_addr + Lay::COL_L, r);
             }
           }
           tmem_wait_st();
@@ -452,17 +448,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     float z[RK], l;
     {
       uint32_t r[32];
-      tmem_ld32(tmem + lane_addr + Lay::COL_L, r);  // l, then Z when RK = 16
+      tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);  // Z, then l when RK = 16
       tmem_wait_ld();
-      l = __uint_as_float(r[0]);
+#pragma unroll
+      for (int k = 0; k < RK; ++k) z[k] = __uint_as_float(r[k]);
       if constexpr (RK == 16) {
-#pragma unroll
-        for (int k = 0; k < RK; ++k) z[k] = __uint_as_float(r[16 + k]);
+        l = __uint_as_float(r[Lay::COL_L - Lay::COL_Z]);
       } else {
-        tmem_ld32(tmem + lane_addr + Lay::COL_Z, r);
+        tmem_ld16(tmem + lane_addr + Lay::COL_L, r);
         tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < RK; ++k) z[k] = __uint_as_float(r[k]);
+        l = __uint_as_float(r[0]);
       }
     }
     const float inv_l = l > 0.f ? 1.f / l : 0.f;

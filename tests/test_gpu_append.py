@@ -25,6 +25,11 @@ def _bits(t):
     (5, 65, 16, 1, 3, 8),
     (70, 100, 8, 2, 0, 100),
     (17, 300, 32, 1, 40, 64),
+    # Dm a multiple of 8: the pipelined path, with a partial last k-chunk and token block
+    (70, 200, 8, 2, 0, 100),
+    (33, 136, 32, 3, 5, 64),
+    (1, 8, 16, 1, 0, 4),
+    (130, 1032, 16, 2, 7, 200),
 ])
 def test_append_bit_exact(T, Dm, r, n_a, start, cap):
     g = torch.Generator(device=DEV)
