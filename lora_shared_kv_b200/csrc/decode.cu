@@ -519,7 +519,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   constexpr int KV_BYTES = KT * D * 2;
   constexpr int U_BYTES = KT * RK * 2;
   constexpr int REC = RP * (D + RK + 2);
-  constexpr int NOG = kDecodeGroups;
+  constexpr int NOG = decode_groups(NT);
   constexpr int CT = NOG * NT * 32;   // consumer threads
   const int tid = threadIdx.x;        // consumers are warps 0 .. NOG*NT-1
   const int warp = tid >> 5, lane = tid & 31;
@@ -877,11 +877,11 @@ __device__ void decode_epilogue(const DecodeParams& p, uint8_t* smem, const Deco
   }
 }
 
-// Warp roles: warps 0 .. kDecodeGroups*NT-1 consume, then one producer warp
+// Warp roles: warps 0 .. decode_groups(NT)*NT-1 consume, then one producer warp
 // and one epilogue warp.
 template <int NT>
 struct Roles {
-  static constexpr int CONSUMER_WARPS = kDecodeGroups * NT;
+  static constexpr int CONSUMER_WARPS = decode_groups(NT) * NT;
   static constexpr int THREADS = (CONSUMER_WARPS + 2) * 32;
 };
 

@@ -54,10 +54,11 @@ struct DecodeParams {
   unsigned* flags;
 };
 
-// Consumer warp groups of the decode kernel.  Tile n of a CTA goes to group
-// n % kDecodeGroups and to ring stage n % stages; the warps of a group split
-// the query rows, eight each.
-constexpr int kDecodeGroups = 2;
+// Consumer warp groups of the decode kernel (NT warps each, eight query rows
+// per warp).  Tile n of a CTA goes to group n % groups and to ring stage
+// n % stages.  More groups keep more tiles in flight per SM; three fit the
+// register file for up to 16 rows per item (NT <= 2), two for 24.
+__host__ __device__ constexpr int decode_groups(int NT) { return NT <= 2 ? 3 : 2; }
 
 // Shared-memory plan of the decode kernel (bytes from a 1024-aligned base).
 struct DecodeSmem {
