@@ -302,19 +302,41 @@ def cpu_baseline_decode(runner, max_seconds=20.0):
 
 
 def run_e2e(runner, steps, warmup, sync_all):
-    """Public API with host buffers: per step copy every layer's q from pinned host
-    memory, run the 28 decode calls, copy every layer's output back."""
+    """Public API with host buffers.  Per step every layer's q is copied from
+    pinned host memory and every layer's output back, each on its own copy
+    stream and ordered against the decode calls by events, so layer l's copies
+    overlap the neighbouring layers' attention; the step ends when the last
+    output has landed on the host."""
     c = runner.cfg
     nl = len(runner.inp.layers)
-    q_host = torch.stack([lay.q for lay in runner.inp.layers]).cpu().pin_memory()
+    lrkv = runner.lrkv
+    inp = runner.inp
+    q_host = torch.stack([lay.q for lay in inp.layers]).cpu().pin_memory()
     out_host = torch.empty((nl, c.S, c.N, c.Hq, c.d), dtype=torch.bfloat16).pin_memory()
     q_dev = torch.empty_like(q_host, device=runner.dev)
     out_dev = torch.empty_like(out_host, device=runner.dev)
+    comp = torch.cuda.current_stream(runner.dev)
+    h2d = torch.cuda.Stream(runner.dev)
+    d2h = torch.cuda.Stream(runner.dev)
+    ev_in = [torch.cuda.Event() for _ in range(nl)]
+    ev_out = [torch.cuda.Event() for _ in range(nl)]
 
     def step():
-        q_dev.copy_(q_host, non_blocking=True)
-        runner.step_eager(qs=q_dev, outs=out_dev)
-        out_host.copy_(out_dev, non_blocking=True)
+        h2d.wait_stream(comp)  # the previous step no longer reads q_dev
+        with torch.cuda.stream(h2d):
+            for li in range(nl):
+                q_dev[li].copy_(q_host[li], non_blocking=True)
+                ev_in[li].record(h2d)
+        for li, lay in enumerate(inp.layers):
+            comp.wait_event(ev_in[li])
+            lrkv.lrkv_attn_decode(runner.prob, q_dev[li], runner.kvs[li], inp.seq_lens, c.L, runner.uvs[li], lay.b,
+                                  inp.offsets, out_dev[li], runner.ws)
+            ev_out[li].record(comp)
+        with torch.cuda.stream(d2h):
+            for li in range(nl):
+                d2h.wait_event(ev_out[li])
+                out_host[li].copy_(out_dev[li], non_blocking=True)
+        comp.wait_stream(d2h)
 
     ms = _timed(step, steps, warmup, sync_all)
     return ms / steps, q_host.numel() * 2, out_host.numel() * 2
