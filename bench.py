@@ -342,6 +342,101 @@ def run_e2e(runner, steps, warmup, sync_all):
     return ms / steps, q_host.numel() * 2, out_host.numel() * 2
 
 
+def _eager_ms(fn, steps, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    e1.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3):
+    """The pages' comparison of cache sharing, on the same decode kernel.
+
+    - shared: the split value cache (base K/V once for all agents, rank-r U_i);
+    - non-shared: every agent holds its own K and its own materialised
+      V_i = V_base + Umask_i B_i (N times the K/V bytes), run as S*N single-agent
+      sessions with B = 0;
+    - full-shared: the base K/V alone, the adapter's value term dropped (no U
+      read, B = 0): the approximation the split cache avoids.
+    Times are per layer (eager launches) over the first layers whose non-shared
+    copies fit in max_bytes; the non-shared outputs are checked against the
+    shared ones (they differ only by the bf16 rounding of V_i)."""
+    lrkv, c, inp, dev = runner.lrkv, runner.cfg, runner.inp, runner.dev
+    S, N, Hq, Hkv, d, r, L = c.S, c.N, c.Hq, c.Hkv, c.d, c.r, c.L
+    per_layer_ns = 2 * S * N * Hkv * L * d * BF16
+    nl = max(1, min(len(inp.layers), int(max_bytes // per_layer_ns)))
+    keep = torch.arange(L, device=dev)[None, None, :] >= inp.offsets[:, :, None].long()  # [S, N, L]
+    prob_ns = lrkv.make_problem(S * N, 1, Hq, Hkv, d, r, lrkv.BASE_SHARED)
+    ws_ns = torch.zeros(lrkv.lrkv_decode_workspace_bytes(prob_ns, L), dtype=torch.uint8, device=dev)
+    u_none = torch.zeros((S * N, 1, L, r), dtype=torch.bfloat16, device=dev)
+    uv_none = lrkv.u_view(u_none)
+    b_zero = torch.zeros((1, r, Hkv * d), dtype=torch.bfloat16, device=dev)
+    offs_ns = torch.full((S * N, 1), L, dtype=torch.int32, device=dev)
+    offs_full = torch.full_like(inp.offsets, L)
+    b_zero_n = torch.zeros((N, r, Hkv * d), dtype=torch.bfloat16, device=dev)
+    ns = []
+    for li in range(nl):
+        lay = inp.layers[li]
+        if c.paged:
+            pt = lay.page_table.long()
+            k = lay.k[pt].permute(0, 2, 1, 3, 4).reshape(S, Hkv, L, d)
+            v = lay.v[pt].permute(0, 2, 1, 3, 4).reshape(S, Hkv, L, d)
+        else:
+            k, v = lay.k, lay.v
+        k_ns = k.repeat_interleave(N, dim=0).contiguous()
+        v_ns = torch.empty_like(k_ns)
+        for i in range(N):
+            ui = lay.u[:, i if c.mode == 0 else 0].float() * keep[:, i, :, None]          # [S, L, r]
+            vi = v.float() + torch.einsum("slr,rgd->sgld", ui, lay.b[i].float().view(r, Hkv, d))
+            v_ns[i::N] = vi.to(torch.bfloat16)
+        ns.append((k_ns, v_ns, lay.q.reshape(S * N, 1, Hq, d).contiguous(),
+                   torch.empty((S * N, 1, Hq, d), dtype=torch.bfloat16, device=dev)))
+    kv_ns = [lrkv.kv_view_dense(k_ns, v_ns) for k_ns, v_ns, _, _ in ns]
+
+    def run_shared():
+        for li in range(nl):
+            lay = inp.layers[li]
+            lrkv.lrkv_attn_decode(runner.prob, lay.q, runner.kvs[li], inp.seq_lens, L, runner.uvs[li], lay.b,
+                                  inp.offsets, runner.outs[li], runner.ws)
+
+    def run_full_shared():
+        for li in range(nl):
+            lay = inp.layers[li]
+            lrkv.lrkv_attn_decode(runner.prob, lay.q, runner.kvs[li], inp.seq_lens, L, runner.uvs[li], b_zero_n,
+                                  offs_full, runner.outs[li], runner.ws)
+
+    seq_ns = inp.seq_lens.repeat_interleave(N)
+
+    def run_non_shared():
+        for li in range(nl):
+            _, _, q_ns, o_ns = ns[li]
+            lrkv.lrkv_attn_decode(prob_ns, q_ns, kv_ns[li], seq_ns, L, uv_none, b_zero, offs_ns, o_ns, ws_ns)
+
+    t_ns = _eager_ms(run_non_shared, steps, warmup) / nl
+    t_full = _eager_ms(run_full_shared, steps, warmup) / nl
+    t_sh = _eager_ms(run_shared, steps, warmup) / nl  # leaves the shared outputs in runner.outs
+    torch.cuda.synchronize()
+    max_abs = max(float((runner.outs[li].float() - ns[li][3].view(S, N, Hq, d).float()).abs().max())
+                  for li in range(nl))
+    kv_shared = 2 * S * Hkv * L * d * BF16 + S * c.n_u * L * r * BF16
+    out = {"workload": c.name, "layers_timed": nl, "ms_per_layer_shared": t_sh,
+           "ms_per_layer_non_shared": t_ns, "ms_per_layer_full_shared": t_full,
+           "speedup_shared_vs_non_shared": t_ns / t_sh,
+           "cache_bytes_per_layer_shared": kv_shared, "cache_bytes_per_layer_non_shared": per_layer_ns,
+           "max_abs_non_shared_vs_shared": max_abs,
+           "note": "eager launches; non-shared = per-agent K and materialised V_i, B = 0; full-shared = base K/V only"}
+    del ns, kv_ns
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_prefill(device, steps=20, warmup=5):
     """Prefill chunk workload: append the chunk's U rows, then the causal chunk
     attention for 4 agents (one layer).  Returns a dict, or None if unavailable."""
@@ -398,6 +493,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-sharing", action="store_true",
+                    help="skip the shared / non-shared / full-shared cache comparison")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the layer count (small profiling cases only; not a bench line)")
     ap.add_argument("--context", type=int, default=None,
@@ -469,6 +566,10 @@ def main():
     if not args.no_prefill and rank == 0:
         prefill = bench_prefill(dev)
 
+    sharing = None
+    if not args.no_sharing and rank == 0 and world == 1:
+        sharing = sharing_comparison(runner)
+
     cpu = None
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         cpu = cpu_baseline_decode(runner)
@@ -491,6 +592,7 @@ def main():
             "clocks": ck,
             "cpu_baseline": cpu,
             "prefill": prefill,
+            "sharing": sharing,
         }
         print(json.dumps(line))
     if world > 1:
