@@ -222,7 +222,10 @@ lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q
 /* Prefill chunk: T new rows per agent, causal, over one session.          */
 /* ---------------------------------------------------------------------- */
 
-/* Bytes of workspace lrkv_attn_prefill_chunk needs; 0 if the shape is invalid. */
+/* Bytes of workspace lrkv_attn_prefill_chunk needs; 0 if the shape is invalid.
+ * It holds the status header, one ticket per 128-row tile and the partial
+ * (m, l, O, Z) rows of tiles whose key blocks are split between CTAs (the
+ * blocks of all tiles are divided evenly over one CTA per SM). */
 size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T);
 
 /*
@@ -237,6 +240,8 @@ size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int3
  *   alora_offsets  device int32 [N], or NULL for all zero
  *   out            device [N, T, Hq, d] contiguous, bf16 or fp32
  *   workspace      device, >= lrkv_prefill_workspace_bytes, zero-filled once
+ *                  (the tickets return to zero by the end of every call; calls
+ *                  sharing a workspace must be ordered on one stream)
  */
 lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv,
                                     int32_t session, int32_t ctx_len, int32_t T,

@@ -458,7 +458,12 @@ lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q
 
 size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T) {
   if (check_problem(p) != LRKV_OK || ctx_len < 0 || T < 0) return 0;
-  return lrkv::kWsHeaderBytes;  // device-side flags only
+  if (T == 0) return lrkv::kWsHeaderBytes;
+  DeviceInfo dev;
+  if (device_info(&dev) != LRKV_OK) dev.sms = 148;
+  const int G = p->num_q_heads / p->num_kv_heads;
+  if (G < 1 || 128 % G != 0) return lrkv::kWsHeaderBytes;
+  return lrkv::plan_prefill(T, ctx_len, G, p->num_kv_heads, p->num_agents, p->head_dim, p->rank, dev.sms).bytes;
 }
 
 lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv, int32_t session,
@@ -489,9 +494,8 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
 
   alignas(64) CUtensorMap maps[4];
   // V and U blocks sit side by side in shared memory as one [keys, d + r]
-  // operand of RK-element swizzle atoms, so that P [V | U] is one MMA per k-step
+  // operand of RK-element swizzle atoms, so that P [V | U | 1] is one MMA per k-step
   const CUtensorMapSwizzle vu_swizzle = RK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  const int TM = 128 / G;
   if (kv->page_table) {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)kv->page_size, (uint64_t)p->num_kv_heads, (uint64_t)kv->num_pages};
     const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_page};
@@ -514,11 +518,12 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
     const uint32_t box[4] = {(uint32_t)RK, 128, 1, 1};
     if ((s = make_map4(&maps[2], u->u, dims, str, box, vu_swizzle, "U")) != LRKV_OK) return s;
   }
-  {  // B [N, r, Hkv*d]: box = d dims of one KV head x r ranks of one agent
+  {  // B [N, r, Hkv*d]: box = 64 dims of one KV head x r ranks of one agent, 128B-swizzled
+     // (the B operand of the Z B MMA, d-major)
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p->num_kv_heads, (uint64_t)RK, (uint64_t)p->num_agents};
     const int64_t str[3] = {D, (int64_t)p->num_kv_heads * D, (int64_t)RK * p->num_kv_heads * D};
-    const uint32_t box[4] = {(uint32_t)D, 1, (uint32_t)RK, 1};
-    if ((s = make_map4(&maps[3], b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE, "B")) != LRKV_OK) return s;
+    const uint32_t box[4] = {64, 1, (uint32_t)RK, 1};
+    if ((s = make_map4(&maps[3], b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "B")) != LRKV_OK) return s;
   }
   lrkv::PrefillParams pp = {};
   pp.q = q;
@@ -536,13 +541,19 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
   pp.L0 = ctx_len;
   pp.session = session;
   pp.mode = p->mode;
-  pp.n_tb = (T + TM - 1) / TM;
   pp.scale_log2 = scale_of(p) * 1.4426950408889634f;
   pp.flags = static_cast<unsigned*>(workspace);
-  const long long grid = (long long)p->num_kv_heads * p->num_agents * pp.n_tb;
-  if (grid > 0x7fffffffLL) return fail(LRKV_ERR_UNSUPPORTED, "too many prefill tiles");
+  const lrkv::PrefillPlan pl = lrkv::plan_prefill(T, ctx_len, G, p->num_kv_heads, p->num_agents, D, RK, dev.sms);
+  if (workspace_bytes < pl.bytes)
+    return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes (lrkv_prefill_workspace_bytes)", workspace_bytes, pl.bytes);
+  pp.n_tb = pl.n_tb;
+  pp.W_ga = pl.W_ga;
+  pp.W = pl.W;
+  pp.max_parts = pl.max_parts;
+  pp.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + pl.tickets_off);
+  pp.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pl.partials_off);
   lrkv::PrefillMaps pm = {maps};
-  s = lrkv::launch_prefill(pp, pm, D, RK, (int)grid, stream);
+  s = lrkv::launch_prefill(pp, pm, D, RK, pl.ctas, stream);
   if (s != LRKV_OK) return fail(s, "prefill launch failed: %s", cudaGetErrorString(cudaGetLastError()));
   return LRKV_OK;
 }

@@ -19,7 +19,22 @@ struct PrefillParams {
   int n_tb;                  // 128-row tiles per (KV head, agent)
   float scale_log2;
   unsigned* flags;
+  // stream-K split of the (tile, 128-key block) pairs over the CTAs
+  long long W_ga;            // blocks of the n_tb tiles of one (KV head, agent)
+  long long W;               // blocks in all
+  int max_parts;             // CTAs that can share one tile
+  int* tickets;              // [tiles], zero between launches
+  float* partials;           // [tiles][max_parts][128 rows: m, l, O + Z B (d)]
 };
+
+// Stream-K plan of a prefill launch and its workspace (bytes from the start of
+// the workspace: the status header, tickets, partial records).
+struct PrefillPlan {
+  int n_tb, tiles, ctas, max_parts;
+  long long W_ga, W;
+  size_t tickets_off, partials_off, bytes;
+};
+PrefillPlan plan_prefill(int T, int L0, int G, int Hkv, int N, int D, int RK, int sms);
 
 // Four CUtensorMap objects, in order: K, V, U, B.
 struct PrefillMaps {
