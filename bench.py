@@ -270,35 +270,44 @@ def _timed(fn, steps, warmup, sync_all):
     return e0.elapsed_time(e1)
 
 
-def cpu_baseline_decode(runner, max_seconds=20.0):
-    """fp64 oracle on the host cores: sessions x all layers until about max_seconds."""
+def cpu_baseline_decode(runner, min_seconds=10.0, max_seconds=25.0):
+    """fp64 oracle on the host cores: session after session, each through all
+    layers, until at least min_seconds of oracle time (at most max_seconds).
+    Only the oracle calls are timed, not the copies of the inputs to the host."""
     import oracle
     from threadpoolctl import threadpool_info
     cfg, inp = runner.cfg, runner.inp
     cores = len(os.sched_getaffinity(0))
     blas_threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    host = []
-    for lay in inp.layers:
-        if cfg.paged:
-            host.append(None)
-        else:
-            host.append((lay.q[:1].cpu(), lay.k[:1].cpu(), lay.v[:1].cpu(), lay.u[:1].cpu(), lay.b.cpu()))
-    offs = inp.offsets[:1].cpu()
-    sl = inp.seq_lens[:1].cpu()
-    t0 = time.perf_counter()
+    dt = 0.0
     done_layers = 0
-    for li in range(len(inp.layers)):
-        q, k, v, u, b = host[li]
-        oracle.decode(q, k, v, u, b, offs, sl, cfg.mode)
-        done_layers += 1
-        if time.perf_counter() - t0 > max_seconds:
+    sessions = 0
+    for s in range(cfg.S):
+        offs = inp.offsets[s:s + 1].cpu()
+        sl = inp.seq_lens[s:s + 1].cpu()
+        for lay in inp.layers:
+            q, u, b = lay.q[s:s + 1].cpu(), lay.u[s:s + 1].cpu(), lay.b.cpu()
+            if cfg.paged:  # this session's pages, in logical order
+                pt = lay.page_table[s].long()
+                k, v = lay.k[pt].cpu(), lay.v[pt].cpu()
+                table = torch.arange(pt.numel(), dtype=torch.int32).view(1, -1)
+            else:
+                k, v, table = lay.k[s:s + 1].cpu(), lay.v[s:s + 1].cpu(), None
+            t0 = time.perf_counter()
+            oracle.decode(q, k, v, u, b, offs, sl, cfg.mode, page_table=table)
+            dt += time.perf_counter() - t0
+            done_layers += 1
+            if dt > max_seconds:
+                break
+        sessions += 1
+        if dt > min_seconds:
             break
-    dt = time.perf_counter() - t0
     queries = cfg.N * done_layers / len(inp.layers)
     return {"value": queries / dt, "unit": UNIT, "cores": min(cores, blas_threads) if blas_threads else cores,
             "kind": "oracle",
-            "sample": f"session 0 ({cfg.N} queries) x {done_layers} of {len(inp.layers)} layers, fp64 numpy, "
-                      f"{dt:.1f} s; {cores} cores visible, BLAS threads {blas_threads}"}
+            "sample": f"{sessions} session(s) x {len(inp.layers)} layers ({done_layers} session-layers, "
+                      f"{queries:.1f} queries), fp64 numpy, {dt:.1f} s of oracle time; {cores} cores visible, "
+                      f"BLAS threads {blas_threads}"}
 
 
 def run_e2e(runner, steps, warmup, sync_all):
