@@ -149,6 +149,27 @@ lrkv_status lrkv_append_lr_cache(const void* x, const void* a, int32_t n_a, int3
                                  int32_t Dm, int32_t r, const lrkv_u_view* u_dst,
                                  int32_t session, int32_t start_row, lrkv_stream_t stream);
 
+/*
+ * Catch-up append over per-agent ranges: for every agent slot i in [0, n_a),
+ * U_i[t, :] = X[t, :] A_i for t in [row_begin[i], row_end[i]) of session
+ * `session` of u_dst (LRAgent page, Fig. 3(a): in BaseShared every agent
+ * computes its own rank-r cache for the context tokens it has not processed
+ * yet, so the ranges differ per agent; Fig. 3(b): in BaseLRShared the one
+ * shared U is appended once: n_a = 1).  X row t is the hidden state of
+ * absolute position t.
+ *   x          device bf16 [x_rows, Dm], row-major
+ *   a          device bf16 [n_a, Dm, r], row-major
+ *   row_begin, row_end   HOST int32 [n_a] (the caller's scheduler knows them)
+ * Same fixed-order numerics as lrkv_append_lr_cache (bit-determined).  Rows
+ * outside each agent's range are not written.  Empty ranges are no-ops.
+ * Errors: a range with row_begin < 0, row_begin > row_end, row_end > x_rows or
+ * row_end > u_dst->num_rows, n_a < 1, Dm < 1 return LRKV_ERR_INVALID_ARGUMENT;
+ * r not in {8, 16, 32} returns LRKV_ERR_UNSUPPORTED.
+ */
+lrkv_status lrkv_append_lr_cache_ranges(const void* x, int32_t x_rows, const void* a, int32_t n_a, int32_t Dm,
+                                        int32_t r, const int32_t* row_begin, const int32_t* row_end,
+                                        const lrkv_u_view* u_dst, int32_t session, lrkv_stream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* Decode: one query token per (session, agent) over the shared cache.     */
 /* ---------------------------------------------------------------------- */

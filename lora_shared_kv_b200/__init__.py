@@ -42,6 +42,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblrkv.so"
 # Every exported symbol of include/lrkv.h.
 EXPORTS = (
     "lrkv_append_lr_cache",
+    "lrkv_append_lr_cache_ranges",
     "lrkv_decode_workspace_bytes",
     "lrkv_attn_decode",
     "lrkv_attn_decode_static_scratch",
@@ -96,6 +97,7 @@ def lib():
         P = ctypes.POINTER
         vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         L.lrkv_append_lr_cache.argtypes = [vp, vp, i32, i32, i32, i32, P(UView), i32, i32, vp]
+        L.lrkv_append_lr_cache_ranges.argtypes = [vp, i32, vp, i32, i32, i32, P(i32), P(i32), P(UView), i32, vp]
         L.lrkv_decode_workspace_bytes.argtypes = [P(Problem), i32]
         L.lrkv_decode_workspace_bytes.restype = sz
         L.lrkv_attn_decode.argtypes = [P(Problem), vp, P(KVView), vp, i32, P(UView), vp, vp, vp, i32, vp, sz, vp]
@@ -177,6 +179,20 @@ def lrkv_append_lr_cache(x, a, u, session, start_row, stream=None, uview=None):
     uv = uview if uview is not None else u_view(u)
     _check(lib().lrkv_append_lr_cache(_ptr(x), _ptr(a), n_a, T, Dm, r, ctypes.byref(uv), session, start_row,
                                       _stream(stream)))
+
+
+def lrkv_append_lr_cache_ranges(x, a, u, session, row_begin, row_end, stream=None, uview=None):
+    """U[session, i, t, :] = x[t] @ a[i] for t in [row_begin[i], row_end[i]) of every slot i of a:
+    the per-agent catch-up append (bit-exact fixed order).  x holds the hidden states by absolute position."""
+    x_rows, Dm = x.shape
+    n_a, Dm2, r = a.shape
+    assert Dm == Dm2 and x.is_contiguous() and a.is_contiguous()
+    assert len(row_begin) == n_a and len(row_end) == n_a
+    uv = uview if uview is not None else u_view(u)
+    b = (ctypes.c_int32 * n_a)(*[int(v) for v in row_begin])
+    e = (ctypes.c_int32 * n_a)(*[int(v) for v in row_end])
+    _check(lib().lrkv_append_lr_cache_ranges(_ptr(x), x_rows, _ptr(a), n_a, Dm, r, b, e, ctypes.byref(uv),
+                                             session, _stream(stream)))
 
 
 def lrkv_decode_workspace_bytes(problem, max_seq_len):

@@ -1,4 +1,6 @@
-// Low-rank cache append: U_i[start + t, :] = X[t, :] A_i for new tokens.
+// Low-rank cache append: U_i[t + shift, :] = X[t, :] A_i for the rows t of
+// each agent's range: a contiguous block of new tokens for every agent, or
+// per-agent ranges (the tokens each agent has not processed yet).
 //
 // The rank-r cache X A_i is the adapter half of the split value projection
 // (Eq. 3 of "LRAgent: Efficient KV Cache Sharing for Multi-LoRA LLM Agents");
@@ -26,6 +28,15 @@ namespace {
 constexpr int APP_THREADS = 128;
 constexpr int KC = 64;  // k per chunk
 
+// The x rows of each agent of one launch (agent agent_base + blockIdx.y):
+// block x covers rows begin + TB * blockIdx.x ..; U row = x row + u_shift.
+struct AppendRows {
+  int begin[kMaxAgents];
+  int end[kMaxAgents];
+  int agent_base;
+  int u_shift;
+};
+
 template <int R>
 struct AppShape {
   static constexpr int CG = R / 8;                      // column groups of 8
@@ -38,17 +49,19 @@ struct AppShape {
 
 template <int R>
 __global__ void __launch_bounds__(APP_THREADS)
-    append_kernel_generic(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int T, int Dm,
-                  __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st, int session,
-                  int start_row) {
+    append_kernel_generic(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, const AppendRows rows,
+                          int Dm, __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st,
+                          int session) {
   using S = AppShape<R>;
   __shared__ float xs[KC * S::XS];                // xs[k * XS + token]
   __shared__ __align__(16) float as[KC * R];      // as[k * R + column]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cg = warp % S::CG;                    // this warp's 8 columns: [8 cg, 8 cg + 8)
   const int tl = (warp / S::CG) * 32 + lane;      // this thread's token within the block
-  const int agent = blockIdx.y;
-  const int t0 = blockIdx.x * S::TB;
+  const int agent = rows.agent_base + blockIdx.y;
+  const int T = rows.end[blockIdx.y];
+  const int t0 = rows.begin[blockIdx.y] + blockIdx.x * S::TB;
+  if (t0 >= T) return;  // past this agent's range (block-uniform)
   const uint16_t* a_ag = a + (size_t)agent * Dm * R;
 
   // staging: chunk element e = tid + i * APP_THREADS of X sits at token e / KC,
@@ -114,19 +127,20 @@ __global__ void __launch_bounds__(APP_THREADS)
   }
   const int t = t0 + tl;
   if (t < T) {
-    __nv_bfloat16* dst = u + (size_t)session * u_ss + (size_t)agent * u_sa + (size_t)(start_row + t) * u_st + cg * 8;
+    __nv_bfloat16* dst = u + (size_t)session * u_ss + (size_t)agent * u_sa + (size_t)(t + rows.u_shift) * u_st + cg * 8;
 #pragma unroll
     for (int c = 0; c < 8; ++c) dst[c] = __float2bfloat16_rn(acc[c]);
   }
 }
 
 template <int R>
-void launch_generic(const void* x, const void* a, int n_a, int T, int Dm, void* u, long long u_ss, long long u_sa,
-              long long u_st, int session, int start_row, cudaStream_t stream) {
-  dim3 grid((T + AppShape<R>::TB - 1) / AppShape<R>::TB, n_a);
-  append_kernel_generic<R><<<grid, APP_THREADS, 0, stream>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(a),
-                                                     T, Dm, static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st,
-                                                     session, start_row);
+void launch_generic(const void* x, const void* a, const AppendRows& rows, int n, int max_len, int Dm, void* u,
+                    long long u_ss, long long u_sa, long long u_st, int session, cudaStream_t stream) {
+  dim3 grid((max_len + AppShape<R>::TB - 1) / AppShape<R>::TB, n);
+  append_kernel_generic<R><<<grid, APP_THREADS, 0, stream>>>(static_cast<const uint16_t*>(x),
+                                                             static_cast<const uint16_t*>(a), rows, Dm,
+                                                             static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st,
+                                                             session);
 }
 
 // ---------------------------------------------------------------------------
@@ -156,9 +170,8 @@ struct FastShape {
 
 template <int R>
 __global__ void __launch_bounds__(APP_THREADS)
-    append_kernel_fast(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, int T, int Dm,
-                       __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st, int session,
-                       int start_row) {
+    append_kernel_fast(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, const AppendRows rows, int Dm,
+                       __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st, int session) {
   using S = FastShape<R>;
   __shared__ __align__(16) uint16_t xr[F_NS][S::TB * F_XP];
   __shared__ __align__(16) uint16_t ar[F_NS][F_KC * S::CB];
@@ -166,8 +179,10 @@ __global__ void __launch_bounds__(APP_THREADS)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cg = warp % S::CGB;
   const int tl = (warp / S::CGB) * 32 + lane;  // token within the block
-  const int agent = blockIdx.y;
-  const int t0 = blockIdx.x * S::TB;
+  const int agent = rows.agent_base + blockIdx.y;
+  const int T = rows.end[blockIdx.y];
+  const int t0 = rows.begin[blockIdx.y] + blockIdx.x * S::TB;
+  if (t0 >= T) return;  // past this agent's range (block-uniform)
   const int c0 = blockIdx.z * S::CB;           // first column of the block
   const uint16_t* a_ag = a + (size_t)agent * Dm * R;
   const int n_chunks = (Dm + F_KC - 1) / F_KC;
@@ -228,7 +243,7 @@ __global__ void __launch_bounds__(APP_THREADS)
   const int t = t0 + tl;
   if (t < T) {
     __nv_bfloat16* dst =
-        u + (size_t)session * u_ss + (size_t)agent * u_sa + (size_t)(start_row + t) * u_st + c0 + cg * 4;
+        u + (size_t)session * u_ss + (size_t)agent * u_sa + (size_t)(t + rows.u_shift) * u_st + c0 + cg * 4;
     dst[0] = __float2bfloat16_rn(acc0);
     dst[1] = __float2bfloat16_rn(acc1);
     dst[2] = __float2bfloat16_rn(acc2);
@@ -237,34 +252,47 @@ __global__ void __launch_bounds__(APP_THREADS)
 }
 
 template <int R>
-void launch_r(const void* x, const void* a, int n_a, int T, int Dm, void* u, long long u_ss, long long u_sa,
-              long long u_st, int session, int start_row, cudaStream_t stream) {
+void launch_r(const void* x, const void* a, const AppendRows& rows, int n, int max_len, int Dm, void* u,
+              long long u_ss, long long u_sa, long long u_st, int session, cudaStream_t stream) {
   const bool fast = Dm % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 && (reinterpret_cast<uintptr_t>(a) & 15) == 0;
   if (!fast) {
-    launch_generic<R>(x, a, n_a, T, Dm, u, u_ss, u_sa, u_st, session, start_row, stream);
+    launch_generic<R>(x, a, rows, n, max_len, Dm, u, u_ss, u_sa, u_st, session, stream);
     return;
   }
   using S = FastShape<R>;
-  dim3 grid((T + S::TB - 1) / S::TB, n_a, S::NCB);
+  dim3 grid((max_len + S::TB - 1) / S::TB, n, S::NCB);
   append_kernel_fast<R><<<grid, APP_THREADS, 0, stream>>>(static_cast<const uint16_t*>(x),
-                                                          static_cast<const uint16_t*>(a), T, Dm,
-                                                          static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st,
-                                                          session, start_row);
+                                                          static_cast<const uint16_t*>(a), rows, Dm,
+                                                          static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st, session);
 }
 
 }  // namespace
 
-lrkv_status launch_append(const void* x, const void* a, int n_a, int T, int Dm, int r, void* u, long long u_ss,
-                          long long u_sa, long long u_st, int session, int start_row, void* stream) {
-  if (T == 0) return LRKV_OK;
+lrkv_status launch_append(const void* x, const void* a, int n_a, const int* row_begin, const int* row_end,
+                          int u_shift, int Dm, int r, void* u, long long u_ss, long long u_sa, long long u_st,
+                          int session, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  switch (r) {
-    case 8: launch_r<8>(x, a, n_a, T, Dm, u, u_ss, u_sa, u_st, session, start_row, st); break;
-    case 16: launch_r<16>(x, a, n_a, T, Dm, u, u_ss, u_sa, u_st, session, start_row, st); break;
-    case 32: launch_r<32>(x, a, n_a, T, Dm, u, u_ss, u_sa, u_st, session, start_row, st); break;
-    default: return LRKV_ERR_UNSUPPORTED;
+  for (int base = 0; base < n_a; base += kMaxAgents) {  // the ranges of up to kMaxAgents agents per launch
+    AppendRows rows = {};
+    rows.agent_base = base;
+    rows.u_shift = u_shift;
+    const int n = n_a - base < kMaxAgents ? n_a - base : kMaxAgents;
+    int max_len = 0;
+    for (int i = 0; i < n; ++i) {
+      rows.begin[i] = row_begin[base + i];
+      rows.end[i] = row_end[base + i];
+      max_len = rows.end[i] - rows.begin[i] > max_len ? rows.end[i] - rows.begin[i] : max_len;
+    }
+    if (max_len == 0) continue;
+    switch (r) {
+      case 8: launch_r<8>(x, a, rows, n, max_len, Dm, u, u_ss, u_sa, u_st, session, st); break;
+      case 16: launch_r<16>(x, a, rows, n, max_len, Dm, u, u_ss, u_sa, u_st, session, st); break;
+      case 32: launch_r<32>(x, a, rows, n, max_len, Dm, u, u_ss, u_sa, u_st, session, st); break;
+      default: return LRKV_ERR_UNSUPPORTED;
+    }
+    if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+  return LRKV_OK;
 }
 
 }  // namespace lrkv

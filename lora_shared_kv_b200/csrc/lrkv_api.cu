@@ -10,6 +10,8 @@
 
 #include <mutex>
 
+#include <vector>
+
 #include "lrkv_internal.h"
 #include "prefill.h"
 
@@ -281,8 +283,38 @@ lrkv_status lrkv_append_lr_cache(const void* x, const void* a, int32_t n_a, int3
   DeviceInfo dev;
   lrkv_status s = device_info(&dev);
   if (s != LRKV_OK) return s;
-  s = lrkv::launch_append(x, a, n_a, T, Dm, r, u_dst->u, u_dst->stride_session, u_dst->stride_agent,
-                          u_dst->stride_token, session, start_row, stream);
+  std::vector<int> begin(n_a, 0), end(n_a, T);
+  s = lrkv::launch_append(x, a, n_a, begin.data(), end.data(), start_row, Dm, r, u_dst->u, u_dst->stride_session,
+                          u_dst->stride_agent, u_dst->stride_token, session, stream);
+  if (s != LRKV_OK) return fail(s, "append launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+  return LRKV_OK;
+}
+
+lrkv_status lrkv_append_lr_cache_ranges(const void* x, int32_t x_rows, const void* a, int32_t n_a, int32_t Dm,
+                                        int32_t r, const int32_t* row_begin, const int32_t* row_end,
+                                        const lrkv_u_view* u_dst, int32_t session, lrkv_stream_t stream) {
+  if (!x || !a || !u_dst || !u_dst->u || !row_begin || !row_end)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "x, a, row_begin, row_end and u_dst->u must not be NULL");
+  if (x_rows < 0 || Dm < 1 || n_a < 1 || session < 0)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "need x_rows >= 0, Dm >= 1, n_a >= 1, session >= 0");
+  if (r != 8 && r != 16 && r != 32) return fail(LRKV_ERR_UNSUPPORTED, "rank %d (supported: 8, 16, 32)", r);
+  if (u_dst->stride_token < r) return fail(LRKV_ERR_INVALID_ARGUMENT, "u stride_token < rank");
+  if (n_a > 1 && u_dst->stride_agent < 1) return fail(LRKV_ERR_INVALID_ARGUMENT, "u stride_agent must be >= 1 when n_a > 1");
+  if (session > 0 && u_dst->stride_session < 1) return fail(LRKV_ERR_INVALID_ARGUMENT, "u stride_session must be >= 1");
+  bool any = false;
+  for (int i = 0; i < n_a; ++i) {
+    if (row_begin[i] < 0 || row_begin[i] > row_end[i])
+      return fail(LRKV_ERR_INVALID_ARGUMENT, "agent %d: need 0 <= row_begin <= row_end (got %d, %d)", i, row_begin[i], row_end[i]);
+    if (row_end[i] > x_rows || row_end[i] > u_dst->num_rows)
+      return fail(LRKV_ERR_INVALID_ARGUMENT, "agent %d: row_end %d exceeds x_rows %d or the U capacity %d", i, row_end[i], x_rows, u_dst->num_rows);
+    any = any || row_end[i] > row_begin[i];
+  }
+  if (!any) return LRKV_OK;
+  DeviceInfo dev;
+  lrkv_status s = device_info(&dev);
+  if (s != LRKV_OK) return s;
+  s = lrkv::launch_append(x, a, n_a, row_begin, row_end, 0, Dm, r, u_dst->u, u_dst->stride_session,
+                          u_dst->stride_agent, u_dst->stride_token, session, stream);
   if (s != LRKV_OK) return fail(s, "append launch failed: %s", cudaGetErrorString(cudaGetLastError()));
   return LRKV_OK;
 }

@@ -90,6 +90,25 @@ def test_append_argument_errors():
     assert L.lrkv_append_lr_cache(None, None, 1, 1, 1, 16, None, 0, 0, None) == 1
 
 
+def test_append_ranges_argument_errors():
+    L = lrkv.lib()
+    uv = lrkv.UView(FAKE, 0, 100 * 16, 16, 100)
+
+    def f(begin, end, x_rows=100, r=16, Dm=64):
+        n = len(begin)
+        b = (ctypes.c_int32 * n)(*begin)
+        e = (ctypes.c_int32 * n)(*end)
+        return L.lrkv_append_lr_cache_ranges(ctypes.c_void_p(FAKE), x_rows, ctypes.c_void_p(FAKE), n, Dm, r, b, e,
+                                             ctypes.byref(uv), 0, None)
+    assert f([5, 0], [4, 10]) == 1         # begin > end
+    assert f([-1], [3]) == 1               # negative begin
+    assert f([0], [101]) == 1              # past the U capacity
+    assert f([0], [60], x_rows=50) == 1    # past the hidden states given
+    assert f([0], [10], r=12) == 2         # unsupported rank
+    assert f([3, 7], [3, 7]) == 0          # all ranges empty: a no-op, no launch
+    assert L.lrkv_append_lr_cache_ranges(None, 1, None, 1, 1, 16, None, None, None, 0, None) == 1
+
+
 def test_workspace_bytes_shape_rules():
     # without a device the plan falls back to 148 SMs; invalid shapes give 0
     assert lrkv.lib().lrkv_decode_workspace_bytes(ctypes.byref(_problem(d=96)), 128) == 0
