@@ -50,6 +50,7 @@ __all__ = [
     "decode",
     "prefill_chunk",
     "ref_append_fp32",
+    "value_projection",
 ]
 
 BASE_SHARED = 0
@@ -279,3 +280,29 @@ def ref_append_fp32(x, a) -> np.ndarray:
             acc = (acc + prod).astype(np.float32)
         out[ag] = f32_to_bf16_bits_rne(acc)
     return out
+
+
+# --------------------------------------------------------------------------
+# the value projection with the adapters' down-projections side by side
+# --------------------------------------------------------------------------
+
+def value_projection(x, w, num_kv_heads: int, head_dim: int, n_u: int, rank: int):
+    """[V_base | U_1 ... U_n] = X [W0_v | A_1 ... A_n], in float64.
+
+    Eq. 3 of the LRAgent page splits the value projection of agent i as
+    X W0 + (X A_i) B_i: the base value cache X W0 is shared and U_i = X A_i is
+    the agent's rank-r cache.  Both come from the same hidden states, so one
+    product with the weights side by side yields the base values and every
+    agent's (or, with one shared A, the one) U rows.
+    x [T, Dm]; w [Dm, Hkv * d + n_u * r], columns: W0_v (KV head g in
+    [g d, (g + 1) d)), then A_1, ..., A_n (r columns each).
+    Returns v [Hkv, T, d] and u [n_u, T, r].
+    """
+    x64 = to_f64(x)
+    w64 = to_f64(w)
+    T = x64.shape[0]
+    hd = num_kv_heads * head_dim
+    y = x64 @ w64
+    v = y[:, :hd].reshape(T, num_kv_heads, head_dim).transpose(1, 0, 2)
+    u = y[:, hd:hd + n_u * rank].reshape(T, n_u, rank).transpose(1, 0, 2)
+    return v, u

@@ -296,9 +296,37 @@ def pin_nan_rows_selected_out(mod):
     return bool(np.all(np.isfinite(out)) and np.array_equal(out, ref))
 
 
+def pin_value_projection(mod):
+    """[V_base | U_1 .. U_n] = X [W0_v | A_1 .. A_n]: element by element on small
+    integers (exact), and the split caches it yields rebuild the unsplit projection."""
+    g = _rng(41)
+    T, Dm, Hkv, d, n, r = 3, 5, 2, 3, 2, 2
+    X = g.integers(-3, 4, (T, Dm)).astype(np.float64)
+    W = g.integers(-3, 4, (Dm, Hkv * d + n * r)).astype(np.float64)
+    v, u = mod.value_projection(X, W, Hkv, d, n, r)
+    ok = v.shape == (Hkv, T, d) and u.shape == (n, T, r)
+    for t in range(T):
+        for gg in range(Hkv):
+            for c in range(d):
+                ok &= v[gg, t, c] == sum(X[t, k] * W[k, gg * d + c] for k in range(Dm))
+        for i in range(n):
+            for j in range(r):
+                ok &= u[i, t, j] == sum(X[t, k] * W[k, Hkv * d + i * r + j] for k in range(Dm))
+    # Eq. 3: V_base + U_i B_i = X (W0 + A_i B_i)
+    Xf = g.standard_normal((6, 7))
+    W0 = g.standard_normal((7, Hkv * d))
+    A = [g.standard_normal((7, r)) for _ in range(n)]
+    B = [g.standard_normal((r, Hkv * d)) for _ in range(n)]
+    v, u = mod.value_projection(Xf, np.concatenate([W0] + A, axis=1), Hkv, d, n, r)
+    for i in range(n):
+        unsplit = (Xf @ (W0 + A[i] @ B[i])).reshape(6, Hkv, d).transpose(1, 0, 2)
+        ok &= _close(mod.agent_value_cache(v, mod.masked_lr_cache(u[i], 0), B[i]), unsplit, 1e-12)
+    return bool(ok)
+
+
 ALL_PINS = [pin_decomposition, pin_reordering, pin_sdpa_decode, pin_sdpa_prefill,
             pin_rows_before_offset, pin_brute_decode, pin_brute_prefill, pin_shared_a,
-            pin_closed_forms, pin_paged, pin_nan_rows_selected_out]
+            pin_closed_forms, pin_paged, pin_nan_rows_selected_out, pin_value_projection]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=[p.__name__ for p in ALL_PINS])
@@ -423,6 +451,19 @@ def _mut_no_scale(d, scale):
 
 
 _ORIG_ATTN = O.attention_rows
+_ORIG_VPROJ = O.value_projection
+
+
+def _mut_u_from_front(x, w, Hkv, d, n, r):
+    v, _ = _ORIG_VPROJ(x, w, Hkv, d, n, r)
+    y = O.to_f64(x) @ O.to_f64(w)
+    return v, y[:, :n * r].reshape(y.shape[0], n, r).transpose(1, 0, 2)
+
+
+def _mut_dim_major_heads(x, w, Hkv, d, n, r):
+    _, u = _ORIG_VPROJ(x, w, Hkv, d, n, r)
+    y = O.to_f64(x) @ O.to_f64(w)
+    return y[:, :Hkv * d].reshape(y.shape[0], d, Hkv).transpose(2, 0, 1), u
 
 MUTANTS = [
     ("masked_lr_cache", _mut_exclusive_offset),
@@ -433,6 +474,8 @@ MUTANTS = [
     ("attention_rows", _mut_exclude_diagonal),
     ("attention_rows", _mut_unnormalised),
     ("_scale", _mut_no_scale),
+    ("value_projection", _mut_u_from_front),
+    ("value_projection", _mut_dim_major_heads),
 ]
 
 
