@@ -274,6 +274,37 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
 /* ---------------------------------------------------------------------- */
 /* Workspace and status.                                                   */
 /* ---------------------------------------------------------------------- */
+/* Value projection into the split caches.                                 */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * [V_base | U_1 ... U_n] = X [W0_v | A_1 ... A_n] for T new tokens, written
+ * into the caches: base value rows start_row .. start_row+T-1 of session
+ * `session` for every KV head (kv->v; kv->k is not touched), and the same rows
+ * of every low-rank slot of u_dst (LRAgent page, Eq. 3: agent i's value
+ * projection splits as X W0 + (X A_i) B_i, so one product with the weights side
+ * by side gives the shared base values and all U_i rows).
+ *   x        device bf16 [T, Dm] row-major, Dm % 8 == 0
+ *   w        device bf16 [Dm, Hkv*d + n_u*r] row-major: W0_v (KV head g in
+ *            columns [g d, (g+1) d)), then A_1 .. A_{n_u} (r columns each);
+ *            n_u = N in BaseShared, 1 in BaseLRShared
+ *   kv       dense: kv_rows is the row capacity of each (session, head);
+ *            paged: rows map through the session's page-table row
+ *   workspace  device, >= 256 bytes, zero-filled once: status flags
+ * Numerics: bf16 inputs, fp32 accumulation on the tensor cores in an
+ * unspecified order, round to nearest even bf16.  The U rows are therefore not
+ * bit-identical to lrkv_append_lr_cache's fixed-order ones.
+ * Errors: invalid shapes or rows past the caches return
+ * LRKV_ERR_INVALID_ARGUMENT, unaligned pointers or strides LRKV_ERR_MISALIGNED;
+ * an out-of-range page id sets a device flag (lrkv_query_device_status) and
+ * that row's values are not written.  T == 0 is a no-op.
+ */
+lrkv_status lrkv_value_projection(const lrkv_problem* p, const void* x, int32_t T, int32_t Dm, const void* w,
+                                  const lrkv_kv_view* kv, int32_t kv_rows, const lrkv_u_view* u_dst,
+                                  int32_t session, int32_t start_row, void* workspace, size_t workspace_bytes,
+                                  lrkv_stream_t stream);
+
+/* ---------------------------------------------------------------------- */
 
 /* Zero-fill a workspace on `stream` (asynchronous). */
 lrkv_status lrkv_workspace_reset(void* workspace, size_t workspace_bytes, lrkv_stream_t stream);

@@ -43,6 +43,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblrkv.so"
 EXPORTS = (
     "lrkv_append_lr_cache",
     "lrkv_append_lr_cache_ranges",
+    "lrkv_value_projection",
     "lrkv_decode_workspace_bytes",
     "lrkv_attn_decode",
     "lrkv_attn_decode_static_scratch",
@@ -98,6 +99,8 @@ def lib():
         vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         L.lrkv_append_lr_cache.argtypes = [vp, vp, i32, i32, i32, i32, P(UView), i32, i32, vp]
         L.lrkv_append_lr_cache_ranges.argtypes = [vp, i32, vp, i32, i32, i32, P(i32), P(i32), P(UView), i32, vp]
+        L.lrkv_value_projection.argtypes = [P(Problem), vp, i32, i32, vp, P(KVView), i32, P(UView), i32, i32, vp, sz,
+                                            vp]
         L.lrkv_decode_workspace_bytes.argtypes = [P(Problem), i32]
         L.lrkv_decode_workspace_bytes.restype = sz
         L.lrkv_attn_decode.argtypes = [P(Problem), vp, P(KVView), vp, i32, P(UView), vp, vp, vp, i32, vp, sz, vp]
@@ -193,6 +196,17 @@ def lrkv_append_lr_cache_ranges(x, a, u, session, row_begin, row_end, stream=Non
     e = (ctypes.c_int32 * n_a)(*[int(v) for v in row_end])
     _check(lib().lrkv_append_lr_cache_ranges(_ptr(x), x_rows, _ptr(a), n_a, Dm, r, b, e, ctypes.byref(uv),
                                              session, _stream(stream)))
+
+
+def lrkv_value_projection(problem, x, w, kv, kv_rows, u, session, start_row, workspace, stream=None):
+    """[V_base | U_1..U_n] = x @ w for T new tokens, written into kv.v rows and u rows
+    [start_row, start_row + T) of `session` (x [T, Dm], w [Dm, Hkv*d + n_u*r])."""
+    T, Dm = x.shape
+    assert x.is_contiguous() and w.is_contiguous() and w.shape[0] == Dm
+    uv = u if isinstance(u, UView) else u_view(u)
+    _check(lib().lrkv_value_projection(ctypes.byref(problem), _ptr(x), T, Dm, _ptr(w), ctypes.byref(kv), int(kv_rows),
+                                       ctypes.byref(uv), session, start_row, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def lrkv_decode_workspace_bytes(problem, max_seq_len):

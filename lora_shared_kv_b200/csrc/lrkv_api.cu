@@ -239,6 +239,81 @@ const char* lrkv_last_error_detail(void) { return g_detail; }
 
 int32_t lrkv_version(void) { return 100; }
 
+lrkv_status lrkv_value_projection(const lrkv_problem* p, const void* x, int32_t T, int32_t Dm, const void* w,
+                                  const lrkv_kv_view* kv, int32_t kv_rows, const lrkv_u_view* u_dst,
+                                  int32_t session, int32_t start_row, void* workspace, size_t workspace_bytes,
+                                  lrkv_stream_t stream) {
+  lrkv_status s = check_problem(p);
+  if (s != LRKV_OK) return s;
+  if (!x || !w || !kv || !kv->v || !u_dst || !u_dst->u || !workspace)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "x, w, kv->v, u_dst->u and workspace must not be NULL");
+  if (T < 0 || Dm < 1 || session < 0 || start_row < 0)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "need T >= 0, Dm >= 1, session >= 0, start_row >= 0");
+  if (!kv->page_table && session >= p->num_sessions)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "session %d >= num_sessions %d", session, p->num_sessions);
+  if (Dm % 8) return fail(LRKV_ERR_MISALIGNED, "Dm must be a multiple of 8 (16-byte rows of x)");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(kv->v) || !aligned16(u_dst->u) || !aligned16(workspace))
+    return fail(LRKV_ERR_MISALIGNED, "x, w, kv->v, u and workspace must be 16-byte aligned");
+  if (workspace_bytes < (size_t)lrkv::kWsHeaderBytes)
+    return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %d bytes", workspace_bytes, lrkv::kWsHeaderBytes);
+  if ((kv->stride_token % 8) || (kv->stride_head % 8) || (!kv->page_table && (kv->stride_session % 8)) ||
+      (kv->page_table && (kv->stride_page % 8)))
+    return fail(LRKV_ERR_MISALIGNED, "kv strides must be multiples of 8 elements");
+  const int n_u = p->mode == LRKV_BASE_SHARED ? p->num_agents : 1;
+  if ((s = check_u(u_dst, p, start_row + T)) != LRKV_OK) return s;
+  if (kv->page_table) {
+    if (kv->page_size < 1 || kv->num_pages < 1) return fail(LRKV_ERR_INVALID_ARGUMENT, "paged view needs page_size and num_pages");
+    if ((long long)(start_row + T + kv->page_size - 1) / kv->page_size > kv->page_table_stride)
+      return fail(LRKV_ERR_INVALID_ARGUMENT, "rows past the session's page-table row");
+  } else if (start_row + T > kv_rows) {
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "rows [%d, %d) exceed the value cache's %d rows", start_row, start_row + T, kv_rows);
+  }
+  if (T == 0) return LRKV_OK;
+  DeviceInfo dev;
+  if ((s = device_info(&dev)) != LRKV_OK) return s;
+  const int ncols = p->num_kv_heads * p->head_dim + n_u * p->rank;
+  alignas(64) CUtensorMap maps[2];
+  {  // X [T, Dm]: box 64 k x 128 tokens
+    const uint64_t dims[4] = {(uint64_t)Dm, (uint64_t)T, 1, 1};
+    const int64_t str[3] = {Dm, 0, 0};
+    const uint32_t box[4] = {64, 128, 1, 1};
+    if ((s = make_map4(&maps[0], x, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "X")) != LRKV_OK) return s;
+  }
+  {  // W [Dm, ncols]: box 64 columns x 64 k
+    const uint64_t dims[4] = {(uint64_t)ncols, (uint64_t)Dm, 1, 1};
+    const int64_t str[3] = {ncols, 0, 0};
+    const uint32_t box[4] = {64, 64, 1, 1};
+    if ((s = make_map4(&maps[1], w, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "W")) != LRKV_OK) return s;
+  }
+  lrkv::VprojParams vp = {};
+  vp.T = T;
+  vp.Dm = Dm;
+  vp.Hkv = p->num_kv_heads;
+  vp.d = p->head_dim;
+  vp.n_u = n_u;
+  vp.r = p->rank;
+  vp.ncols = ncols;
+  vp.start_row = start_row;
+  vp.session = session;
+  vp.v = static_cast<uint16_t*>(const_cast<void*>(kv->v));
+  vp.v_ss = kv->stride_session;
+  vp.v_sh = kv->stride_head;
+  vp.v_st = kv->stride_token;
+  vp.v_sp = kv->stride_page;
+  vp.page_table = kv->page_table;
+  vp.pt_stride = kv->page_table_stride;
+  vp.page_size = kv->page_size;
+  vp.num_pages = kv->num_pages;
+  vp.u = static_cast<uint16_t*>(u_dst->u);
+  vp.u_ss = u_dst->stride_session;
+  vp.u_sa = u_dst->stride_agent;
+  vp.u_st = u_dst->stride_token;
+  vp.flags = static_cast<unsigned*>(workspace);
+  s = lrkv::launch_vproj(vp, &maps[0], &maps[1], stream);
+  if (s != LRKV_OK) return fail(s, "value projection launch failed: %s", cudaGetErrorString(cudaGetLastError()));
+  return LRKV_OK;
+}
+
 lrkv_status lrkv_workspace_reset(void* workspace, size_t workspace_bytes, lrkv_stream_t stream) {
   if (!workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "workspace is NULL");
   cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));

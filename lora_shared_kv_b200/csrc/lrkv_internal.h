@@ -89,6 +89,20 @@ __host__ __device__ inline long long owner_cta(long long t, long long W, long lo
   return ((t + 1) * C - 1) / W;
 }
 
+// Value projection [V_base | U_1 .. U_n] = X [W0_v | A_1 .. A_n] into the caches.
+struct VprojParams {
+  int T, Dm, Hkv, d, n_u, r, ncols;  // ncols = Hkv d + n_u r
+  int start_row, session;
+  uint16_t* v;                       // base value cache (bf16)
+  long long v_ss, v_sh, v_st, v_sp;  // strides (elements): session, head, token, page
+  const int32_t* page_table;         // null => dense
+  long long pt_stride;
+  int page_size, num_pages;
+  uint16_t* u;                       // low-rank caches (bf16)
+  long long u_ss, u_sa, u_st;
+  unsigned* flags;                   // device status word
+};
+
 // ---------------------------------------------------------------------------
 // launchers (defined in the kernel translation units)
 // ---------------------------------------------------------------------------
@@ -97,6 +111,8 @@ struct TmaMaps;  // opaque; holds CUtensorMap objects
 lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, const void* tmK, const void* tmV,
                           const void* tmU, int smem_bytes, int ctas, void* stream);
 int decode_max_smem_optin();
+int vproj_smem_bytes();
+lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, void* stream);
 
 lrkv_status launch_append(const void* x, const void* a, int n_a, const int* row_begin, const int* row_end,
                           int u_shift, int Dm, int r, void* u, long long u_ss, long long u_sa, long long u_st,

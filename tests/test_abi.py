@@ -109,6 +109,24 @@ def test_append_ranges_argument_errors():
     assert L.lrkv_append_lr_cache_ranges(None, 1, None, 1, 1, 16, None, None, None, 0, None) == 1
 
 
+def test_value_projection_argument_errors():
+    L = lrkv.lib()
+    kv, uv = _views()
+    prob = _problem()
+
+    def f(T=16, Dm=64, start=0, kv_rows=8192, x=FAKE, ws=FAKE):
+        return L.lrkv_value_projection(ctypes.byref(prob), ctypes.c_void_p(x), T, Dm, ctypes.c_void_p(FAKE),
+                                       ctypes.byref(kv), kv_rows, ctypes.byref(uv), 0, start, ctypes.c_void_p(ws),
+                                       1 << 20, None)
+    assert f(Dm=60) == 3                 # rows of x not 16-byte multiples
+    assert f(x=FAKE + 2) == 3            # misaligned x
+    assert f(T=-1) == 1
+    assert f(start=8190) == 1            # rows past the U capacity
+    assert f(kv_rows=10) == 1            # rows past the value cache
+    assert f(T=0) == 0                   # nothing to project: a no-op
+    assert L.lrkv_value_projection(ctypes.byref(prob), None, 1, 64, None, None, 0, None, 0, 0, None, 0, None) == 1
+
+
 def test_workspace_bytes_shape_rules():
     # without a device the plan falls back to 148 SMs; invalid shapes give 0
     assert lrkv.lib().lrkv_decode_workspace_bytes(ctypes.byref(_problem(d=96)), 128) == 0
