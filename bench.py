@@ -446,6 +446,42 @@ def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3):
     return out
 
 
+def value_projection_timing(cfg, inp, prob, device, steps=20, warmup=5):
+    """The chunk's value projection [V_base | U_1..U_n] = X [W0_v | A_1..A_n]
+    into the caches (the step before the attention): median time and TFLOP/s.
+    The weights are synthetic draws of the model's shapes."""
+    import lora_shared_kv_b200 as lrkv
+    g = torch.Generator(device=device)
+    g.manual_seed(4242)
+    ncols = cfg.Hkv * cfg.d + cfg.n_u * cfg.r
+    w = (torch.randn((cfg.Dm, ncols), generator=g, device=device) * cfg.Dm ** -0.5).to(torch.bfloat16)
+    v = torch.empty_like(inp.v)
+    kv = lrkv.kv_view_dense(inp.k, v)
+    u = torch.empty_like(inp.u)
+    ws = torch.zeros(256, dtype=torch.uint8, device=device)
+    rows = inp.v.shape[2]
+
+    def step():
+        lrkv.lrkv_value_projection(prob, inp.x, w, kv, rows, u, 0, cfg.L0, ws)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    times = []
+    for i in range(warmup + steps):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        e1.synchronize()
+        if i >= warmup:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    flops = 2.0 * cfg.T * cfg.Dm * ncols
+    return {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12, "flops": flops,
+            "shape": f"X [{cfg.T}, {cfg.Dm}] x W [{cfg.Dm}, {ncols}]"}
+
+
 def bench_prefill(device, steps=20, warmup=5):
     """Prefill chunk workload: append the chunk's U rows, then the causal chunk
     attention for 4 agents (one layer).  Returns a dict, or None if unavailable."""
@@ -480,6 +516,7 @@ def bench_prefill(device, steps=20, warmup=5):
         if i >= warmup:
             times.append(e0.elapsed_time(e1))
     ms = statistics.median(times)
+    vproj = value_projection_timing(cfg, inp, prob, device)
     keys = cfg.T * cfg.L0 + cfg.T * (cfg.T + 1) // 2
     rows = cfg.N * cfg.Hq
     flops = 2.0 * rows * keys * cfg.d * 2 + 2.0 * rows * keys * cfg.r + 2.0 * rows * cfg.T * cfg.r * cfg.d
@@ -489,6 +526,7 @@ def bench_prefill(device, steps=20, warmup=5):
     return {"workload": cfg.name, "ms_per_step": ms, "tflops": tf, "flops_per_step": flops,
             "peak_tflops": bf16_peak, "frac": tf / bf16_peak, "peak_source": src,
             "prefill_kernel_traffic": profiled_traffic("prefill_kernel", cfg.name),
+            "value_projection": vproj,
             "l2": "256 MB flush before each step"}
 
 
