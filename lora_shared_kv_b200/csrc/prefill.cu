@@ -56,7 +56,8 @@ constexpr int BN = 128;   // keys per block
 constexpr int KST = 3;    // K ring: a stage is free once S = Q K^T has been computed
 constexpr int VST = 2;    // V/U ring: a stage is free once the PV MMA is done
 constexpr int THREADS = 384;      // K producer, MMA, V/U producer, idle, 2 softmax warpgroups
-constexpr int SMX_THREADS = 256;  // the two softmax warpgroups (named barrier 1)
+constexpr int SMX_THREADS = 256;  // the two softmax warpgroups (named barrier 1); the two warps of
+                                  // one 32-row lane quarter pair up on named barriers 2..5
 constexpr uint32_t TMEM_COLS = 512;
 
 template <int D, int RK>
@@ -502,7 +503,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         float* xm = xmax + (n & 1) * 2 * BM;
         xm[wg * BM + row] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        named_bar_sync(1, SMX_THREADS);  // also: both halves have read their S columns
+        named_bar_sync(2 + (warp & 3), 64);  // the two warps of these 32 rows; both have read their S columns
         float mx = fmaxf(xm[row], xm[BM + row]);
         mx *= p.scale_log2;  // the scale is positive: the max commutes with it
         const bool need = mx > m_ref + 8.f;
