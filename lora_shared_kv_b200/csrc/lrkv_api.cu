@@ -309,7 +309,7 @@ lrkv_status lrkv_value_projection(const lrkv_problem* p, const void* x, int32_t 
   vp.u_sa = u_dst->stride_agent;
   vp.u_st = u_dst->stride_token;
   vp.flags = static_cast<unsigned*>(workspace);
-  s = lrkv::launch_vproj(vp, &maps[0], &maps[1], stream);
+  s = lrkv::launch_vproj(vp, &maps[0], &maps[1], dev.sms, stream);
   if (s != LRKV_OK) return fail(s, "value projection launch failed: %s", cudaGetErrorString(cudaGetLastError()));
   return LRKV_OK;
 }

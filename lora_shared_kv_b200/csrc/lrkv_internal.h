@@ -112,7 +112,7 @@ lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, const vo
                           const void* tmU, int smem_bytes, int ctas, void* stream);
 int decode_max_smem_optin();
 int vproj_smem_bytes();
-lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, void* stream);
+lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, int sms, void* stream);
 
 lrkv_status launch_append(const void* x, const void* a, int n_a, const int* row_begin, const int* row_end,
                           int u_shift, int Dm, int r, void* u, long long u_ss, long long u_sa, long long u_st,

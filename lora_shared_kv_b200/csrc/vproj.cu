@@ -6,9 +6,10 @@
 // projection as X W0 + (X A_i) B_i; both parts read the same hidden states, so
 // one GEMM produces the shared base values and every U_i row at once.
 //
-// A tcgen05 GEMM: one CTA per 128-token x 128-column tile, K in 64-wide steps
-// through a 4-stage TMA ring (X K-major, W column-major atoms, both 128B
-// swizzled), fp32 accumulation in TMEM, and an epilogue that converts to bf16
+// A tcgen05 GEMM: one CTA per 128-token x BN-column tile (BN = 128, or 64 when
+// 128-wide tiles would leave SMs idle), K in 64-wide steps through a TMA ring
+// of 6 or 8 stages (X K-major, W column-major atoms, both 128B swizzled), fp32
+// accumulation in TMEM, and an epilogue that converts to bf16
 // and scatters each row's columns to its cache: column c < Hkv d goes to KV
 // head c / d of the base value cache, the rest to agent slot (c - Hkv d) / r.
 // The summation order inside the tensor core is not specified, so U rows made
@@ -21,26 +22,35 @@ namespace lrkv {
 namespace {
 
 constexpr int VP_BM = 128;     // tokens per tile (TMEM lanes)
-constexpr int VP_BN = 128;     // output columns per tile
 constexpr int VP_BK = 64;      // K per stage
-constexpr int VP_ST = 4;       // ring stages
 constexpr int VP_THREADS = 256;
 constexpr int VP_X_BYTES = VP_BM * VP_BK * 2;   // 16 KB
-constexpr int VP_W_BYTES = VP_BK * VP_BN * 2;   // 16 KB: two 64-column atoms of 64 k-rows
-constexpr int VP_STAGE = VP_X_BYTES + VP_W_BYTES;
-constexpr int VP_SMEM = VP_ST * VP_STAGE + 256;
+constexpr int VP_RING = 192 * 1024;             // shared memory for the ring
+
+template <int BN>
+struct VpShape {
+  static constexpr int W_BYTES = VP_BK * BN * 2;  // BN / 64 atoms of 64 k-rows x 64 columns
+  static constexpr int STAGE = VP_X_BYTES + W_BYTES;
+  static constexpr int ST = VP_RING / STAGE;      // 6 (BN = 128) or 8 (BN = 64) stages
+  static constexpr int SMEM = ST * STAGE + 256;
+};
 
 struct VpBars {
-  uint64_t full[VP_ST];
-  uint64_t empty[VP_ST];
+  uint64_t full[8];
+  uint64_t empty[8];
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
 };
 
+template <int BN>
 __global__ void __launch_bounds__(VP_THREADS, 1)
     vproj_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const VprojParams p) {
+  constexpr int VP_ST = VpShape<BN>::ST;
+  constexpr int VP_STAGE = VpShape<BN>::STAGE;
+  constexpr int VP_BN = BN;
+  static_assert(VP_ST <= 8, "barrier slots");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   VpBars* bars = reinterpret_cast<VpBars*>(smem + VP_ST * VP_STAGE);
@@ -87,8 +97,9 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
         uint8_t* ws = xs + VP_X_BYTES;
         mbar_arrive_expect_tx(&bars->full[st], VP_STAGE);
         tma_load_4d(xs, &tmX, &bars->full[st], kt * VP_BK, m0, 0, 0, pol);
-        tma_load_4d(ws, &tmW, &bars->full[st], n0, kt * VP_BK, 0, 0, pol);
-        tma_load_4d(ws + VP_W_BYTES / 2, &tmW, &bars->full[st], n0 + 64, kt * VP_BK, 0, 0, pol);
+#pragma unroll
+        for (int at = 0; at < BN / 64; ++at)
+          tma_load_4d(ws + at * (VP_BK * 128), &tmW, &bars->full[st], n0 + at * 64, kt * VP_BK, 0, 0, pol);
       }
       if (*abort_flag) {
         for (int kt = issued > VP_ST ? issued - VP_ST : 0; kt < issued; ++kt) {
@@ -113,7 +124,7 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
 #pragma unroll
         for (int ks = 0; ks < VP_BK / 16; ++ks) {
           const uint64_t a = umma_desc(xs + ks * 32, 16, 1024, 2);                 // K-major, 128B swizzle
-          const uint64_t b = umma_desc(ws + ks * 2048, VP_W_BYTES / 2, 1024, 2);   // column-major atoms
+          const uint64_t b = umma_desc(ws + ks * 2048, VP_BK * 128, 1024, 2);     // column-major atoms
           umma_ss(tmem, a, b, ID, (kt > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&bars->empty[st]);
@@ -183,18 +194,23 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
 
 }  // namespace
 
-int vproj_smem_bytes() { return VP_SMEM + 1024; }
+int vproj_smem_bytes() { return VpShape<128>::SMEM + 1024; }
 
-lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, void* stream) {
-  const int smem = VP_SMEM + 1024;
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(vproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, int sms, void* stream) {
+  // 128-wide tiles, unless they would leave more than half of the SMs idle
+  const long long tiles128 = (long long)((p.T + VP_BM - 1) / VP_BM) * ((p.ncols + 127) / 128);
+  const bool narrow = tiles128 * 2 <= sms;
+  const int bn = narrow ? 64 : 128;
+  const int smem = (narrow ? VpShape<64>::SMEM : VpShape<128>::SMEM) + 1024;
+  auto kern = narrow ? vproj_kernel<64> : vproj_kernel<128>;
+  static bool configured[2] = {false, false};
+  if (!configured[narrow]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return LRKV_ERR_CUDA;
-    configured = true;
+    configured[narrow] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.T + VP_BM - 1) / VP_BM, (p.ncols + VP_BN - 1) / VP_BN);
+  cfg.gridDim = dim3((p.T + VP_BM - 1) / VP_BM, (p.ncols + bn - 1) / bn);
   cfg.blockDim = dim3(VP_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
@@ -203,8 +219,8 @@ lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, vproj_kernel, *static_cast<const CUtensorMap*>(tmX),
-                         *static_cast<const CUtensorMap*>(tmW), p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, *static_cast<const CUtensorMap*>(tmX), *static_cast<const CUtensorMap*>(tmW),
+                         p) != cudaSuccess)
     return LRKV_ERR_CUDA;
   return LRKV_OK;
 }

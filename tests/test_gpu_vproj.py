@@ -5,7 +5,8 @@ Each output element is a bf16 rounding of an fp32 tensor-core sum, so it must
 sit within one bf16 half-ulp (2^-9 relative) of the exact value, plus a small
 allowance for the fp32 accumulation.  Rows outside [start_row, start_row + T),
 other sessions and the K cache stay untouched.  Token counts and Dm that are
-not tile multiples, both sharing modes, and a paged value cache are covered."""
+not tile multiples, both sharing modes, a paged value cache and both tile
+widths (64 columns for few tiles, 128 for many) are covered."""
 
 import numpy as np
 import pytest
@@ -32,6 +33,7 @@ def _close_bf16(got, ref):
     (2, 2, 8, 128, 16, 1, 64, 200, 17, False),     # BaseLRShared: one U; Dm not a multiple of 64
     (1, 2, 2, 64, 8, 0, 300, 136, 64, False),
     (3, 3, 2, 128, 16, 0, 150, 512, 100, True),    # paged value cache
+    (1, 4, 8, 128, 32, 0, 2100, 256, 3, False),    # enough tiles for the 128-column tile shape
 ])
 def test_value_projection_matches_oracle(S, N, Hkv, d, r, mode, T, Dm, start, paged):
     g = torch.Generator(device=DEV)
