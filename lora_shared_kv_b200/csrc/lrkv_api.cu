@@ -570,7 +570,7 @@ size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int3
   if (device_info(&dev) != LRKV_OK) dev.sms = 148;
   const int G = p->num_q_heads / p->num_kv_heads;
   if (G < 1 || 128 % G != 0) return lrkv::kWsHeaderBytes;
-  return lrkv::plan_prefill(T, ctx_len, G, p->num_kv_heads, p->num_agents, p->head_dim, p->rank, dev.sms).bytes;
+  return lrkv::plan_prefill(T, ctx_len, G, p->num_kv_heads, p->num_agents, p->head_dim, dev.sms).bytes;
 }
 
 lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv, int32_t session,
@@ -650,7 +650,7 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
   pp.mode = p->mode;
   pp.scale_log2 = scale_of(p) * 1.4426950408889634f;
   pp.flags = static_cast<unsigned*>(workspace);
-  const lrkv::PrefillPlan pl = lrkv::plan_prefill(T, ctx_len, G, p->num_kv_heads, p->num_agents, D, RK, dev.sms);
+  const lrkv::PrefillPlan pl = lrkv::plan_prefill(T, ctx_len, G, p->num_kv_heads, p->num_agents, D, dev.sms);
   if (workspace_bytes < pl.bytes)
     return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes (lrkv_prefill_workspace_bytes)", workspace_bytes, pl.bytes);
   pp.n_tb = pl.n_tb;

@@ -6,8 +6,8 @@
 //     o = ( P V_base,g + (P Umask_i) B_i,g ) / l,   P = exp(q K_base,g^T * scale - m),  keys t <= L0 + j
 // Eq. 12 of "LRAgent: Efficient KV Cache Sharing for Multi-LoRA LLM Agents"
 // (Pith review, "What carries the argument"): the rank-r values are
-// accumulated next to O as Z = P Umask_i and B_i is applied once per row in
-// the epilogue.  Umask_i drops U rows before the agent's aLoRA offset ("RoleKV",
+// accumulated next to O as Z = P Umask_i and B_i is applied once per row, at
+// the end.  Umask_i drops U rows before the agent's aLoRA offset ("RoleKV",
 // "What it does").
 //
 // A 128-row tile is one agent, one KV head, 128/G chunk tokens x the G query
@@ -15,7 +15,7 @@
 // The (tile, 128-key block) pairs are split evenly over one persistent CTA per
 // SM (stream-K): a CTA walks a contiguous range of them, tile after tile, and
 // a tile cut by a range boundary is finished by the last of its CTAs to get
-// there (atomic ticket), which merges the others' partial (m, l, O, Z) rows.
+// there (atomic ticket), which merges the others' partial (m, l, O + Z B) rows.
 // Roles:
 //   warp 0        TMA producer: B_i,g of each tile segment (double buffer),
 //                 then its 128-key blocks of K into a 3-stage ring (a stage
@@ -33,11 +33,12 @@
 //                 adds Z B_i,g to O with one more MMA pair (Z converted to bf16
 //                 in TMEM, B_i,g in shared memory), so the epilogue only divides
 //                 by l.
-//   warps 4..11   Q into TMEM (the next segment's as soon as the last S of the
-//                 current one has been read), softmax and epilogue, in two warpgroups, one
-//                 per half of the block's 128 keys; a thread owns one row (TMEM
-//                 lane) of its half.  The halves agree on each row's reference
-//                 max through shared memory.  The reference max moves only when
+//   warps 4..11   Q into TMEM (the next segment's as soon as the last S of
+//                 the current one has been read), softmax and epilogue, in two
+//                 warpgroups, one per half of the block's 128 keys; a thread
+//                 owns one row (TMEM lane) of its half.  The two warps of a
+//                 lane quarter agree on each row's reference max through
+//                 shared memory.  The reference max moves only when
 //                 a block exceeds it by 2^8, and only then are O, Z and l
 //                 rescaled in TMEM (each half rescales its share of the
 //                 columns).  The epilogue splits the output columns.
@@ -736,7 +737,7 @@ lrkv_status launch_t(const PrefillParams& p, const PrefillMaps& m, int grid, cud
 
 }  // namespace
 
-PrefillPlan plan_prefill(int T, int L0, int G, int Hkv, int N, int D, int RK, int sms) {
+PrefillPlan plan_prefill(int T, int L0, int G, int Hkv, int N, int D, int sms) {
   PrefillPlan pl = {};
   const int TM = BM / G;
   pl.n_tb = (T + TM - 1) / TM;
@@ -758,7 +759,6 @@ PrefillPlan plan_prefill(int T, int L0, int G, int Hkv, int N, int D, int RK, in
   pl.tickets_off = kWsHeaderBytes;
   pl.partials_off = (pl.tickets_off + (size_t)pl.tiles * 4 + 255) / 256 * 256;
   pl.bytes = pl.partials_off + (size_t)pl.tiles * pl.max_parts * BM * (D + 2) * 4;
-  (void)RK;
   return pl;
 }
 

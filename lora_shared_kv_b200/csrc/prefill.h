@@ -34,7 +34,7 @@ struct PrefillPlan {
   long long W_ga, W;
   size_t tickets_off, partials_off, bytes;
 };
-PrefillPlan plan_prefill(int T, int L0, int G, int Hkv, int N, int D, int RK, int sms);
+PrefillPlan plan_prefill(int T, int L0, int G, int Hkv, int N, int D, int sms);
 
 // Four CUtensorMap objects, in order: K, V, U, B.
 struct PrefillMaps {

@@ -134,6 +134,33 @@ def test_workspace_bytes_shape_rules():
     assert n >= 256
 
 
+def _prefill_ws_expected(T, L0, G, Hkv, N, d, sms=148):
+    # the stream-K plan, derived here independently: 128-row tiles of 128/G
+    # tokens, each needing the 128-key blocks its last row sees; the blocks of
+    # all tiles split evenly over min(blocks, SMs) CTAs; a tile spans at most
+    # ceil(blocks / fewest-per-CTA) + 1 CTAs, each keeping 128 rows of (m, l, O)
+    tm = 128 // G
+    n_tb = -(-T // tm)
+    nbs = [-(-(L0 + tb * tm + min(tm, T - tb * tm)) // 128) for tb in range(n_tb)]
+    W = sum(nbs) * Hkv * N
+    C = min(W, sms)
+    parts = -(-max(nbs) // (W // C)) + 1
+    tiles = Hkv * N * n_tb
+    partials_off = -(-(256 + 4 * tiles) // 256) * 256
+    return partials_off + tiles * parts * 128 * (d + 2) * 4
+
+
+@pytest.mark.parametrize("T,L0,Hq,Hkv,N,d,r", [
+    (512, 16384, 16, 8, 4, 128, 32),   # the prefill workload: 2 parts per tile at most
+    (100, 300, 4, 2, 2, 128, 32),      # fewer blocks than SMs: one block per CTA
+    (1, 77, 8, 4, 2, 64, 16),
+])
+def test_prefill_workspace_follows_the_stream_k_plan(T, L0, Hq, Hkv, N, d, r):
+    prob = lrkv.make_problem(1, N, Hq, Hkv, d, r, lrkv.BASE_SHARED)
+    got = lrkv.lib().lrkv_prefill_workspace_bytes(ctypes.byref(prob), L0, T)
+    assert got == _prefill_ws_expected(T, L0, Hq // Hkv, Hkv, N, d)
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(lrkv, "_lib", None)
     monkeypatch.setattr(lrkv, "LIB_PATH", str(tmp_path / "liblrkv.so"))
