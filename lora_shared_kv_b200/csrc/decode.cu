@@ -20,13 +20,19 @@
 //  * A producer warp moves 64-key K/V tiles (128B-swizzled) and the rank-r U
 //    tiles with the Tensor Memory Accelerator into a ring of stages guarded by
 //    mbarriers.  U tiles wholly before an agent's offset are never loaded.
-//  * Four consumer warps each own 16 keys of every tile and run the
+//  * Consumer warps come in owner groups (three when an item has at most 16
+//    rows, two for 24) that take a CTA's tiles round-robin; a warp owns 8
+//    query rows over all 64 keys of its group's tiles and runs the
 //    contractions on the tensor cores with keys as the M dimension
 //    (S^T = K Q^T, O^T += V^T P^T, Z^T += U_i^T P^T), so a handful of query
-//    rows pads only to a multiple of 8.  The score accumulators are
-//    re-laid into the P^T operand with movmatrix; the online-softmax row
-//    reductions are warp shuffles.  Rows past seq_len and U rows before a_i
-//    are removed by selects on the operands, never by multiplying with 0.
+//    rows pads only to a multiple of 8.  The score accumulators are re-laid
+//    into the P^T operand with movmatrix; the row max takes warp shuffles.
+//    Rows past seq_len and U rows before a_i are removed by selects on the
+//    operands, never by multiplying with 0.  The groups merge their rows at
+//    the end of a CTA's segment of an item.
+//  * An epilogue warp publishes (or, as the item's last CTA, combines and
+//    finishes) every segment but the CTA's last while the consumers stream
+//    on; the consumers finish the last one themselves.
 #include <float.h>
 #include <math.h>
 
