@@ -66,17 +66,18 @@ KERNEL_SOURCES = {
 
 
 def kernel_sources_sha256(kernel):
-    """sha256 of the kernel's sources with their comments removed (a change of
-    comments alone does not change what the kernel reads and writes)."""
+    """sha256 of the kernel's sources with their comments removed and whitespace
+    folded (a change of comments or layout alone does not change what the
+    kernel reads and writes)."""
     import hashlib
     import re
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "lora_shared_kv_b200", "csrc", name)) as f:
             src = f.read()
-        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-        src = re.sub(r"//[^\n]*", "", src)
-        h.update(src.encode())
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())  # and with whitespace runs folded
     return h.hexdigest()
 
 
