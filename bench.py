@@ -39,6 +39,8 @@ import torch  # noqa: E402
 from workloads import CONFIGS, make_decode_inputs, make_prefill_inputs  # noqa: E402
 
 METRIC = "LoRA-split KV attention: decode queries/s, HBM GB/s vs ~8 TB/s peak"
+NOMINAL_HBM_GBS = 8000.0        # B200 HBM3e, nominal
+NOMINAL_BF16_TFLOPS = 2250.0    # B200 dense bf16, nominal
 UNIT = "queries/s"
 BF16 = 2
 
@@ -532,6 +534,7 @@ def bench_prefill(device, steps=20, warmup=5):
     tf = flops / (ms * 1e-3) / 1e12
     return {"workload": cfg.name, "ms_per_step": ms, "tflops": tf, "flops_per_step": flops,
             "peak_tflops": bf16_peak, "frac": tf / bf16_peak, "peak_source": src,
+            "nominal_peak_tflops": NOMINAL_BF16_TFLOPS, "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS,
             "prefill_kernel_traffic": profiled_traffic("prefill_kernel", cfg.name),
             "value_projection": vproj,
             "l2": "256 MB flush before each step"}
@@ -606,6 +609,7 @@ def main():
     achieved = lb / (per_launch_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
             "traffic": profiled_traffic("decode_kernel", cfg.name), "peak_source": f"{peak_src} copy bandwidth",
+            "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
             "kernel": "decode_kernel", "algorithmic_bytes_per_launch": lb,
             "launch_ms": per_launch_ms, "launch_ms_note": "step time / launches per step (gaps included)"}
 
