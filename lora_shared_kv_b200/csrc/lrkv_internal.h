@@ -18,7 +18,7 @@ constexpr int kWsHeaderBytes = 256;     // flags word + padding at the start of 
 constexpr int kKeysPerTile = 64;        // keys per K/V tile (one TMA box, one page)
 constexpr int kMaxRowsPerItem = 32;     // query rows (agents x GQA heads) per decode work item
 constexpr int kMaxAgents = 16;
-constexpr int kTileRun = 4;             // decode tiles visited contiguously (see tile_of in decode.cu)
+constexpr int kTileRun = 4;             // decode tiles visited contiguously (see TileOrder in decode.cu)
 
 // ---------------------------------------------------------------------------
 // decode
