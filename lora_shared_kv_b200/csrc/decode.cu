@@ -388,6 +388,24 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
   constexpr int E4 = RP * (D + RK) / 4;
   constexpr int PERC = 6;  // float4 elements per thread per combine pass
   const float NEG_INF = -INFINITY;
+  const int HD = p.Hkv * D;
+  const int n_pairs = si.n_ag * D;
+  // The B columns of this thread's first (agent, dim) pairs are requested
+  // before the record is published, so that their latency overlaps the
+  // publish, the ticket and the combine rather than following them.
+  float bb[PB][RK];
+  auto load_b = [&](int e0) {
+#pragma unroll
+    for (int k = 0; k < PB; ++k) {
+      const int e = e0 + k * NTH;
+      if (e >= n_pairs) continue;
+      const uint16_t* bp =
+          static_cast<const uint16_t*>(p.b) + ((size_t)(si.i_lo + e / D) * RK) * HD + (size_t)si.g * D + e % D;
+#pragma unroll
+      for (int r = 0; r < RK; ++r) bb[k][r] = bf16_to_f32(__ldg(bp + (size_t)r * HD));
+    }
+  };
+  load_b(tid);
   bool finish = true;
   if (si.segs > 1) {
     float* grec = p.partials + ((size_t)si.item * p.max_segs + (size_t)si.slot) * REC;
@@ -406,8 +424,31 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
     if (!finish) return;
     __threadfence();
     const float* base = p.partials + (size_t)si.item * p.max_segs * REC;
-    // maxima and sums of every record (chunks of SEG_CHUNK records); rows <= 32 <= NTH
-    if (tid < RP) {
+    // With at most SEG_CHUNK records, one round of loads gives every record's
+    // maximum and sum, hence the scales and l, before the O and Z pass; more
+    // records take a pass for the maxima and then a scale table per chunk.
+    const bool one_chunk = si.segs <= SEG_CHUNK;
+    if (one_chunk) {
+      if (tid < RP) {
+        float mj[SEG_CHUNK], lj[SEG_CHUNK];
+#pragma unroll
+        for (int jj = 0; jj < SEG_CHUNK; ++jj) {
+          mj[jj] = jj < si.segs ? __ldcg(base + (size_t)jj * REC + tid) : NEG_INF;
+          lj[jj] = jj < si.segs ? __ldcg(base + (size_t)jj * REC + RP + tid) : 0.f;
+        }
+        float M = NEG_INF;
+#pragma unroll
+        for (int jj = 0; jj < SEG_CHUNK; ++jj) M = fmaxf(M, mj[jj]);
+        float L = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < SEG_CHUNK; ++jj) {
+          const float sc = mj[jj] == NEG_INF ? 0.f : fast_exp2(mj[jj] - M);
+          scw[jj * RP + tid] = sc;
+          L += lj[jj] * sc;
+        }
+        rec[RP + tid] = L;
+      }
+    } else if (tid < RP) {  // maxima of every record, chunk by chunk; rows <= 32 <= NTH
       float M = NEG_INF;
       for (int j0 = 0; j0 < si.segs; j0 += SEG_CHUNK) {
         float mj[SEG_CHUNK];
@@ -428,18 +469,20 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
       float L = 0.f;
       for (int j0 = 0; j0 < si.segs; j0 += SEG_CHUNK) {
         const int nj = min(SEG_CHUNK, si.segs - j0);
-        if (tid < RP) {
-          const float M = rec[tid];
+        if (!one_chunk) {
+          if (tid < RP) {
+            const float M = rec[tid];
 #pragma unroll
-          for (int jj = 0; jj < SEG_CHUNK; ++jj) {
-            const float mj = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + tid) : NEG_INF;
-            const float lj = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + RP + tid) : 0.f;
-            const float sc = mj == NEG_INF ? 0.f : fast_exp2(mj - M);
-            scw[jj * RP + tid] = sc;
-            L += lj * sc;
+            for (int jj = 0; jj < SEG_CHUNK; ++jj) {
+              const float mj = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + tid) : NEG_INF;
+              const float lj = jj < nj ? __ldcg(base + (size_t)(j0 + jj) * REC + RP + tid) : 0.f;
+              const float sc = mj == NEG_INF ? 0.f : fast_exp2(mj - M);
+              scw[jj * RP + tid] = sc;
+              L += lj * sc;
+            }
           }
+          sync();
         }
-        sync();
         for (int jj = 0; jj < nj; ++jj) {
           const float4* rj = reinterpret_cast<const float4*>(base + (size_t)(j0 + jj) * REC + 2 * RP);
           float4 v[PERC];
@@ -461,34 +504,23 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
             acc[u].w += v[u].w * sc;
           }
         }
-        sync();
+        if (!one_chunk) sync();  // the next chunk rewrites the scale table
       }
 #pragma unroll
       for (int u = 0; u < PERC; ++u) {
         const int e4 = e0 + tid + u * NTH;
         if (e4 < E4) *reinterpret_cast<float4*>(rec + 2 * RP + e4 * 4) = acc[u];
       }
-      if (e0 == 0 && tid < RP) rec[RP + tid] = L;
+      if (!one_chunk && e0 == 0 && tid < RP) rec[RP + tid] = L;
     }
     sync();
   }
   // out = (O + Z B_i,g) / l; one thread per (agent, dim), the agent's B column serves its GQA rows
-  const int HD = p.Hkv * D;
-  const int n_pairs = si.n_ag * D;
   const float* mL = rec + RP;
   const float* mO = rec + 2 * RP;
   const float* mZ = mO + RP * D;
   for (int e0 = tid; e0 < n_pairs; e0 += PB * NTH) {
-    float bb[PB][RK];
-#pragma unroll
-    for (int k = 0; k < PB; ++k) {
-      const int e = e0 + k * NTH;
-      if (e >= n_pairs) continue;
-      const uint16_t* bp =
-          static_cast<const uint16_t*>(p.b) + ((size_t)(si.i_lo + e / D) * RK) * HD + (size_t)si.g * D + e % D;
-#pragma unroll
-      for (int r = 0; r < RK; ++r) bb[k][r] = bf16_to_f32(__ldg(bp + (size_t)r * HD));
-    }
+    if (e0 != tid) load_b(e0);  // the first pairs' columns were requested at the start
 #pragma unroll
     for (int k = 0; k < PB; ++k) {
       const int e = e0 + k * NTH;
