@@ -134,6 +134,43 @@ def test_workspace_bytes_shape_rules():
     assert n >= 256
 
 
+def _decode_ws_expected(S, N, Hq, Hkv, d, r, L, sms=148):
+    # the decode plan, derived here independently: the N*G rows of a KV head
+    # in as few groups of at most 32 as cover them, each padded to a multiple
+    # of 8; work items (session, KV head, row group) of ceil(L/64) key tiles;
+    # the flattened tiles split evenly over min(tiles, SMs) CTAs, CTA c taking
+    # [c W / C, (c + 1) W / C); one partial record per CTA that touches an
+    # item, when more than one does
+    R = N * (Hq // Hkv)
+    n_rg = -(-R // 32)
+    NT = -(-(-(-R // n_rg)) // 8)
+    nt = max(1, -(-L // 64))
+    items = S * Hkv * n_rg
+    W = items * nt
+    C = min(W, sms)
+    touching = [0] * items
+    for c in range(C):
+        lo, hi = c * W // C, (c + 1) * W // C
+        for it in range(lo // nt, (hi - 1) // nt + 1):
+            touching[it] += 1
+    segs = max(touching)
+    partials_off = 256 + -(-(4 * items) // 256) * 256
+    rec = NT * 8 * (d + r + 2) * 4
+    return partials_off + (items * segs * rec if segs > 1 else 0)
+
+
+@pytest.mark.parametrize("S,N,Hq,Hkv,d,r,L", [
+    (32, 3, 12, 2, 128, 16, 8192),   # the Qwen2.5 decode workload: items cut by CTA boundaries
+    (1, 5, 8, 1, 64, 32, 300),       # 40 rows: two row groups, fewer tiles than SMs
+    (16, 2, 16, 8, 128, 16, 1024),   # 4 rows per KV head
+    (200, 1, 4, 4, 128, 8, 64),      # one tile per item, more items than SMs: no partials
+    (1, 16, 32, 8, 128, 32, 65536),  # 64 rows: two full row groups, many CTAs per item
+])
+def test_decode_workspace_follows_the_stream_k_plan(S, N, Hq, Hkv, d, r, L):
+    prob = lrkv.make_problem(S, N, Hq, Hkv, d, r, lrkv.BASE_SHARED)
+    assert lrkv.lib().lrkv_decode_workspace_bytes(ctypes.byref(prob), L) == _decode_ws_expected(S, N, Hq, Hkv, d, r, L)
+
+
 def _prefill_ws_expected(T, L0, G, Hkv, N, d, sms=148):
     # the stream-K plan, derived here independently: 128-row tiles of 128/G
     # tokens, each needing the 128-key blocks its last row sees; the blocks of
