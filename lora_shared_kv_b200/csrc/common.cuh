@@ -7,9 +7,33 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "lrkv_internal.h"
 
 namespace lrkv {
+
+// The dynamic shared-memory limit is an attribute of a kernel on one device:
+// raise it once per (kernel, device) before the first launch that needs it.
+// Thread-safe; once granted, a launch pays one atomic load.
+template <auto Kernel>
+inline cudaError_t ensure_dynamic_smem(int bytes) {
+  constexpr int kDevices = 64;
+  static std::atomic<int> granted[kDevices];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kDevices)
+    return cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (granted[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  if (granted[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) granted[dev].store(bytes, std::memory_order_release);
+  return e;
+}
 
 // Spin cap of every bounded wait.  A try_wait suspends for a short while per
 // attempt, so this is well over a second of waiting: far beyond any healthy

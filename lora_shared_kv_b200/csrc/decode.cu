@@ -979,12 +979,7 @@ template <int D, int NT, int RK>
 lrkv_status launch_one(const DecodeParams& p, const void* tmK, const void* tmV, const void* tmU, int smem,
                        int ctas, cudaStream_t stream) {
   auto kern = decode_kernel<D, NT, RK>;
-  static int configured_smem = 0;
-  if (configured_smem < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return LRKV_ERR_CUDA;
-    configured_smem = smem;
-  }
+  if (ensure_dynamic_smem<decode_kernel<D, NT, RK>>(smem) != cudaSuccess) return LRKV_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
   cfg.blockDim = dim3(Roles<NT>::THREADS);

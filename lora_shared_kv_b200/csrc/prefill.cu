@@ -714,12 +714,7 @@ lrkv_status launch_t(const PrefillParams& p, const PrefillMaps& m, int grid, cud
   using Lay = PrefillLayout<D, RK>;
   auto kern = prefill_kernel<D, RK>;
   const int smem = Lay::TOTAL + 1024;
-  static int configured = 0;
-  if (configured < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return LRKV_ERR_CUDA;
-    configured = smem;
-  }
+  if (ensure_dynamic_smem<prefill_kernel<D, RK>>(smem) != cudaSuccess) return LRKV_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(THREADS);

@@ -203,12 +203,9 @@ lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW,
   const int bn = narrow ? 64 : 128;
   const int smem = (narrow ? VpShape<64>::SMEM : VpShape<128>::SMEM) + 1024;
   auto kern = narrow ? vproj_kernel<64> : vproj_kernel<128>;
-  static bool configured[2] = {false, false};
-  if (!configured[narrow]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return LRKV_ERR_CUDA;
-    configured[narrow] = true;
-  }
+  if ((narrow ? ensure_dynamic_smem<vproj_kernel<64>>(smem) : ensure_dynamic_smem<vproj_kernel<128>>(smem)) !=
+      cudaSuccess)
+    return LRKV_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((p.T + VP_BM - 1) / VP_BM, (p.ncols + bn - 1) / bn);
   cfg.blockDim = dim3(VP_THREADS);
