@@ -140,6 +140,29 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _require(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _on_device(**tensors):
+    """Every tensor the kernels read or write must live in the current CUDA device's memory: the GPU would
+    dereference a host pointer, or another device's memory, as if it were its own.  None is skipped (an
+    optional argument)."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor, got one on {t.device}")
+        if dev is None:
+            dev = torch.cuda.current_device()
+        if t.get_device() != dev:
+            raise ValueError(f"{name} is on cuda:{t.get_device()} but the current device is cuda:{dev}")
+
+
 # ---------------------------------------------------------------------------
 # views
 # ---------------------------------------------------------------------------
@@ -150,15 +173,19 @@ def make_problem(S, N, Hq, Hkv, d, r, mode=BASE_SHARED, softmax_scale=0.0):
 
 def kv_view_dense(k, v):
     """k, v: bf16 [S, Hkv, L, d] with d contiguous (same strides)."""
-    assert k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16 and k.dim() == 4
-    assert k.stride() == v.stride() and k.stride(3) == 1
+    _require(k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16 and k.dim() == 4, "k, v: bf16 [S, Hkv, L, d]")
+    _require(k.stride() == v.stride() and k.stride(3) == 1, "k, v: same strides, d contiguous")
+    _on_device(k=k, v=v)
     return KVView(k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), k.stride(2), None, 0, 0, 0, 0)
 
 
 def kv_view_paged(k_pages, v_pages, page_table):
     """k_pages, v_pages: bf16 [P, Hkv, page, d]; page_table: int32 [S, n_logical_pages] on the device."""
-    assert k_pages.dtype == torch.bfloat16 and k_pages.dim() == 4 and k_pages.stride() == v_pages.stride()
-    assert page_table.dtype == torch.int32 and page_table.dim() == 2 and page_table.stride(1) == 1
+    _require(k_pages.dtype == torch.bfloat16 and v_pages.dtype == torch.bfloat16 and k_pages.dim() == 4
+             and k_pages.stride() == v_pages.stride(), "k_pages, v_pages: bf16 [P, Hkv, page, d], same strides")
+    _require(page_table.dtype == torch.int32 and page_table.dim() == 2 and page_table.stride(1) == 1,
+             "page_table: int32 [S, n_logical_pages], rows contiguous")
+    _on_device(k_pages=k_pages, v_pages=v_pages, page_table=page_table)
     return KVView(k_pages.data_ptr(), v_pages.data_ptr(), 0, k_pages.stride(1), k_pages.stride(2),
                   page_table.data_ptr(), page_table.stride(0), k_pages.stride(0), k_pages.shape[2],
                   k_pages.shape[0])
@@ -166,7 +193,8 @@ def kv_view_paged(k_pages, v_pages, page_table):
 
 def u_view(u):
     """u: bf16 [S, N_U, rows, r] with r contiguous."""
-    assert u.dtype == torch.bfloat16 and u.dim() == 4 and u.stride(3) == 1
+    _require(u.dtype == torch.bfloat16 and u.dim() == 4 and u.stride(3) == 1, "u: bf16 [S, N_U, rows, r], r contiguous")
+    _on_device(u=u)
     return UView(u.data_ptr(), u.stride(0), u.stride(1), u.stride(2), u.shape[2])
 
 
@@ -178,7 +206,8 @@ def lrkv_append_lr_cache(x, a, u, session, start_row, stream=None, uview=None):
     """U[session, i, start_row + t, :] = x[t] @ a[i] for every slot i of a (bit-exact fixed order)."""
     T, Dm = x.shape
     n_a, Dm2, r = a.shape
-    assert Dm == Dm2 and x.is_contiguous() and a.is_contiguous()
+    _require(Dm == Dm2 and x.is_contiguous() and a.is_contiguous(), "x [T, Dm] and a [n_a, Dm, r], contiguous")
+    _on_device(x=x, a=a)
     uv = uview if uview is not None else u_view(u)
     _check(lib().lrkv_append_lr_cache(_ptr(x), _ptr(a), n_a, T, Dm, r, ctypes.byref(uv), session, start_row,
                                       _stream(stream)))
@@ -189,8 +218,9 @@ def lrkv_append_lr_cache_ranges(x, a, u, session, row_begin, row_end, stream=Non
     the per-agent catch-up append (bit-exact fixed order).  x holds the hidden states by absolute position."""
     x_rows, Dm = x.shape
     n_a, Dm2, r = a.shape
-    assert Dm == Dm2 and x.is_contiguous() and a.is_contiguous()
-    assert len(row_begin) == n_a and len(row_end) == n_a
+    _require(Dm == Dm2 and x.is_contiguous() and a.is_contiguous(), "x [rows, Dm] and a [n_a, Dm, r], contiguous")
+    _require(len(row_begin) == n_a and len(row_end) == n_a, "one row_begin and one row_end per slot of a")
+    _on_device(x=x, a=a)
     uv = uview if uview is not None else u_view(u)
     b = (ctypes.c_int32 * n_a)(*[int(v) for v in row_begin])
     e = (ctypes.c_int32 * n_a)(*[int(v) for v in row_end])
@@ -202,7 +232,8 @@ def lrkv_value_projection(problem, x, w, kv, kv_rows, u, session, start_row, wor
     """[V_base | U_1..U_n] = x @ w for T new tokens, written into kv.v rows and u rows
     [start_row, start_row + T) of `session` (x [T, Dm], w [Dm, Hkv*d + n_u*r])."""
     T, Dm = x.shape
-    assert x.is_contiguous() and w.is_contiguous() and w.shape[0] == Dm
+    _require(x.is_contiguous() and w.is_contiguous() and w.shape[0] == Dm, "x [T, Dm] and w [Dm, cols], contiguous")
+    _on_device(x=x, w=w, workspace=workspace)
     uv = u if isinstance(u, UView) else u_view(u)
     _check(lib().lrkv_value_projection(ctypes.byref(problem), _ptr(x), T, Dm, _ptr(w), ctypes.byref(kv), int(kv_rows),
                                        ctypes.byref(uv), session, start_row, _ptr(workspace),
@@ -218,7 +249,8 @@ def lrkv_decode_workspace_bytes(problem, max_seq_len):
 
 def lrkv_attn_decode(problem, q, kv, seq_lens, max_seq_len, u, b, offsets, out, workspace, stream=None):
     """out[s, i, h] = attention of q[s, i, h] over the shared cache with agent i's low-rank values."""
-    assert q.is_contiguous() and b.is_contiguous() and out.is_contiguous()
+    _require(q.is_contiguous() and b.is_contiguous() and out.is_contiguous(), "q, b and out must be contiguous")
+    _on_device(q=q, seq_lens=seq_lens, b=b, offsets=offsets, out=out, workspace=workspace)
     odt = F32 if out.dtype == torch.float32 else BF16
     uv = u if isinstance(u, UView) else u_view(u)
     _check(lib().lrkv_attn_decode(ctypes.byref(problem), _ptr(q), ctypes.byref(kv), _ptr(seq_lens),
@@ -233,7 +265,8 @@ def lrkv_attn_decode_static_scratch(problem, q, kv, seq_lens, max_seq_len, u, b,
     The library keeps one fixed scratch array per GPU (LRKV_STATIC_SCRATCH_BYTES); shapes that need more
     are rejected with LRKV_ERR_WORKSPACE_TOO_SMALL.  Calls share that array: keep them ordered on one stream.
     """
-    assert q.is_contiguous() and b.is_contiguous() and out.is_contiguous()
+    _require(q.is_contiguous() and b.is_contiguous() and out.is_contiguous(), "q, b and out must be contiguous")
+    _on_device(q=q, seq_lens=seq_lens, b=b, offsets=offsets, out=out)
     odt = F32 if out.dtype == torch.float32 else BF16
     uv = u if isinstance(u, UView) else u_view(u)
     _check(lib().lrkv_attn_decode_static_scratch(ctypes.byref(problem), _ptr(q), ctypes.byref(kv), _ptr(seq_lens),
@@ -247,7 +280,8 @@ def lrkv_prefill_workspace_bytes(problem, ctx_len, T):
 
 def lrkv_attn_prefill_chunk(problem, q, kv, session, ctx_len, T, u, b, offsets, out, workspace, stream=None):
     """Causal chunk: row j of every agent sits at ctx_len + j and sees keys t <= ctx_len + j."""
-    assert q.is_contiguous() and b.is_contiguous() and out.is_contiguous()
+    _require(q.is_contiguous() and b.is_contiguous() and out.is_contiguous(), "q, b and out must be contiguous")
+    _on_device(q=q, b=b, offsets=offsets, out=out, workspace=workspace)
     odt = F32 if out.dtype == torch.float32 else BF16
     uv = u if isinstance(u, UView) else u_view(u)
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -257,12 +291,14 @@ def lrkv_attn_prefill_chunk(problem, q, kv, session, ctx_len, T, u, b, offsets, 
 
 
 def lrkv_workspace_reset(workspace, stream=None):
+    _on_device(workspace=workspace)
     _check(lib().lrkv_workspace_reset(_ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _stream(stream)))
 
 
 def lrkv_query_device_status(workspace, clear=True, stream=None):
     """Synchronise and return (status_name, flags); does not raise on device-side flags."""
+    _on_device(workspace=workspace)
     flags = ctypes.c_uint32(0)
     st = lib().lrkv_query_device_status(_ptr(workspace), 1 if clear else 0, ctypes.byref(flags), _stream(stream))
     if st not in (0, 6, 7):
