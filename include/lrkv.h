@@ -41,9 +41,11 @@
  *    a bounded wait that gave up) never fault: they record a flag in the
  *    workspace and are read back with lrkv_query_device_status.
  *    lrkv_last_error_detail() gives a thread-local text for the last failure.
- *  - Supported: head_dim in {64, 128}; rank in {8, 16, 32}; Hq a multiple of
- *    Hkv; page_size 64; at most 16 agents per call.  Anything else returns
- *    LRKV_ERR_UNSUPPORTED.
+ *    A pointer argument not documented as optional ("or NULL") must not be
+ *    NULL: LRKV_ERR_INVALID_ARGUMENT.
+ *  - Supported: an sm_100 GPU (B200) as the current device; head_dim in
+ *    {64, 128}; rank in {8, 16, 32}; Hq a multiple of Hkv; page_size 64; at
+ *    most 16 agents per call.  Anything else returns LRKV_ERR_UNSUPPORTED.
  */
 #ifndef LRKV_H
 #define LRKV_H
