@@ -25,21 +25,24 @@
  *
  * Conventions of every entry point:
  *  - Ownership: the caller owns every buffer.  The library allocates and frees
- *    nothing, and never copies device memory to the host (the one exception is
- *    lrkv_query_device_status, which exists to do exactly that).
+ *    nothing, and never copies device memory to the host (the exceptions are
+ *    the two status queries, which exist to do exactly that).
  *  - Pointers documented as "device" must be device (or managed) memory of the
  *    current device.  Tensors are bf16 unless stated.  Base addresses of q, K,
  *    V, U, B and out must be 16-byte aligned, and the token/head/session/page
  *    strides of K, V and U must be multiples of 8 elements (16 bytes): the
  *    tiles are moved by the Tensor Memory Accelerator.
  *  - Streams: every launch goes on the caller's stream (a cudaStream_t; 0 is
- *    the legacy default stream).  No call synchronises, except
- *    lrkv_query_device_status.
+ *    the legacy default stream).  No call synchronises, except the status
+ *    queries lrkv_query_device_status and lrkv_query_static_scratch_status.
  *  - Errors: every call returns an lrkv_status and never throws.  Host-side
  *    argument errors return before anything is launched.  Device-side checks
  *    (a seq_len beyond max_seq_len, a negative offset, a page id out of range,
  *    a bounded wait that gave up) never fault: they record a flag in the
- *    workspace and are read back with lrkv_query_device_status.
+ *    workspace and are read back with lrkv_query_device_status (the
+ *    static-scratch decode: lrkv_query_static_scratch_status).  After a
+ *    timeout, reset the workspace (lrkv_workspace_reset) before reusing it:
+ *    the abandoned launch may have left its merge tickets counting.
  *    lrkv_last_error_detail() gives a thread-local text for the last failure.
  *    A pointer argument not documented as optional ("or NULL") must not be
  *    NULL: LRKV_ERR_INVALID_ARGUMENT.
@@ -231,8 +234,10 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
  *    runs the same kernel as lrkv_attn_decode.  All calls share the one array
  *    and it keeps the last call's contents, so calls that can overlap on the GPU
  *    (different streams, or different host threads on one device) race and
- *    give wrong results: order them.  Device-side flags of these calls are not
- *    reported (the scratch is not visible to the caller).
+ *    give wrong results: order them.  The device-side flags of the most recent
+ *    call (a bad seq_len, offset or page id, a bounded wait that gave up) stay
+ *    in the scratch until the next call clears them: read them with
+ *    lrkv_query_static_scratch_status.
  */
 #define LRKV_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
 lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv,
@@ -241,14 +246,23 @@ lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q
                                             const int32_t* alora_offsets, void* out, int32_t out_dtype,
                                             lrkv_stream_t stream);
 
+/*
+ * The device-side flags of the most recent lrkv_attn_decode_static_scratch call
+ * on the current device: synchronise `stream`, read them and, when `clear` is
+ * non-zero, reset them.  Same results as lrkv_query_device_status (LRKV_OK,
+ * LRKV_ERR_DEVICE_FAULT, LRKV_ERR_TIMEOUT; *flags_out gets the raw bits).
+ * Like the scratch itself this has no counterpart on the pages.
+ */
+lrkv_status lrkv_query_static_scratch_status(int32_t clear, uint32_t* flags_out, lrkv_stream_t stream);
+
 /* ---------------------------------------------------------------------- */
 /* Prefill chunk: T new rows per agent, causal, over one session.          */
 /* ---------------------------------------------------------------------- */
 
-/* Bytes of workspace lrkv_attn_prefill_chunk needs; 0 if the shape is invalid.
- * It holds the status header, one ticket per 128-row tile and the partial
- * (m, l, O, Z) rows of tiles whose key blocks are split between CTAs (the
- * blocks of all tiles are divided evenly over one CTA per SM). */
+/* Bytes of workspace lrkv_attn_prefill_chunk needs; 0 if the call would refuse
+ * the shape.  It holds the status header, one ticket per 128-row tile and the
+ * partial (m, l, O, Z) rows of tiles whose key blocks are split between CTAs
+ * (the blocks of all tiles are divided evenly over one CTA per SM). */
 size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T);
 
 /*
@@ -257,6 +271,12 @@ size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int3
  * out[i, j, h, :] = sum_t P[t] (V_base,g[t] + [t >= a_i] U_i[t] B_i,g).
  * The chunk's own base K/V must already be in the cache at rows
  * [ctx_len, ctx_len + T), and its U rows appended (lrkv_append_lr_cache).
+ * A role switch ("RoleKV", "What it does") is such a chunk: the new role's
+ * header rows over the shared context, its adapter active from its offset.
+ * Supported set: the global one (any G = Hq / Hkv up to 128; every rank).
+ * Numerics: bf16 Q K^T and P [V | U] on the tensor cores with fp32
+ * accumulation; the rank-r accumulator Z = P Umask_i enters Z B_i,g as two
+ * bf16 terms (Z = Z_hi + Z_lo), about 2^-17 of |Z| from the fp32 value.
  *   q              device bf16 [N, T, Hq, d] contiguous
  *   kv, u          views as above (u->num_rows >= ctx_len + T)
  *   b              device bf16 [N, r, Hkv*d]
@@ -319,6 +339,21 @@ lrkv_status lrkv_workspace_reset(void* workspace, size_t workspace_bytes, lrkv_s
  */
 lrkv_status lrkv_query_device_status(const void* workspace, int32_t clear, uint32_t* flags_out,
                                      lrkv_stream_t stream);
+
+/*
+ * Failure-detection test hook (no counterpart on the pages: it tests the
+ * library's own error path).  Arms the next lrkv_attn_decode,
+ * lrkv_attn_decode_static_scratch or lrkv_attn_prefill_chunk call made from
+ * this host thread: in that launch the copy-issuing warps issue nothing and
+ * every bounded wait gives up after `spin_cap` failed attempts, so the waits
+ * run out the way they would if a copy never arrived.  The launch records
+ * LRKV_DEVFLAG_TIMEOUT (lrkv_query_device_status then returns
+ * LRKV_ERR_TIMEOUT), leaves its output undefined, and returns with no copy or
+ * tensor-core operation in flight, so the context stays usable; reset the
+ * workspace before reusing it.  spin_cap 0 disarms.  Never faults, traps or
+ * hangs the GPU: every wait stays bounded.
+ */
+lrkv_status lrkv_debug_stall_next_launch(uint32_t spin_cap);
 
 const char* lrkv_status_string(lrkv_status s);
 const char* lrkv_last_error_detail(void);

@@ -19,6 +19,17 @@ namespace {
 
 thread_local char g_detail[512] = "";
 
+// Failure-detection test hook: armed by lrkv_debug_stall_next_launch, consumed
+// by the next decode or prefill launch of this thread.
+thread_local uint32_t g_stall_cap = 0;
+
+// Spin cap and stall flag of a launch (disarms the hook).
+void take_stall_hook(unsigned* spin_cap, int* stall) {
+  *spin_cap = g_stall_cap ? g_stall_cap : lrkv::kSpinCap;
+  *stall = g_stall_cap ? 1 : 0;
+  g_stall_cap = 0;
+}
+
 lrkv_status fail(lrkv_status s, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -237,6 +248,11 @@ const char* lrkv_status_string(lrkv_status s) {
 
 const char* lrkv_last_error_detail(void) { return g_detail; }
 
+lrkv_status lrkv_debug_stall_next_launch(uint32_t spin_cap) {
+  g_stall_cap = spin_cap;
+  return LRKV_OK;
+}
+
 int32_t lrkv_version(void) { return 100; }
 
 lrkv_status lrkv_value_projection(const lrkv_problem* p, const void* x, int32_t T, int32_t Dm, const void* w,
@@ -321,9 +337,13 @@ lrkv_status lrkv_workspace_reset(void* workspace, size_t workspace_bytes, lrkv_s
   return LRKV_OK;
 }
 
-lrkv_status lrkv_query_device_status(const void* workspace, int32_t clear, uint32_t* flags_out,
-                                     lrkv_stream_t stream) {
-  if (!workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "workspace is NULL");
+}  // extern "C"
+
+namespace {
+
+// Read (and optionally clear) the flag word at the start of a workspace on
+// `stream`, then turn its bits into a status.
+lrkv_status read_device_flags(const void* workspace, int32_t clear, uint32_t* flags_out, lrkv_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint32_t flags = 0;
   cudaError_t e = cudaMemcpyAsync(&flags, workspace, sizeof(flags), cudaMemcpyDeviceToHost, st);
@@ -340,6 +360,16 @@ lrkv_status lrkv_query_device_status(const void* workspace, int32_t clear, uint3
                          (flags & LRKV_DEVFLAG_SEQLEN) ? "seq_len " : "", (flags & LRKV_DEVFLAG_OFFSET) ? "offset " : "",
                          (flags & LRKV_DEVFLAG_PAGE) ? "page-id" : "");
   return LRKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lrkv_status lrkv_query_device_status(const void* workspace, int32_t clear, uint32_t* flags_out,
+                                     lrkv_stream_t stream) {
+  if (!workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "workspace is NULL");
+  return read_device_flags(workspace, clear, flags_out, stream);
 }
 
 lrkv_status lrkv_append_lr_cache(const void* x, const void* a, int32_t n_a, int32_t T, int32_t Dm, int32_t r,
@@ -497,6 +527,7 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
   dp.flags = reinterpret_cast<unsigned*>(ws);
   dp.tickets = reinterpret_cast<int*>(ws + pl.tickets_off);
   dp.partials = reinterpret_cast<float*>(ws + pl.partials_off);
+  take_stall_hook(&dp.spin_cap, &dp.stall);
   s = lrkv::launch_decode(dp, D, pl.NT, RK, &tmK, &tmV, &tmU, pl.smem, pl.ctas, stream);
   if (s != LRKV_OK) return fail(s, "decode launch failed: %s", cudaGetErrorString(cudaGetLastError()));
   return LRKV_OK;
@@ -563,13 +594,45 @@ lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q
                           kStaticScratchBytes, stream);
 }
 
+// The flags of the most recent static-scratch call (every call clears them first).
+lrkv_status lrkv_query_static_scratch_status(int32_t clear, uint32_t* flags_out, lrkv_stream_t stream) {
+  void* scratch = nullptr;
+  lrkv_status s = static_scratch_address(&scratch);
+  if (s != LRKV_OK) return s;
+  return read_device_flags(scratch, clear, flags_out, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shape rules of the prefill chunk beyond check_problem: a 128-row tile holds
+// floor(128 / G) tokens x G query heads, so G may be at most 128.
+lrkv_status check_prefill_shape(const lrkv_problem* p, int32_t ctx_len, int32_t T) {
+  lrkv_status s = check_problem(p);
+  if (s != LRKV_OK) return s;
+  if (ctx_len < 0 || T < 0) return fail(LRKV_ERR_INVALID_ARGUMENT, "need ctx_len >= 0 and T >= 0");
+  if ((long long)ctx_len + T > 0x7fffffffLL) return fail(LRKV_ERR_INVALID_ARGUMENT, "ctx_len + T overflows");
+  const int G = p->num_q_heads / p->num_kv_heads;
+  if (G > 128) return fail(LRKV_ERR_UNSUPPORTED, "prefill needs Hq / Hkv <= 128 (got %d)", G);
+  return LRKV_OK;
+}
+
+// Rank of the kernel instance that serves rank r: rank 8 runs in the rank-16
+// instance, whose U and B tiles are 16 wide; the tensor maps of U and B keep
+// their true rank, so the Tensor Memory Accelerator fills ranks 8..15 with zeros.
+int prefill_kernel_rank(int r) { return r == 8 ? 16 : r; }
+
+}  // namespace
+
+extern "C" {
+
 size_t lrkv_prefill_workspace_bytes(const lrkv_problem* p, int32_t ctx_len, int32_t T) {
-  if (check_problem(p) != LRKV_OK || ctx_len < 0 || T < 0) return 0;
+  if (check_prefill_shape(p, ctx_len, T) != LRKV_OK) return 0;
   if (T == 0) return lrkv::kWsHeaderBytes;
   DeviceInfo dev;
   if (device_info(&dev) != LRKV_OK) dev.sms = 148;
   const int G = p->num_q_heads / p->num_kv_heads;
-  if (G < 1 || 128 % G != 0) return lrkv::kWsHeaderBytes;
   return lrkv::plan_prefill(T, ctx_len, G, p->num_kv_heads, p->num_agents, p->head_dim, dev.sms).bytes;
 }
 
@@ -577,26 +640,24 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
                                     int32_t ctx_len, int32_t T, const lrkv_u_view* u, const void* b,
                                     const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
                                     size_t workspace_bytes, lrkv_stream_t stream) {
-  lrkv_status s = check_problem(p);
+  lrkv_status s = check_prefill_shape(p, ctx_len, T);
   if (s != LRKV_OK) return s;
   if (!q || !b || !out || !workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "q, b, out and workspace must not be NULL");
   if (!aligned16(q) || !aligned16(b) || !aligned16(out) || !aligned16(workspace))
     return fail(LRKV_ERR_MISALIGNED, "q, b, out and workspace must be 16-byte aligned");
   if (out_dtype != LRKV_BF16 && out_dtype != LRKV_F32) return fail(LRKV_ERR_INVALID_ARGUMENT, "out_dtype %d", out_dtype);
-  if (ctx_len < 0 || T < 0 || session < 0 || session >= p->num_sessions)
-    return fail(LRKV_ERR_INVALID_ARGUMENT, "need ctx_len >= 0, T >= 0 and 0 <= session < num_sessions");
+  if (session < 0 || session >= p->num_sessions)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "need 0 <= session < num_sessions (got %d of %d)", session, p->num_sessions);
   const int G = p->num_q_heads / p->num_kv_heads;
-  if (128 % G != 0) return fail(LRKV_ERR_UNSUPPORTED, "prefill needs Hq/Hkv to divide 128 (got %d)", G);
-  if (p->rank == 8) return fail(LRKV_ERR_UNSUPPORTED, "prefill supports rank 16 and 32");
   const long long Ltot = (long long)ctx_len + T;
-  if (Ltot > 0x7fffffffLL) return fail(LRKV_ERR_INVALID_ARGUMENT, "ctx_len + T overflows");
   if ((s = check_kv(kv, p)) != LRKV_OK) return s;
   if ((s = check_u(u, p, (int)Ltot)) != LRKV_OK) return s;
   if (workspace_bytes < (size_t)lrkv::kWsHeaderBytes) return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %d bytes", workspace_bytes, lrkv::kWsHeaderBytes);
   if (T == 0) return LRKV_OK;
   DeviceInfo dev;
   if ((s = device_info(&dev)) != LRKV_OK) return s;
-  const int D = p->head_dim, RK = p->rank;
+  // RK: the width of the U and B tiles (the kernel instance); p->rank: the caches' true rank
+  const int D = p->head_dim, RK = prefill_kernel_rank(p->rank);
   if (lrkv::prefill_smem_bytes(D, RK) > dev.smem_optin) return fail(LRKV_ERR_UNSUPPORTED, "prefill tiles do not fit in shared memory");
 
   alignas(64) CUtensorMap maps[4];
@@ -619,16 +680,17 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
     if ((s = make_map4(&maps[1], kv->v, dims, str, vbox, vu_swizzle, "V")) != LRKV_OK) return s;
   }
   {
+    // the box is RK wide; ranks past p->rank lie outside the map and arrive as zeros
     const int slots = p->mode == LRKV_BASE_SHARED ? p->num_agents : 1;
-    const uint64_t dims[4] = {(uint64_t)RK, (uint64_t)Ltot, (uint64_t)slots, (uint64_t)p->num_sessions};
+    const uint64_t dims[4] = {(uint64_t)p->rank, (uint64_t)Ltot, (uint64_t)slots, (uint64_t)p->num_sessions};
     const int64_t str[3] = {u->stride_token, u->stride_agent, u->stride_session};
     const uint32_t box[4] = {(uint32_t)RK, 128, 1, 1};
     if ((s = make_map4(&maps[2], u->u, dims, str, box, vu_swizzle, "U")) != LRKV_OK) return s;
   }
-  {  // B [N, r, Hkv*d]: box = 64 dims of one KV head x r ranks of one agent, 128B-swizzled
-     // (the B operand of the Z B MMA, d-major)
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p->num_kv_heads, (uint64_t)RK, (uint64_t)p->num_agents};
-    const int64_t str[3] = {D, (int64_t)p->num_kv_heads * D, (int64_t)RK * p->num_kv_heads * D};
+  {  // B [N, r, Hkv*d]: box = 64 dims of one KV head x RK ranks of one agent, 128B-swizzled
+     // (the B operand of the Z B MMA, d-major; ranks past p->rank arrive as zeros)
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p->num_kv_heads, (uint64_t)p->rank, (uint64_t)p->num_agents};
+    const int64_t str[3] = {D, (int64_t)p->num_kv_heads * D, (int64_t)p->rank * p->num_kv_heads * D};
     const uint32_t box[4] = {64, 1, (uint32_t)RK, 1};
     if ((s = make_map4(&maps[3], b, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B, "B")) != LRKV_OK) return s;
   }
@@ -659,6 +721,7 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
   pp.max_parts = pl.max_parts;
   pp.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + pl.tickets_off);
   pp.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pl.partials_off);
+  take_stall_hook(&pp.spin_cap, &pp.stall);
   lrkv::PrefillMaps pm = {maps};
   s = lrkv::launch_prefill(pp, pm, D, RK, pl.ctas, stream);
   if (s != LRKV_OK) return fail(s, "prefill launch failed: %s", cudaGetErrorString(cudaGetLastError()));

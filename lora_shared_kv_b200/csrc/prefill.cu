@@ -10,8 +10,9 @@
 // the end.  Umask_i drops U rows before the agent's aLoRA offset ("RoleKV",
 // "What it does").
 //
-// A 128-row tile is one agent, one KV head, 128/G chunk tokens x the G query
-// heads that share the KV head, so every K/V block loaded serves all of them.
+// A 128-row tile is one agent, one KV head, floor(128/G) chunk tokens x the G
+// query heads that share the KV head, so every K/V block loaded serves all of
+// them (when G does not divide 128, the last 128 mod G rows are unused).
 // The (tile, 128-key block) pairs are split evenly over one persistent CTA per
 // SM (stream-K): a CTA walks a contiguous range of them, tile after tile, and
 // a tile cut by a range boundary is finished by the last of its CTAs to get
@@ -30,9 +31,9 @@
 //                 sums l of exactly the bf16 weights come out with O.  U rows
 //                 before the aLoRA offset are zero-filled (the U of blocks
 //                 wholly before it is not loaded).  At the end of a segment it
-//                 adds Z B_i,g to O with one more MMA pair (Z converted to bf16
-//                 in TMEM, B_i,g in shared memory), so the epilogue only divides
-//                 by l.
+//                 adds Z B_i,g to O with two more MMA pairs (Z split into bf16
+//                 high and low parts in TMEM, B_i,g in shared memory), so the
+//                 epilogue only divides by l.
 //   warps 4..11   Q into TMEM (the next segment's as soon as the last S of
 //                 the current one has been read), softmax and epilogue, in two
 //                 warpgroups, one per half of the block's 128 keys; a thread
@@ -222,7 +223,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ======================= producers: K and B (warp 0), V and U (warp 2) =======================
     // Separate issuers, so that K blocks run ahead by their own ring depth and
     // never wait behind a V stage that the PV of two blocks back still holds.
-    if (lane == 0) {
+    // (With the stall test hook they issue nothing, so the other roles' waits run out.)
+    if (lane == 0 && !p.stall) {
       const bool k_role = warp == 0;
       const uint64_t pol_kv = policy_evict_last();  // K/V blocks are reused by the other tiles of the KV head
       const int n_pages = p.page_table ? (p.L0 + p.T + 63) / 64 : 0;
@@ -238,7 +240,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int u_slot = p.mode == LRKV_BASE_SHARED ? sg.agent : 0;
         if (k_role) {
           // B_i,g of this segment into buffer si & 1, once segment si - 2's epilogue is done with it
-          if (si >= 2 && !mbar_wait_bounded(&bars->b_free[si & 1], ((si >> 1) - 1) & 1, abort_flag, p.flags)) {
+          // After an abort the softmax warps release B buffers whose copies may still be
+          // landing: issue nothing more (the abort word is read after the wait's acquire).
+          if ((si >= 2 && !mbar_wait_bounded(&bars->b_free[si & 1], ((si >> 1) - 1) & 1, abort_flag, p.flags, p.spin_cap)) ||
+              *abort_flag) {
             ok = false;
             break;
           }
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int jb = sg.lo; jb < sg.hi; ++jb, ++n) {
           const int st = n % NS;
-          if (!mbar_wait_bounded(&empty[st], ((n / NS) & 1) ^ 1, abort_flag, p.flags)) {
+          if (!mbar_wait_bounded(&empty[st], ((n / NS) & 1) ^ 1, abort_flag, p.flags, p.spin_cap) || *abort_flag) {
             ok = false;
             break;
           }
@@ -336,8 +341,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr uint32_t ID_ZB = umma_idesc_bf16(BM, D, 0, 1);  // O += Z B_i,g
     auto issue_pv = [&]() -> bool {
       const int st = pv_n % VST;
-      if (!mbar_wait_bounded(&bars->p_full[pv_n & 1], (pv_n >> 1) & 1, abort_flag, p.flags)) return false;
-      if (!mbar_wait_bounded(&bars->v_full[st], (pv_n / VST) & 1, abort_flag, p.flags)) return false;
+      if (!mbar_wait_bounded(&bars->p_full[pv_n & 1], (pv_n >> 1) & 1, abort_flag, p.flags, p.spin_cap)) return false;
+      if (!mbar_wait_bounded(&bars->v_full[st], (pv_n / VST) & 1, abort_flag, p.flags, p.spin_cap)) return false;
       uint8_t* Us = smem + Lay::V_OFF + st * Lay::V_STAGE + Lay::U_OFF;
       if (pv_jb * BN < pv_a) {
         // U rows before the offset are zero-filled before the MMA reads them: all
@@ -365,16 +370,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (pv_last) {
         // the segment's O += Z B_i,g: Z (bf16 pairs) in the S buffer of its last block, B in buffer pv_si & 1
-        if (!mbar_wait_bounded(&bars->zb_full, pv_si & 1, abort_flag, p.flags)) return false;
-        if (!mbar_wait_bounded(&bars->b_full[pv_si & 1], (pv_si >> 1) & 1, abort_flag, p.flags)) return false;
+        if (!mbar_wait_bounded(&bars->zb_full, pv_si & 1, abort_flag, p.flags, p.spin_cap)) return false;
+        if (!mbar_wait_bounded(&bars->b_full[pv_si & 1], (pv_si >> 1) & 1, abort_flag, p.flags, p.spin_cap)) return false;
         if (lane == 0) {
           tc_fence_after();
           const uint32_t b_base = smem_u32(smem + Lay::B_OFF + (pv_si & 1) * Lay::B_BYTES);
           const uint32_t a_z = tmem + (pv_n & 1 ? Lay::COL_S1 : Lay::COL_S0);
 #pragma unroll
-          for (int kk = 0; kk < RK / 16; ++kk) {
-            const uint64_t b = umma_desc(b_base + kk * (16 * 128), RK * 128, 1024, 2);
-            umma_ts(tmem + Lay::COL_O, a_z + kk * 8, b, ID_ZB, 1u);
+          for (int part = 0; part < 2; ++part) {  // Z_hi B, then Z_lo B (columns RK / 2 on)
+#pragma unroll
+            for (int kk = 0; kk < RK / 16; ++kk) {
+              const uint64_t b = umma_desc(b_base + kk * (16 * 128), RK * 128, 1024, 2);
+              umma_ts(tmem + Lay::COL_O, a_z + part * (RK / 2) + kk * 8, b, ID_ZB, 1u);
+            }
           }
           umma_commit(&bars->zb_done);
         }
@@ -387,10 +395,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       f += sg.hi - sg.lo;
       const int a_i = agent_offset(p, sg.agent, false);
       // the segment's Q is in TMEM (its previous content was read by the last S issued)
-      ok = mbar_wait_bounded(&bars->q_full, si & 1, abort_flag, p.flags);
+      ok = mbar_wait_bounded(&bars->q_full, si & 1, abort_flag, p.flags, p.spin_cap);
       for (int jb = sg.lo; jb < sg.hi && ok; ++jb, ++n) {
         const int st = n % KST;
-        ok = mbar_wait_bounded(&bars->k_full[st], (n / KST) & 1, abort_flag, p.flags);
+        ok = mbar_wait_bounded(&bars->k_full[st], (n / KST) & 1, abort_flag, p.flags, p.spin_cap);
         if (!ok) break;
         if (lane == 0) {
           tc_fence_after();
@@ -426,6 +434,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     float* xmax = reinterpret_cast<float*>(smem + Lay::XCH_OFF);  // [blk & 1][half][row]
     volatile int* ticket_last = reinterpret_cast<volatile int*>(xmax + 4 * BM);
     const int jj = row / p.G, hh = row % p.G;
+    // A tile holds floor(128 / G) tokens x G heads; when G does not divide 128
+    // the last 128 mod G rows belong to no token: no query, no output.
+    const bool row_used = jj < BM / p.G;
     const float NEG_INF = -INFINITY;
     bool ok = true;
 
@@ -439,7 +450,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           wg * QH);
 #pragma unroll
       for (int v = 0; v < QH / 8; ++v) {
-        const uint4 w = token < p.T ? __ldg(qsrc + v) : make_uint4(0, 0, 0, 0);
+        const uint4 w = (row_used && token < p.T) ? __ldg(qsrc + v) : make_uint4(0, 0, 0, 0);
         qw[4 * v] = w.x;
         qw[4 * v + 1] = w.y;
         qw[4 * v + 2] = w.z;
@@ -480,7 +491,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int limit = p.L0 + token;  // last visible key of this row
       float m_ref = NEG_INF;
       for (int jb = sg.lo; jb < sg.hi; ++jb, ++n) {
-        if (ok) ok = mbar_wait_bounded(&bars->s_full[n & 1], (n >> 1) & 1, abort_flag, p.flags);
+        if (ok) ok = mbar_wait_bounded(&bars->s_full[n & 1], (n >> 1) & 1, abort_flag, p.flags, p.spin_cap);
         tc_fence_after();
         const uint32_t s_col = n & 1 ? Lay::COL_S1 : Lay::COL_S0;
         float x[HB];
@@ -514,7 +525,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (jb > sg.lo) {
             // O, Z and l hold the segment's blocks before this one: rescale this
             // half's share of their columns in TMEM once the previous PV is done
-            if (ok) ok = mbar_wait_bounded(&bars->o_ready[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, p.flags);
+            if (ok) ok = mbar_wait_bounded(&bars->o_ready[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, p.flags, p.spin_cap);
             tc_fence_after();
 #pragma unroll
             for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
@@ -565,7 +576,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // last block, free once its PV is done) for the O += Z B_i,g MMA; then
       // out = O / l, or this segment's rows are published for the tile's last CTA.
       const int nl = n - 1;  // the segment's last block
-      if (ok) ok = mbar_wait_bounded(&bars->o_ready[nl & 1], (nl >> 1) & 1, abort_flag, p.flags);
+      if (ok) ok = mbar_wait_bounded(&bars->o_ready[nl & 1], (nl >> 1) & 1, abort_flag, p.flags, p.spin_cap);
       tc_fence_after();
       float l;
       {
@@ -581,19 +592,31 @@ __global__ void __launch_bounds__(THREADS, 1)
           l = __uint_as_float(r2[0]);
         }
         if (wg == 1) {
-          uint32_t zp[RK / 2];
+          // Z = Z_hi + Z_lo with both parts bf16: Z_hi = bf16(Z), Z_lo = bf16(Z - Z_hi)
+          // (the difference is exact in fp32), so the two MMAs Z_hi B + Z_lo B carry
+          // Z to about 2^-17 of its size instead of the 2^-9 of one bf16 rounding.
+          uint32_t zh[RK / 2], zl[RK / 2];
 #pragma unroll
-          for (int k = 0; k < RK / 2; ++k) zp[k] = pack_bf16x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+          for (int k = 0; k < RK / 2; ++k) {
+            const float z0 = __uint_as_float(r[2 * k]), z1 = __uint_as_float(r[2 * k + 1]);
+            zh[k] = pack_bf16x2(z0, z1);
+            zl[k] = pack_bf16x2(z0 - __uint_as_float(zh[k] << 16), z1 - __uint_as_float(zh[k] & 0xffff0000u));
+          }
           const uint32_t zcol = nl & 1 ? Lay::COL_S1 : Lay::COL_S0;
-          if constexpr (RK == 32) tmem_st16(tmem + lane_addr + zcol, zp);
-          else tmem_st8(tmem + lane_addr + zcol, zp);
+          if constexpr (RK == 32) {
+            tmem_st16(tmem + lane_addr + zcol, zh);
+            tmem_st16(tmem + lane_addr + zcol + RK / 2, zl);
+          } else {
+            tmem_st8(tmem + lane_addr + zcol, zh);
+            tmem_st8(tmem + lane_addr + zcol + RK / 2, zl);
+          }
           tmem_wait_st();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->zb_full);
-      if (ok) ok = mbar_wait_bounded(&bars->zb_done, si & 1, abort_flag, p.flags);
+      if (ok) ok = mbar_wait_bounded(&bars->zb_done, si & 1, abort_flag, p.flags, p.spin_cap);
       tc_fence_after();
       const bool whole = sg.lo == 0 && sg.hi == sg.nb;
       bool finish = true;
@@ -646,7 +669,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (finish) {
         const float inv_l = l > 0.f ? 1.f / l : 0.f;
-        const bool write = token < p.T && ok;
+        const bool write = row_used && token < p.T && ok;
         const int h = sg.g * p.G + hh;
 #pragma unroll 1
         for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {

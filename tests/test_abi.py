@@ -191,11 +191,61 @@ def _prefill_ws_expected(T, L0, G, Hkv, N, d, sms=148):
     (512, 16384, 16, 8, 4, 128, 32),   # the prefill workload: 2 parts per tile at most
     (100, 300, 4, 2, 2, 128, 32),      # fewer blocks than SMs: one block per CTA
     (1, 77, 8, 4, 2, 64, 16),
+    (64, 8192, 12, 2, 3, 128, 16),     # Qwen2.5-Coder role header: G = 6, tiles of 21 tokens (126 rows)
+    (300, 1000, 10, 2, 2, 64, 8),      # G = 5 (25 tokens per tile), rank 8
+    (9, 40, 128, 1, 1, 64, 16),        # G = 128: one token per tile
 ])
 def test_prefill_workspace_follows_the_stream_k_plan(T, L0, Hq, Hkv, N, d, r):
     prob = lrkv.make_problem(1, N, Hq, Hkv, d, r, lrkv.BASE_SHARED)
     got = lrkv.lib().lrkv_prefill_workspace_bytes(ctypes.byref(prob), L0, T)
     assert got == _prefill_ws_expected(T, L0, Hq // Hkv, Hkv, N, d)
+
+
+def _prefill(prob, kv=None, uv=None, q=FAKE, session=0, L0=1000, T=64, ws=FAKE, ws_bytes=1 << 20, out_dtype=0):
+    L = lrkv.lib()
+    if kv is None:
+        kv, uv = _views()
+    return L.lrkv_attn_prefill_chunk(ctypes.byref(prob), ctypes.c_void_p(q), ctypes.byref(kv), session, L0, T,
+                                     ctypes.byref(uv), ctypes.c_void_p(FAKE), None, ctypes.c_void_p(FAKE), out_dtype,
+                                     ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def test_prefill_argument_errors():
+    kv, uv = _views()
+    p = _problem(S=2)
+    assert _prefill(_problem(d=96), kv, uv) == 2             # unsupported head_dim
+    assert _prefill(_problem(r=12), kv, uv) == 2             # unsupported rank
+    assert _prefill(_problem(Hq=10, Hkv=4), kv, uv) == 2     # Hq not a multiple of Hkv
+    assert _prefill(_problem(Hq=129 * 2, Hkv=2), kv, uv) == 2  # G > 128: a tile cannot hold one token
+    assert _prefill(_problem(N=17), kv, uv) == 2             # too many agents
+    assert _prefill(_problem(mode=3), kv, uv) == 1
+    assert _prefill(p, kv, uv, q=0) == 1                     # NULL q
+    assert _prefill(p, kv, uv, ws=0) == 1                    # NULL workspace
+    assert _prefill(p, kv, uv, q=FAKE + 4) == 3              # misaligned q
+    assert _prefill(p, kv, uv, ws=FAKE + 8) == 3             # misaligned workspace
+    assert _prefill(p, kv, uv, out_dtype=7) == 1             # unknown output dtype
+    assert _prefill(p, kv, uv, session=2) == 1               # session out of range
+    assert _prefill(p, kv, uv, session=-1) == 1
+    assert _prefill(p, kv, uv, L0=-1) == 1
+    assert _prefill(p, kv, uv, T=-5) == 1
+    assert _prefill(p, kv, uv, L0=8190, T=64) == 1           # rows past the U capacity (8192)
+    assert _prefill(p, kv, uv, L0=0x7fffffff, T=2) == 1      # ctx_len + T overflows
+    kvm, _ = _views(misaligned=True)
+    assert _prefill(p, kvm, uv) == 3                         # misaligned k
+    assert _prefill(p, kv, uv, ws_bytes=100) == 4            # workspace below its status header
+    assert _prefill(p, kv, uv, T=0) == 0                     # an empty chunk is a no-op, no launch
+    L = lrkv.lib()
+    assert L.lrkv_attn_prefill_chunk(None, None, None, 0, 0, 0, None, None, None, None, 0, None, 0, None) == 1
+
+
+def test_prefill_workspace_is_zero_for_refused_shapes():
+    L = lrkv.lib()
+    for prob, L0, T in [(_problem(d=96), 100, 10), (_problem(r=12), 100, 10), (_problem(Hq=10, Hkv=4), 100, 10),
+                        (_problem(Hq=129 * 2, Hkv=2), 100, 10), (_problem(), -1, 10), (_problem(), 100, -1),
+                        (_problem(), 0x7fffffff, 2)]:
+        assert L.lrkv_prefill_workspace_bytes(ctypes.byref(prob), L0, T) == 0
+    for r in (8, 16, 32):  # every supported rank and G = 6 get a plan
+        assert L.lrkv_prefill_workspace_bytes(ctypes.byref(_problem(r=r)), 8192, 64) > 256
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -2,10 +2,12 @@
 
 Row j of the chunk sits at absolute position L0 + j and sees keys t <= L0 + j.
 The small cases span several 128-key blocks, a ragged last tile and block,
-G in {1, 2, 4}, both head dims, both ranks, both sharing modes, offsets inside
-a block and before the chunk; NaN-poisoned U rows must not leak.  The
-full-size case is the prefill workload (4 agents, 512 rows onto 16384) with
-the low-rank append in front, checked on sampled rows.
+G in {1, 2, 3, 4, 5, 6, 7} (tiles of floor(128 / G) tokens when G does not
+divide 128), both head dims, every rank, both sharing modes, offsets inside a
+block, inside the chunk and before it; NaN-poisoned U rows must not leak.  The
+full-size cases are the prefill workload (4 agents, 512 rows onto 16384) with
+the low-rank append in front, checked on sampled rows, once with the
+workload's offsets and once with offsets inside the context and the chunk.
 """
 
 import zlib
@@ -74,6 +76,12 @@ SHAPES = [
     (2, 130, 16, 8, 128, 32, 4096, 0, [4200, 0]),
     (2, 1, 8, 4, 128, 16, 77, 1, [30, 0]),
     (1, 257, 2, 2, 64, 32, 129, 0, [129]),
+    # Qwen2.5-Coder-1.5B role switch (RoleKV): 12/2 heads (G = 6, tiles of 21 tokens = 126 rows),
+    # a 64-row role header onto 8192 shared tokens, three roles, offsets inside the context and the chunk
+    (3, 64, 12, 2, 128, 16, 8192, 0, [6000, 7000, 8200]),
+    (2, 90, 10, 2, 64, 8, 500, 0, [0, 530]),       # G = 5, rank 8
+    (2, 50, 6, 2, 128, 8, 300, 1, [10, 320]),      # G = 3, rank 8, one shared U
+    (1, 30, 7, 1, 128, 32, 200, 0, [100]),         # G = 7
 ]
 
 
@@ -132,14 +140,26 @@ def test_prefill_rows_before_offset_equal_base():
     assert torch.equal(out, base)
 
 
-def test_prefill_workload_with_append_sampled():
+@pytest.mark.parametrize("offsets,rows", [
+    (None, [0, 1, 63, 64, 200, 383, 384, 511]),
+    # aLoRA boundaries inside the 16384-token context and one inside the chunk (row 216):
+    # rows on both sides of it
+    ((9000, 12000, 16000, 16600), [0, 1, 64, 200, 215, 216, 217, 300, 511]),
+], ids=["workload-offsets", "offsets-inside"])
+def test_prefill_workload_with_append_sampled(offsets, rows):
     cfg = CONFIGS["cfg4"]
-    inp = make_prefill_inputs(cfg, device=DEV)
+    offs = None if offsets is None else torch.tensor(offsets, dtype=torch.int32)
+    inp = make_prefill_inputs(cfg, device=DEV, offsets=offs)
     lrkv.lrkv_append_lr_cache(inp.x, inp.a_down, inp.u, session=0, start_row=cfg.L0)
     out = prefill_gpu(inp.q, inp.k, inp.v, inp.u, inp.b, inp.offsets, cfg.L0, cfg.T, cfg.mode)
-    rows = [0, 1, 63, 64, 200, 383, 384, 511]
     ref = oracle.prefill_chunk(inp.q.cpu(), inp.k[0].cpu(), inp.v[0].cpu(), inp.u[0].cpu(), inp.b.cpu(),
                                inp.offsets.cpu(), cfg.L0, cfg.mode, rows=rows)
     got = to_np(out)
     assert_parity(got[:, rows], ref[:, rows], "prefill workload")
     assert torch.isfinite(out.float()).all()
+    if offsets is not None:
+        # rows whose every visible key lies before the last agent's offset carry no adapter term
+        base = prefill_gpu(inp.q, inp.k, inp.v, inp.u, torch.zeros_like(inp.b), inp.offsets, cfg.L0, cfg.T,
+                           cfg.mode)
+        early = [j for j in rows if cfg.L0 + j < offsets[3]]
+        assert early and torch.equal(out[3, early], base[3, early])
