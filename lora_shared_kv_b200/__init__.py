@@ -47,10 +47,12 @@ EXPORTS = (
     "lrkv_decode_workspace_bytes",
     "lrkv_attn_decode",
     "lrkv_attn_decode_static_scratch",
+    "lrkv_query_static_scratch_status",
     "lrkv_prefill_workspace_bytes",
     "lrkv_attn_prefill_chunk",
     "lrkv_workspace_reset",
     "lrkv_query_device_status",
+    "lrkv_debug_stall_next_launch",
     "lrkv_status_string",
     "lrkv_last_error_detail",
     "lrkv_version",
@@ -112,6 +114,8 @@ def lib():
                                               i32, vp, sz, vp]
         L.lrkv_workspace_reset.argtypes = [vp, sz, vp]
         L.lrkv_query_device_status.argtypes = [vp, i32, P(ctypes.c_uint32), vp]
+        L.lrkv_query_static_scratch_status.argtypes = [i32, P(ctypes.c_uint32), vp]
+        L.lrkv_debug_stall_next_launch.argtypes = [ctypes.c_uint32]
         L.lrkv_status_string.argtypes = [i32]
         L.lrkv_status_string.restype = ctypes.c_char_p
         L.lrkv_last_error_detail.argtypes = []
@@ -119,7 +123,8 @@ def lib():
         L.lrkv_version.restype = i32
         for name in ("lrkv_append_lr_cache", "lrkv_attn_decode", "lrkv_attn_decode_static_scratch",
                      "lrkv_attn_prefill_chunk",
-                     "lrkv_workspace_reset", "lrkv_query_device_status"):
+                     "lrkv_workspace_reset", "lrkv_query_device_status", "lrkv_query_static_scratch_status",
+                     "lrkv_debug_stall_next_launch"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -304,6 +309,22 @@ def lrkv_query_device_status(workspace, clear=True, stream=None):
     if st not in (0, 6, 7):
         _check(st)
     return _STATUS[st], flags.value
+
+
+def lrkv_query_static_scratch_status(clear=True, stream=None):
+    """Flags of the most recent lrkv_attn_decode_static_scratch call on the current device: synchronise and
+    return (status_name, flags); does not raise on device-side flags."""
+    flags = ctypes.c_uint32(0)
+    st = lib().lrkv_query_static_scratch_status(1 if clear else 0, ctypes.byref(flags), _stream(stream))
+    if st not in (0, 6, 7):
+        _check(st)
+    return _STATUS[st], flags.value
+
+
+def lrkv_debug_stall_next_launch(spin_cap):
+    """Test hook: the next decode or prefill call from this thread issues no copies and its bounded waits give
+    up after spin_cap attempts (the launch then reports LRKV_ERR_TIMEOUT).  0 disarms."""
+    _check(lib().lrkv_debug_stall_next_launch(int(spin_cap)))
 
 
 def version():

@@ -35,11 +35,6 @@ inline cudaError_t ensure_dynamic_smem(int bytes) {
   return e;
 }
 
-// Spin cap of every bounded wait.  A try_wait suspends for a short while per
-// attempt, so this is well over a second of waiting: far beyond any healthy
-// pipeline stall, and the kernel then records LRKV_DEVFLAG_TIMEOUT and returns.
-constexpr uint32_t kSpinCap = 1u << 24;
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -77,14 +72,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait on a phase of an mbarrier.  Returns false (and records a
-// timeout flag and raises the CTA's abort word) when the cap is reached or
-// another thread of the CTA has already aborted.
+// timeout flag and raises the CTA's abort word) when `cap` failed attempts are
+// reached or another thread of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, unsigned* err) {
+                                                  volatile int* abort_flag, unsigned* err,
+                                                  uint32_t cap = kSpinCap) {
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (++spins >= kSpinCap) {
+    if (++spins >= cap) {
       *abort_flag = 1;
       if (err) atomicOr(err, LRKV_DEVFLAG_TIMEOUT);
       return false;

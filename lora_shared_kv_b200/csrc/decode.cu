@@ -169,7 +169,8 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
   int stage = 0;
   uint32_t phase = 0;
   int n = 0;
-  for (long long t = t_begin; t < t_end;) {
+  bool stop = p.stall != 0;  // the test hook: issue nothing, so the consumers' waits run out
+  for (long long t = t_begin; t < t_end && !stop;) {
     Seg sg = make_seg(p, t, t_end, false);
     t += sg.hi - sg.lo;
     seg_rows(p, sg);
@@ -194,7 +195,16 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
       const unsigned umask = p.mode == LRKV_BASE_SHARED ? need : (need ? 1u : 0u);
       const bool page_ok = !p.paged || (phys >= 0 && phys < p.num_pages);
       const uint32_t bytes = (page_ok ? 2 * KV_BYTES : 0) + __popc(umask) * U_BYTES;
-      mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.flags);
+      const bool freed = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.flags, p.spin_cap);
+      // After an abort the consumers release stages without waiting for their
+      // copies, so nothing more may be issued: a stage could receive a second
+      // copy while the first is still landing.  The abort word is read after the
+      // wait (whose acquire orders it), and the whole warp leaves together.
+      if (__any_sync(0xffffffffu, !freed || *abort_flag)) {
+        stop = true;
+        --n;  // this tile was not issued
+        break;
+      }
       if (lane == 0) {
         if (!page_ok) atomicOr(p.flags, LRKV_DEVFLAG_PAGE);
         seq[stage] = n - 1;
@@ -643,7 +653,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       {
         uint32_t spins = 0;
         while (seq[my_stage] != my_n) {
-          if (*abort_flag || ++spins >= kSpinCap) {
+          if (*abort_flag || ++spins >= p.spin_cap) {
             if (!*abort_flag) {
               *abort_flag = 1;
               atomicOr(p.flags, LRKV_DEVFLAG_TIMEOUT);
@@ -652,7 +662,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           }
         }
       }
-      mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags);
+      mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags, p.spin_cap);
       const uint32_t Ks = ring_s + my_stage * lay.stage_bytes;
       const uint32_t Vs = Ks + KV_BYTES;
       const uint32_t Us = Vs + KV_BYTES;
@@ -864,7 +874,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       st.l[e] = v;
     }
     // the record buffer of segment sn - 2 must have been released by the epilogue warp
-    if (sn >= 2) mbar_wait_bounded(&rec_free[buf], ((sn >> 1) - 1) & 1, abort_flag, p.flags);
+    if (sn >= 2) mbar_wait_bounded(&rec_free[buf], ((sn >> 1) - 1) & 1, abort_flag, p.flags, p.spin_cap);
     // chain the owner groups into the record (same rows, different tiles)
     for (int src = NOG - 1; src >= 1; --src) {
       if (og == src) store_rows<D, RK>(st, merge, RP, rbase, g8, t4);
@@ -905,7 +915,7 @@ __device__ void decode_epilogue(const DecodeParams& p, uint8_t* smem, const Deco
     seg_rows(p, sg);
     if (t >= t_end) break;  // the consumers finish the last segment
     const int buf = sn & 1;
-    if (!mbar_wait_bounded(&rec_full[buf], (sn >> 1) & 1, abort_flag, p.flags)) break;
+    if (!mbar_wait_bounded(&rec_full[buf], (sn >> 1) & 1, abort_flag, p.flags, p.spin_cap)) break;
     const SegInfo si = seg_info(p, sg);
     finish_segment<D, NT, RK, 32, (RK >= 32 ? 1 : 2)>(p, si, merge0 + buf * REC, scw, bcast, lane,
                                                       [] { __syncwarp(); });

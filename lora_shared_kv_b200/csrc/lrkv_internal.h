@@ -20,6 +20,11 @@ constexpr int kMaxRowsPerItem = 32;     // query rows (agents x GQA heads) per d
 constexpr int kMaxAgents = 16;
 constexpr int kTileRun = 4;             // decode tiles visited contiguously (see TileOrder in decode.cu)
 
+// Spin cap of every bounded wait.  A try_wait suspends for a short while per
+// attempt, so this is well over a second of waiting: far beyond any healthy
+// pipeline stall, and the kernel then records LRKV_DEVFLAG_TIMEOUT and returns.
+constexpr uint32_t kSpinCap = 1u << 24;
+
 // ---------------------------------------------------------------------------
 // decode
 // ---------------------------------------------------------------------------
@@ -52,6 +57,11 @@ struct DecodeParams {
   float* partials;
   int* tickets;
   unsigned* flags;
+  // Failure-detection test hook (lrkv_debug_stall_next_launch): every bounded
+  // wait gives up after spin_cap failed attempts, and with `stall` the
+  // producer issues no copies, so the consumers' waits run out.
+  unsigned spin_cap;
+  int stall;
 };
 
 // Consumer warp groups of the decode kernel (NT warps each, eight query rows

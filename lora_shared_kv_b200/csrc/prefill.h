@@ -25,6 +25,8 @@ struct PrefillParams {
   int max_parts;             // CTAs that can share one tile
   int* tickets;              // [tiles], zero between launches
   float* partials;           // [tiles][max_parts][128 rows: m, l, O + Z B (d)]
+  unsigned spin_cap;         // failed attempts after which a bounded wait gives up
+  int stall;                 // test hook: the producers issue no copies (the waits run out)
 };
 
 // Stream-K plan of a prefill launch and its workspace (bytes from the start of

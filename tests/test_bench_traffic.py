@@ -52,6 +52,6 @@ def test_traffic_only_while_the_sources_match(tmp_path, monkeypatch):
     assert bench.profiled_traffic(KERNEL, WORKLOAD) is None            # no summary
     _summary(tmp_path, bench.kernel_sources_sha256(KERNEL), 123456789)
     assert bench.profiled_traffic(KERNEL, WORKLOAD) == 123456789
-    _edit(os.path.join(src, "common.cuh"), "constexpr uint32_t kSpinCap = 1u << 24;",
+    _edit(os.path.join(src, "lrkv_internal.h"), "constexpr uint32_t kSpinCap = 1u << 24;",
           "constexpr uint32_t kSpinCap = 1u << 23;")
     assert bench.profiled_traffic(KERNEL, WORKLOAD) is None            # the kernel changed since

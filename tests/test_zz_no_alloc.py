@@ -6,49 +6,88 @@ own allocator, or a long-running server where cudaMalloc would synchronise the
 device and can fail on a fragmented heap.  lrkv_attn_decode_static_scratch
 serves them from one fixed scratch array inside the library.  These tests call
 it through the C ABI, twice in a row (the scratch keeps the previous call's
-contents), and compare with the regular entry point that takes a caller-owned
-workspace, under the same tolerance as the other decode tests.
+contents), and compare each output with the fp64 oracle and with the regular
+entry point that takes a caller-owned workspace, under the same tolerance as
+the other decode tests.  The scratch's device-side flags are read back with
+lrkv_query_static_scratch_status.
 """
 
 import pytest
 import torch
 
 import lora_shared_kv_b200 as lrkv
-from gpu_util import MAX_ABS, REL_L2, errors, to_np
+from gpu_util import MAX_ABS, REL_L2, assert_parity, decode_oracle, errors, to_np
 from workloads.gen import _normal
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _case(seed, S=4, N=3, Hq=12, Hkv=2, d=128, r=16, L=2048):
+def _case(seed, S=4, N=3, Hq=12, Hkv=2, d=128, r=16, L=2048, mode=lrkv.BASE_SHARED, paged=False):
     g = torch.Generator(device=DEV)
     g.manual_seed(seed)
     q = _normal((S, N, Hq, d), 1.0, g, DEV)
-    k = _normal((S, Hkv, L, d), 1.0, g, DEV)
-    v = _normal((S, Hkv, L, d), 1.0, g, DEV)
-    u = _normal((S, N, L, r), 1.0, g, DEV)
+    u = _normal((S, N if mode == lrkv.BASE_SHARED else 1, L, r), 1.0, g, DEV)
     b = _normal((N, r, Hkv * d), 0.05, g, DEV)
-    offs = torch.tensor([[100, 1500, 2047]] * S, dtype=torch.int32, device=DEV)
+    offs = torch.tensor([[100, 1500, 2047, 5][:N]] * S, dtype=torch.int32, device=DEV)
     seq = torch.tensor([L, L - 1, L // 2, 77][:S], dtype=torch.int32, device=DEV)
-    return q, k, v, u, b, offs, seq
+    if not paged:
+        k = _normal((S, Hkv, L, d), 1.0, g, DEV)
+        v = _normal((S, Hkv, L, d), 1.0, g, DEV)
+        return q, k, v, u, b, offs, seq, None
+    n_lp = L // 64
+    k = _normal((S * n_lp + 3, Hkv, 64, d), 1.0, g, DEV)
+    v = _normal((S * n_lp + 3, Hkv, 64, d), 1.0, g, DEV)
+    perm = torch.randperm(S * n_lp + 3, generator=g, device=DEV)[:S * n_lp]
+    table = perm.to(torch.int32).view(S, n_lp).contiguous()
+    return q, k, v, u, b, offs, seq, table
 
 
-def test_static_scratch_decode_matches_workspace_decode_twice():
+CASES = [
+    dict(),                                                          # dense BaseShared, Qwen2.5-Coder heads
+    dict(S=2, N=4, Hq=16, Hkv=8, L=4096, mode=lrkv.BASE_LR_SHARED, paged=True),  # paged, one shared U
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=["dense-shared", "paged-lrshared"])
+def test_static_scratch_decode_matches_oracle_and_workspace_decode_twice(case):
     for seed in (101, 202):  # two calls in a row on different inputs
-        q, k, v, u, b, offs, seq = _case(seed)
+        q, k, v, u, b, offs, seq, table = _case(seed, **case)
         S, N, Hq, d = q.shape
-        prob = lrkv.make_problem(S, N, Hq, k.shape[1], d, u.shape[-1], lrkv.BASE_SHARED)
-        kv = lrkv.kv_view_dense(k, v)
-        ws = torch.zeros(lrkv.lrkv_decode_workspace_bytes(prob, k.shape[2]), dtype=torch.uint8, device=DEV)
+        L = u.shape[2]
+        mode = case.get("mode", lrkv.BASE_SHARED)
+        prob = lrkv.make_problem(S, N, Hq, k.shape[1], d, u.shape[-1], mode)
+        kv = lrkv.kv_view_dense(k, v) if table is None else lrkv.kv_view_paged(k, v, table)
+        ws = torch.zeros(lrkv.lrkv_decode_workspace_bytes(prob, L), dtype=torch.uint8, device=DEV)
         ref = torch.empty_like(q)
-        lrkv.lrkv_attn_decode(prob, q, kv, seq, k.shape[2], u, b, offs, ref, ws)
+        lrkv.lrkv_attn_decode(prob, q, kv, seq, L, u, b, offs, ref, ws)
         got = torch.full_like(q, float("nan"))
-        lrkv.lrkv_attn_decode_static_scratch(prob, q, kv, seq, k.shape[2], u, b, offs, got)
+        lrkv.lrkv_attn_decode_static_scratch(prob, q, kv, seq, L, u, b, offs, got)
         torch.cuda.synchronize()
-        max_abs, rel = errors(to_np(got), to_np(ref))
+        assert lrkv.lrkv_query_static_scratch_status() == ("LRKV_OK", 0)
         assert torch.isfinite(got.float()).all()
+        max_abs, rel = errors(to_np(got), to_np(ref))
         assert max_abs <= MAX_ABS and rel <= REL_L2, (seed, max_abs, rel)
+        want = decode_oracle(q, k, v, u, b, offs, seq, mode, page_table=table)
+        assert_parity(to_np(got), want, f"static scratch seed {seed}")
+
+
+def test_static_scratch_reports_a_bad_page_id():
+    q, k, v, u, b, offs, seq, table = _case(7, S=2, N=2, Hq=4, Hkv=2, L=1024, paged=True)
+    S, N, Hq, d = q.shape
+    prob = lrkv.make_problem(S, N, Hq, k.shape[1], d, u.shape[-1], lrkv.BASE_SHARED)
+    bad = table.clone()
+    bad[1, 3] = k.shape[0]  # one page id past the pool: that tile is skipped and flagged
+    out = torch.empty_like(q)
+    lrkv.lrkv_attn_decode_static_scratch(prob, q, lrkv.kv_view_paged(k, v, bad), seq, 1024, u, b, offs, out)
+    st, flags = lrkv.lrkv_query_static_scratch_status(clear=False)
+    assert st == "LRKV_ERR_DEVICE_FAULT" and flags & 0x4, (st, hex(flags))
+    assert lrkv.lrkv_query_static_scratch_status()[0] == "LRKV_ERR_DEVICE_FAULT"  # read once more, then cleared
+    assert lrkv.lrkv_query_static_scratch_status() == ("LRKV_OK", 0)
+    # the next call clears the flags itself and, with a good table, raises none
+    lrkv.lrkv_attn_decode_static_scratch(prob, q, lrkv.kv_view_paged(k, v, table), seq, 1024, u, b, offs, out)
+    assert lrkv.lrkv_query_static_scratch_status() == ("LRKV_OK", 0)
+    assert_parity(to_np(out), decode_oracle(q, k, v, u, b, offs, seq, lrkv.BASE_SHARED, page_table=table), "after")
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size():
