@@ -2,14 +2,21 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lrkv|reference] [--workload NAME]
 
-Default workload: the Qwen2.5-Coder-1.5B-shaped decode (28 layers, 12 query /
-2 KV heads, d = 128, three roles in BaseShared mode at r = 16, 32 sessions,
-8192 shared tokens, offsets 6000 / 7000 / 7800).  One step = one decode query
-per (session, agent) through the attention of all 28 layers (28 launches of
-the decode kernel, captured once in a CUDA graph and replayed).  Inputs are
-synthetic (seeded N(0, 1) draws of the model's shapes) and resident in HBM;
-each layer has its own buffers, so a step streams 7.5 GB (> L2) and no L2
-flush is needed between steps.
+Default workload (the headline): the largest single-GPU decode workload, the
+Qwen3-1.7B-shaped long-context case (28 layers, 16 query / 8 KV heads, d = 128,
+eight agents in BaseShared mode at r = 16, 4 sessions, 65536 shared tokens in
+64-token pages with a random page order, offsets drawn in [32768, 65536)).  One
+step = one decode query per (session, agent) through the attention of all 28
+layers (28 launches of the decode kernel, captured once in a CUDA graph and
+replayed).  Inputs are synthetic (seeded N(0, 1) draws of the model's shapes)
+and resident in HBM; each layer has its own buffers, so a step streams 30 GB
+(> L2) and no L2 flush is needed between steps.
+
+The same JSON line carries, under ``decode_workloads``, the other decode
+workloads timed the same way (the Qwen2.5-Coder-1.5B case and each context
+length of the Qwen3-1.7B sweep), and under ``prefill`` the append + causal
+prefill-chunk step, under ``sharing`` the shared / non-shared / full-shared
+comparison.
 
 Prints ONE JSON line (rank 0).  Under torchrun each rank runs the same
 workload on its own data (weak scaling, no collective on the data path); the
@@ -151,7 +158,7 @@ class ClockSampler:
             sel = []
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "50"] + sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                          "-lms", "10"] + sel, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
         except Exception:
             self.proc = None
@@ -279,13 +286,26 @@ def _timed(fn, steps, warmup, sync_all):
     return e0.elapsed_time(e1)
 
 
+def cpu_sample_layers(cfg, n_layers):
+    """Layers the CPU baseline times per session: all of them, or for the long
+    contexts (where one session through every layer would take minutes of fp64
+    work) the first, middle and last layer, with the time scaled by
+    n_layers / 3 (reported as extrapolated)."""
+    if cfg.L >= 32768 and n_layers > 3:
+        return [0, n_layers // 2, n_layers - 1]
+    return list(range(n_layers))
+
+
 def cpu_baseline_decode(runner, min_seconds=10.0, max_seconds=25.0):
-    """fp64 oracle on the host cores: session after session, each through all
-    layers, until at least min_seconds of oracle time (at most max_seconds).
-    Only the oracle calls are timed, not the copies of the inputs to the host."""
+    """fp64 oracle on the host cores: session after session, each through the
+    sampled layers (cpu_sample_layers), until at least min_seconds of oracle
+    time (at most max_seconds).  Only the oracle calls are timed, not the
+    copies of the inputs to the host."""
     import oracle
     from threadpoolctl import threadpool_info
     cfg, inp = runner.cfg, runner.inp
+    nl = len(inp.layers)
+    layers = cpu_sample_layers(cfg, nl)
     cores = len(os.sched_getaffinity(0))
     blas_threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
     dt = 0.0
@@ -294,7 +314,8 @@ def cpu_baseline_decode(runner, min_seconds=10.0, max_seconds=25.0):
     for s in range(cfg.S):
         offs = inp.offsets[s:s + 1].cpu()
         sl = inp.seq_lens[s:s + 1].cpu()
-        for lay in inp.layers:
+        for li in layers:
+            lay = inp.layers[li]
             q, u, b = lay.q[s:s + 1].cpu(), lay.u[s:s + 1].cpu(), lay.b.cpu()
             if cfg.paged:  # this session's pages, in logical order
                 pt = lay.page_table[s].long()
@@ -311,12 +332,17 @@ def cpu_baseline_decode(runner, min_seconds=10.0, max_seconds=25.0):
         sessions += 1
         if dt > min_seconds:
             break
-    queries = cfg.N * done_layers / len(inp.layers)
-    return {"value": queries / dt, "unit": UNIT, "cores": min(cores, blas_threads) if blas_threads else cores,
-            "kind": "oracle",
-            "sample": f"{sessions} session(s) x {len(inp.layers)} layers ({done_layers} session-layers, "
-                      f"{queries:.1f} queries), fp64 numpy, {dt:.1f} s of oracle time; {cores} cores visible, "
-                      f"BLAS threads {blas_threads}"}
+    # one query = one (session, agent) through all nl layers; the sampled layers stand for all of them
+    queries = cfg.N * done_layers / len(layers)
+    t_all = dt * nl / len(layers)
+    extrap = len(layers) < nl
+    sample = (f"{sessions} session(s) x layers {layers if extrap else f'0..{nl - 1}'} "
+              f"({done_layers} session-layers, {queries:.2f} queries), fp64 numpy, {dt:.1f} s of oracle time")
+    if extrap:
+        sample += f"; extrapolated to all {nl} layers (time x {nl}/{len(layers)})"
+    sample += f"; {cores} cores visible, BLAS threads {blas_threads}"
+    return {"value": queries / t_all, "unit": UNIT, "cores": min(cores, blas_threads) if blas_threads else cores,
+            "kind": "oracle", "extrapolated": extrap, "sample": sample}
 
 
 def run_e2e(runner, steps, warmup, sync_all):
@@ -374,7 +400,7 @@ def _eager_ms(fn, steps, warmup):
     return e0.elapsed_time(e1) / steps
 
 
-def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3):
+def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3, return_outputs=False):
     """The pages' comparison of cache sharing, on the same decode kernel.
 
     - shared: the split value cache (base K/V once for all agents, rank-r U_i);
@@ -385,7 +411,9 @@ def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3):
       read, B = 0): the approximation the split cache avoids.
     Times are per layer (eager launches) over the first layers whose non-shared
     copies fit in max_bytes; the non-shared outputs are checked against the
-    shared ones (they differ only by the bf16 rounding of V_i)."""
+    shared ones (they differ only by the bf16 rounding of V_i).  With
+    return_outputs, also returns every arm's outputs per timed layer
+    ({"shared", "non_shared", "full_shared"}: lists of [S, N, Hq, d] tensors)."""
     lrkv, c, inp, dev = runner.lrkv, runner.cfg, runner.inp, runner.dev
     S, N, Hq, Hkv, d, r, L = c.S, c.N, c.Hq, c.Hkv, c.d, c.r, c.L
     per_layer_ns = 2 * S * N * Hkv * L * d * BF16
@@ -399,6 +427,7 @@ def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3):
     offs_ns = torch.full((S * N, 1), L, dtype=torch.int32, device=dev)
     offs_full = torch.full_like(inp.offsets, L)
     b_zero_n = torch.zeros((N, r, Hkv * d), dtype=torch.bfloat16, device=dev)
+    outs_full = [torch.empty_like(runner.outs[li]) for li in range(nl)]
     ns = []
     for li in range(nl):
         lay = inp.layers[li]
@@ -428,7 +457,7 @@ def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3):
         for li in range(nl):
             lay = inp.layers[li]
             lrkv.lrkv_attn_decode(runner.prob, lay.q, runner.kvs[li], inp.seq_lens, L, runner.uvs[li], b_zero_n,
-                                  offs_full, runner.outs[li], runner.ws)
+                                  offs_full, outs_full[li], runner.ws)
 
     seq_ns = inp.seq_lens.repeat_interleave(N)
 
@@ -450,9 +479,14 @@ def sharing_comparison(runner, max_bytes=40e9, steps=10, warmup=3):
            "cache_bytes_per_layer_shared": kv_shared, "cache_bytes_per_layer_non_shared": per_layer_ns,
            "max_abs_non_shared_vs_shared": max_abs,
            "note": "eager launches; non-shared = per-agent K and materialised V_i, B = 0; full-shared = base K/V only"}
+    arms = None
+    if return_outputs:
+        arms = {"shared": [runner.outs[li].clone() for li in range(nl)],
+                "non_shared": [ns[li][3].view(S, N, Hq, d).clone() for li in range(nl)],
+                "full_shared": outs_full}
     del ns, kv_ns
     torch.cuda.empty_cache()
-    return out
+    return (out, arms) if return_outputs else out
 
 
 def value_projection_timing(cfg, inp, prob, device, steps=20, warmup=5):
@@ -540,16 +574,63 @@ def bench_prefill(device, steps=20, warmup=5):
             "l2": "256 MB flush before each step"}
 
 
+def decode_roofline(runner, ms_step):
+    """Roofline object of the decode kernel for one timed step of `runner`."""
+    hbm, _, _, peak_src = _peaks()
+    lb = runner.layer_bytes()
+    per_launch_ms = ms_step / runner.launches_per_step
+    achieved = lb / (per_launch_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": profiled_traffic("decode_kernel", runner.cfg.name), "peak_source": f"{peak_src} copy bandwidth",
+            "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+            "kernel": "decode_kernel", "algorithmic_bytes_per_launch": lb,
+            "launch_ms": per_launch_ms, "launch_ms_note": "step time / launches per step (gaps included)"}
+
+
+def time_decode(runner, steps, warmup, sync_all, device_index):
+    """Capture the step, then W warm-up and K timed graph replays with the
+    clocks sampled throughout; returns (ms per step on this rank, clocks)."""
+    import torch.cuda.nvtx as nvtx
+    runner.capture()
+    clocks = ClockSampler(device_index)
+    clocks.start()
+    sync_all()
+    nvtx.range_push(f"decode {runner.cfg.name}")
+    ms = _timed(runner.step, steps, warmup, sync_all)
+    nvtx.range_pop()
+    return ms / steps, clocks.stop()
+
+
+def decode_sub_object(cfg, dev, steps, warmup, sync_all, device_index):
+    """One more decode workload timed like the headline, as a sub-object of the line."""
+    runner = DecodeRunner(cfg, dev)
+    ms_step, ck = time_decode(runner, steps, warmup, sync_all, device_index)
+    roof = decode_roofline(runner, ms_step)
+    out = {"workload": cfg.name, "layers": cfg.layers, "sessions": cfg.S, "agents": cfg.N, "q_heads": cfg.Hq,
+           "kv_heads": cfg.Hkv, "rank": cfg.r, "context": cfg.L,
+           "mode": "BaseShared" if cfg.mode == 0 else "BaseLRShared", "paged": cfg.paged,
+           "ms_per_step": ms_step, "queries_per_s": cfg.queries_per_step / (ms_step * 1e-3),
+           "hbm_gbs": roof["achieved"], "frac": roof["frac"], "frac_of_nominal": roof["frac_of_nominal"],
+           "algorithmic_bytes_per_launch": roof["algorithmic_bytes_per_launch"], "traffic": roof["traffic"],
+           "clocks": ck}
+    return out, runner
+
+
+SWEEP = ("cfg2", "cfg3_1k", "cfg3_2k", "cfg3_4k", "cfg3_8k")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lrkv", choices=["lrkv", "reference"])
-    ap.add_argument("--workload", default="cfg2", choices=[k for k in CONFIGS if k != "cfg4"])
+    ap.add_argument("--workload", default="cfg5", choices=[k for k in CONFIGS if k != "cfg4"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the other decode workloads (decode_workloads sub-objects)")
     ap.add_argument("--no-sharing", action="store_true",
                     help="skip the shared / non-shared / full-shared cache comparison")
     ap.add_argument("--layers", type=int, default=None,
@@ -593,25 +674,11 @@ def main():
             torch.cuda.synchronize()
 
     runner = DecodeRunner(cfg, dev, seed_offset=rank_seed_offset(rank))
-    runner.capture()
-    clocks = ClockSampler(local)
-    clocks.start()
-    sync_all()
-    ms = _timed(runner.step, args.steps, args.warmup, sync_all)
-    ck = clocks.stop()
-    ms_step = max_over_ranks(ms / args.steps, dev)
-    queries = cfg.queries_per_step * world
+    ms, ck = time_decode(runner, args.steps, args.warmup, sync_all, local)
+    ms_step = max_over_ranks(ms, dev)
     value = job_throughput(cfg.queries_per_step, world, ms_step)
-
-    hbm, _, _, peak_src = _peaks()
-    lb = runner.layer_bytes()
-    per_launch_ms = ms_step / runner.launches_per_step
-    achieved = lb / (per_launch_ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-            "traffic": profiled_traffic("decode_kernel", cfg.name), "peak_source": f"{peak_src} copy bandwidth",
-            "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
-            "kernel": "decode_kernel", "algorithmic_bytes_per_launch": lb,
-            "launch_ms": per_launch_ms, "launch_ms_note": "step time / launches per step (gaps included)"}
+    roof = decode_roofline(runner, ms_step)
+    lb = roof["algorithmic_bytes_per_launch"]
 
     e2e = None
     if not args.no_e2e:
@@ -620,17 +687,33 @@ def main():
         e2e = {"value": job_throughput(cfg.queries_per_step, world, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "ms_per_step": e_ms}
 
+    # everything below runs on one rank of a one-GPU job only: no collective follows
+    single = rank == 0 and world == 1
+    cpu = None
+    if not args.no_cpu_baseline and single:
+        cpu = cpu_baseline_decode(runner)
+    launches = runner.launches_per_step * args.steps
+    del runner
+    torch.cuda.empty_cache()
+
     prefill = None
-    if not args.no_prefill and rank == 0:
+    if not args.no_prefill and single:
         prefill = bench_prefill(dev)
 
-    sharing = None
-    if not args.no_sharing and rank == 0 and world == 1:
-        sharing = sharing_comparison(runner)
-
-    cpu = None
-    if not args.no_cpu_baseline and rank == 0 and world == 1:
-        cpu = cpu_baseline_decode(runner)
+    sweep, sharing = None, None
+    if single and not (args.no_sweep and args.no_sharing):
+        sweep = []
+        for key in SWEEP:
+            if args.no_sweep and key != "cfg2":
+                continue
+            sub, r2 = decode_sub_object(CONFIGS[key], dev, args.steps, args.warmup, sync_all, local)
+            if not args.no_sweep:
+                sweep.append(sub)
+            if key == "cfg2" and not args.no_sharing:
+                sharing = sharing_comparison(r2)
+            del r2
+            torch.cuda.empty_cache()
+        sweep = sweep or None
 
     if rank == 0:
         line = {
@@ -642,20 +725,20 @@ def main():
                        "context": cfg.L, "mode": "BaseShared" if cfg.mode == 0 else "BaseLRShared",
                        "paged": cfg.paged, "queries_per_step": cfg.queries_per_step,
                        "parallelism": f"replicas x{world} (sessions sharded, no collective)",
-                       "l2": f"inputs larger than L2: {lb * runner.launches_per_step / 1e9:.2f} GB streamed per step"},
-            "hbm_gbs": achieved,
+                       "l2": f"inputs larger than L2: {lb * cfg.layers / 1e9:.2f} GB streamed per step"},
+            "hbm_gbs": roof["achieved"],
             "roofline": roof,
             "e2e": e2e,
-            "gpu_launches": runner.launches_per_step * args.steps,
+            "gpu_launches": launches,
             "clocks": ck,
             "cpu_baseline": cpu,
+            "decode_workloads": sweep,
             "prefill": prefill,
             "sharing": sharing,
         }
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
-        del runner
         dist.destroy_process_group()
 
 
