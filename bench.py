@@ -136,6 +136,23 @@ def decode_layer_bytes(cfg, offsets_cpu):
     return kv + u + qo + b + pt
 
 
+def shard_layer_bytes(cfg, offsets_cpu, blocks):
+    """decode_layer_bytes for the (session_begin, session_count, head_begin,
+    head_count) blocks of one rank: each block reads the K/V of its heads, the
+    U rows of its sessions (U is shared by the heads, so every block that holds
+    a session reads them), its heads' q, out and B columns, and its page-table rows."""
+    N, Hq, Hkv, d, r, L = cfg.N, cfg.Hq, cfg.Hkv, cfg.d, cfg.r, cfg.L
+    G = Hq // Hkv
+    offs = np.clip(offsets_cpu.numpy().astype(np.int64), 0, L)
+    total = 0
+    for (s0, ns, g0, ng) in blocks:
+        o = offs[s0:s0 + ns]
+        u_rows = int(np.sum(L - o)) if cfg.mode == 0 else int(np.sum(L - o.min(axis=1)))
+        total += 2 * ns * ng * L * d * BF16 + u_rows * r * BF16 + 2 * ns * N * ng * G * d * BF16
+        total += N * r * ng * d * BF16 + (ns * math.ceil(L / cfg.page_size) * 4 if cfg.paged else 0)
+    return total
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -214,14 +231,45 @@ class DecodeRunner:
                 self.kvs.append(lrkv.kv_view_dense(lay.k, lay.v))
             self.uvs.append(lrkv.u_view(lay.u))
         self.graph = None
+        self.blocks = None
+
+    def set_shard(self, blocks):
+        """Serve only the given (session_begin, session_count, head_begin, head_count)
+        blocks of every layer (lrkv_attn_decode_kv_heads on views of the shard)."""
+        lrkv, c, inp = self.lrkv, self.cfg, self.inp
+        self.blocks = []
+        ws_bytes = 0
+        for (s0, ns, g0, ng) in blocks:
+            prob = lrkv.make_problem(ns, c.N, c.Hq, c.Hkv, c.d, c.r, c.mode)
+            ws_bytes = max(ws_bytes, lrkv.lrkv_decode_kv_heads_workspace_bytes(prob, ng, c.L))
+            per_layer = []
+            for lay in inp.layers:
+                if c.paged:
+                    kv = lrkv.kv_view_paged(lay.k[:, g0:g0 + ng], lay.v[:, g0:g0 + ng], lay.page_table[s0:s0 + ns])
+                else:
+                    kv = lrkv.kv_view_dense(lay.k[s0:s0 + ns, g0:g0 + ng], lay.v[s0:s0 + ns, g0:g0 + ng])
+                per_layer.append((kv, lrkv.u_view(lay.u[s0:s0 + ns])))
+            self.blocks.append((s0, ns, g0, ng, prob, per_layer))
+        self.ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=self.dev)
+        self.queries_served = c.S * c.N * sum(ns * ng for (_, ns, _, ng, _, _) in self.blocks) // (c.S * c.Hkv)
+
+    def layer(self, li, q, out, stream=None):
+        """Decode attention of layer li (this rank's blocks of it, when sharded)."""
+        lrkv, c, inp = self.lrkv, self.cfg, self.inp
+        lay = inp.layers[li]
+        if self.blocks is None:
+            lrkv.lrkv_attn_decode(self.prob, q, self.kvs[li], inp.seq_lens, c.L, self.uvs[li], lay.b,
+                                  inp.offsets, out, self.ws, stream=stream)
+            return
+        for (s0, ns, g0, ng, prob, per_layer) in self.blocks:
+            kv, uv = per_layer[li]
+            lrkv.lrkv_attn_decode_kv_heads(prob, g0, ng, q[s0:s0 + ns], kv, inp.seq_lens[s0:s0 + ns], c.L, uv,
+                                           lay.b, inp.offsets[s0:s0 + ns], out[s0:s0 + ns], self.ws,
+                                           stream=stream)
 
     def step_eager(self, qs=None, outs=None, stream=None):
-        lrkv, c, inp = self.lrkv, self.cfg, self.inp
-        for li, lay in enumerate(inp.layers):
-            q = lay.q if qs is None else qs[li]
-            out = self.outs[li] if outs is None else outs[li]
-            lrkv.lrkv_attn_decode(self.prob, q, self.kvs[li], inp.seq_lens, c.L, self.uvs[li], lay.b, inp.offsets,
-                                  out, self.ws, stream=stream)
+        for li, lay in enumerate(self.inp.layers):
+            self.layer(li, lay.q if qs is None else qs[li], self.outs[li] if outs is None else outs[li], stream)
 
     def capture(self):
         s = torch.cuda.Stream()
@@ -240,10 +288,13 @@ class DecodeRunner:
 
     @property
     def launches_per_step(self):
-        return len(self.inp.layers)
+        return len(self.inp.layers) * (1 if self.blocks is None else len(self.blocks))
 
     def layer_bytes(self):
-        return decode_layer_bytes(self.cfg, self.inp.offsets.cpu())
+        """Algorithmic bytes of one layer's launches on this rank."""
+        if self.blocks is None:
+            return decode_layer_bytes(self.cfg, self.inp.offsets.cpu())
+        return shard_layer_bytes(self.cfg, self.inp.offsets.cpu(), [b[:4] for b in self.blocks])
 
 
 # ---------------------------------------------------------------------------
@@ -253,6 +304,35 @@ class DecodeRunner:
 def rank_seed_offset(rank: int) -> int:
     """Every rank draws its own sessions: the seed moves by a prime per rank."""
     return 7919 * rank
+
+
+def kv_head_shard_plan(S: int, Hkv: int, world: int):
+    """Split one workload's (session, KV head) pairs over `world` ranks.
+
+    The pairs are taken in session-major order and rank r gets the contiguous
+    range [r U / world, (r + 1) U / world) of the U = S * Hkv pairs, written as
+    blocks (session_begin, session_count, head_begin, head_count) that one
+    lrkv_attn_decode_kv_heads call each serves (whole sessions, or a head range
+    of one session).  Every pair lands in exactly one block of one rank; the
+    ranks exchange nothing (each KV head reads only its own K/V and B columns)."""
+    U = S * Hkv
+    plan = []
+    for r in range(world):
+        lo, hi = r * U // world, (r + 1) * U // world
+        blocks = []
+        u = lo
+        while u < hi:
+            s, g = divmod(u, Hkv)
+            if g == 0 and hi - u >= Hkv:
+                n_s = (hi - u) // Hkv
+                blocks.append((s, n_s, 0, Hkv))
+                u += n_s * Hkv
+            else:
+                cnt = min(Hkv - g, hi - u)
+                blocks.append((s, 1, g, cnt))
+                u += cnt
+        plan.append(blocks)
+    return plan
 
 
 def max_over_ranks(x: float, device=None) -> float:
@@ -371,10 +451,9 @@ def run_e2e(runner, steps, warmup, sync_all):
             for li in range(nl):
                 q_dev[li].copy_(q_host[li], non_blocking=True)
                 ev_in[li].record(h2d)
-        for li, lay in enumerate(inp.layers):
+        for li in range(nl):
             comp.wait_event(ev_in[li])
-            lrkv.lrkv_attn_decode(runner.prob, q_dev[li], runner.kvs[li], inp.seq_lens, c.L, runner.uvs[li], lay.b,
-                                  inp.offsets, out_dev[li], runner.ws)
+            runner.layer(li, q_dev[li], out_dev[li])
             ev_out[li].record(comp)
         with torch.cuda.stream(d2h):
             for li in range(nl):
@@ -579,7 +658,7 @@ def decode_roofline(runner, ms_step):
     hbm, _, _, peak_src = _peaks()
     lb = runner.layer_bytes()
     per_launch_ms = ms_step / runner.launches_per_step
-    achieved = lb / (per_launch_ms * 1e-3) / 1e9
+    achieved = lb * len(runner.inp.layers) / (ms_step * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
             "traffic": profiled_traffic("decode_kernel", runner.cfg.name), "peak_source": f"{peak_src} copy bandwidth",
             "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
@@ -626,6 +705,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="lrkv", choices=["lrkv", "reference"])
     ap.add_argument("--workload", default="cfg5", choices=[k for k in CONFIGS if k != "cfg4"])
+    ap.add_argument("--partition", default="sessions", choices=["sessions", "kv-heads"],
+                    help="sessions: every rank runs the whole workload on its own sessions (weak scaling); "
+                         "kv-heads: the ranks split one workload's (session, KV head) pairs (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
@@ -673,10 +755,15 @@ def main():
         def sync_all():
             torch.cuda.synchronize()
 
-    runner = DecodeRunner(cfg, dev, seed_offset=rank_seed_offset(rank))
+    strong = args.partition == "kv-heads"
+    # weak scaling: every rank its own sessions; strong: one workload (one seed), its pairs split over the ranks
+    runner = DecodeRunner(cfg, dev, seed_offset=0 if strong else rank_seed_offset(rank))
+    if strong:
+        runner.set_shard(kv_head_shard_plan(cfg.S, cfg.Hkv, world)[rank])
     ms, ck = time_decode(runner, args.steps, args.warmup, sync_all, local)
     ms_step = max_over_ranks(ms, dev)
-    value = job_throughput(cfg.queries_per_step, world, ms_step)
+    job_queries = cfg.queries_per_step if strong else cfg.queries_per_step * world
+    value = job_queries / (ms_step * 1e-3)
     roof = decode_roofline(runner, ms_step)
     lb = roof["algorithmic_bytes_per_launch"]
 
@@ -684,7 +771,7 @@ def main():
     if not args.no_e2e:
         e_ms, hb, db = run_e2e(runner, max(10, args.steps // 10), args.warmup, sync_all)
         e_ms = max_over_ranks(e_ms, dev)
-        e2e = {"value": job_throughput(cfg.queries_per_step, world, e_ms), "unit": UNIT,
+        e2e = {"value": job_queries / (e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db, "ms_per_step": e_ms}
 
     # everything below runs on one rank of a one-GPU job only: no collective follows
@@ -718,13 +805,16 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong" if strong else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) draws of the model shapes)",
             "config": {"workload": cfg.name, "layers": cfg.layers, "sessions": cfg.S, "agents": cfg.N,
                        "q_heads": cfg.Hq, "kv_heads": cfg.Hkv, "head_dim": cfg.d, "rank": cfg.r,
                        "context": cfg.L, "mode": "BaseShared" if cfg.mode == 0 else "BaseLRShared",
                        "paged": cfg.paged, "queries_per_step": cfg.queries_per_step,
-                       "parallelism": f"replicas x{world} (sessions sharded, no collective)",
+                       "parallelism": (f"kv-head shards x{world} (one workload's (session, KV head) pairs split, "
+                                       "no collective)") if strong else
+                                      f"replicas x{world} (sessions sharded, no collective)",
                        "l2": f"inputs larger than L2: {lb * cfg.layers / 1e9:.2f} GB streamed per step"},
             "hbm_gbs": roof["achieved"],
             "roofline": roof,

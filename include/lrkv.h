@@ -211,6 +211,34 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
                              void* workspace, size_t workspace_bytes, lrkv_stream_t stream);
 
 /*
+ * Decode over a contiguous range of KV heads: the query heads h with
+ * h / G in [kv_head_begin, kv_head_begin + kv_head_count), same result for
+ * them as lrkv_attn_decode.  Every KV head's rows read only its own K/V slice
+ * and its own column slice of B_i (Eq. 12 of the LRAgent page holds per head),
+ * so the heads of a model can be split over GPUs with no exchange: each GPU
+ * holds the K/V of its heads (the paged long-context case is 30 GB of base K/V
+ * in 28 layers; the LRAgent page, Fig. 5, shows how such caches outgrow one
+ * device), its own copy of q, U and B, and writes its heads of out.
+ *   p            the whole problem (num_kv_heads = the model's Hkv)
+ *   kv           the shard: its head 0 is KV head kv_head_begin; K and V hold
+ *                kv_head_count heads (dense or paged, layout as above)
+ *   q, b, out    the whole problem's tensors ([S, N, Hq, d], [N, r, Hkv*d],
+ *                [S, N, Hq, d]); out rows of other heads are not written
+ *   workspace    >= lrkv_decode_kv_heads_workspace_bytes(p, kv_head_count, ...)
+ * Other arguments as lrkv_attn_decode.  A range outside [0, Hkv) or an empty
+ * one returns LRKV_ERR_INVALID_ARGUMENT.  The split of the keys between CTAs
+ * depends on the number of heads in the launch, so a shard's output may differ
+ * from the same heads of a whole-problem call by fp32 rounding (both are within
+ * the stated tolerance of the exact result).
+ */
+size_t lrkv_decode_kv_heads_workspace_bytes(const lrkv_problem* p, int32_t kv_head_count, int32_t max_seq_len);
+lrkv_status lrkv_attn_decode_kv_heads(const lrkv_problem* p, int32_t kv_head_begin, int32_t kv_head_count,
+                                      const void* q, const lrkv_kv_view* kv, const int32_t* seq_lens,
+                                      int32_t max_seq_len, const lrkv_u_view* u, const void* b,
+                                      const int32_t* alora_offsets, void* out, int32_t out_dtype,
+                                      void* workspace, size_t workspace_bytes, lrkv_stream_t stream);
+
+/*
  * Decode with the library's own scratch, for callers that cannot allocate
  * device memory.  The pages have no counterpart: this is a convenience of the
  * library, not part of the method.

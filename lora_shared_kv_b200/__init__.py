@@ -46,6 +46,8 @@ EXPORTS = (
     "lrkv_value_projection",
     "lrkv_decode_workspace_bytes",
     "lrkv_attn_decode",
+    "lrkv_decode_kv_heads_workspace_bytes",
+    "lrkv_attn_decode_kv_heads",
     "lrkv_attn_decode_static_scratch",
     "lrkv_query_static_scratch_status",
     "lrkv_prefill_workspace_bytes",
@@ -106,6 +108,10 @@ def lib():
         L.lrkv_decode_workspace_bytes.argtypes = [P(Problem), i32]
         L.lrkv_decode_workspace_bytes.restype = sz
         L.lrkv_attn_decode.argtypes = [P(Problem), vp, P(KVView), vp, i32, P(UView), vp, vp, vp, i32, vp, sz, vp]
+        L.lrkv_decode_kv_heads_workspace_bytes.argtypes = [P(Problem), i32, i32]
+        L.lrkv_decode_kv_heads_workspace_bytes.restype = sz
+        L.lrkv_attn_decode_kv_heads.argtypes = [P(Problem), i32, i32, vp, P(KVView), vp, i32, P(UView), vp, vp, vp,
+                                                i32, vp, sz, vp]
         L.lrkv_attn_decode_static_scratch.argtypes = [P(Problem), vp, P(KVView), vp, i32, P(UView), vp, vp, vp,
                                                       i32, vp]
         L.lrkv_prefill_workspace_bytes.argtypes = [P(Problem), i32, i32]
@@ -121,7 +127,8 @@ def lib():
         L.lrkv_last_error_detail.argtypes = []
         L.lrkv_last_error_detail.restype = ctypes.c_char_p
         L.lrkv_version.restype = i32
-        for name in ("lrkv_append_lr_cache", "lrkv_attn_decode", "lrkv_attn_decode_static_scratch",
+        for name in ("lrkv_append_lr_cache", "lrkv_attn_decode", "lrkv_attn_decode_kv_heads",
+                     "lrkv_attn_decode_static_scratch",
                      "lrkv_attn_prefill_chunk",
                      "lrkv_workspace_reset", "lrkv_query_device_status", "lrkv_query_static_scratch_status",
                      "lrkv_debug_stall_next_launch"):
@@ -262,6 +269,27 @@ def lrkv_attn_decode(problem, q, kv, seq_lens, max_seq_len, u, b, offsets, out, 
                                   int(max_seq_len), ctypes.byref(uv), _ptr(b), _ptr(offsets), _ptr(out), odt,
                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                                   _stream(stream)))
+
+
+def lrkv_decode_kv_heads_workspace_bytes(problem, kv_head_count, max_seq_len):
+    n = lib().lrkv_decode_kv_heads_workspace_bytes(ctypes.byref(problem), int(kv_head_count), int(max_seq_len))
+    if n == 0:
+        raise LrkvError(1, "invalid decode shape or KV-head count")
+    return n
+
+
+def lrkv_attn_decode_kv_heads(problem, kv_head_begin, kv_head_count, q, kv, seq_lens, max_seq_len, u, b, offsets,
+                              out, workspace, stream=None):
+    """lrkv_attn_decode for the query heads of KV heads [kv_head_begin, kv_head_begin + kv_head_count) only.
+    kv holds those KV heads (its head 0 is kv_head_begin); q, b and out are the whole problem's tensors."""
+    _require(q.is_contiguous() and b.is_contiguous() and out.is_contiguous(), "q, b and out must be contiguous")
+    _on_device(q=q, seq_lens=seq_lens, b=b, offsets=offsets, out=out, workspace=workspace)
+    odt = F32 if out.dtype == torch.float32 else BF16
+    uv = u if isinstance(u, UView) else u_view(u)
+    _check(lib().lrkv_attn_decode_kv_heads(ctypes.byref(problem), int(kv_head_begin), int(kv_head_count), _ptr(q),
+                                           ctypes.byref(kv), _ptr(seq_lens), int(max_seq_len), ctypes.byref(uv),
+                                           _ptr(b), _ptr(offsets), _ptr(out), odt, _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def lrkv_attn_decode_static_scratch(problem, q, kv, seq_lens, max_seq_len, u, b, offsets, out, stream=None):

@@ -351,7 +351,7 @@ __device__ __forceinline__ void load_q_frags(const DecodeParams& p, const Seg& s
   const __nv_bfloat16* qptr = nullptr;
   if (qvalid) {
     const int grow = sg.row_lo + qrow;
-    qptr = static_cast<const __nv_bfloat16*>(p.q) + (((size_t)sg.s * p.N + grow / p.G) * p.Hq + sg.g * p.G + grow % p.G) * D;
+    qptr = static_cast<const __nv_bfloat16*>(p.q) + (((size_t)sg.s * p.N + grow / p.G) * p.Hq + (p.g_base + sg.g) * p.G + grow % p.G) * D;
   }
 #pragma unroll
   for (int ks = 0; ks < D / 16; ++ks) {
@@ -398,7 +398,7 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
   constexpr int E4 = RP * (D + RK) / 4;
   constexpr int PERC = 6;  // float4 elements per thread per combine pass
   const float NEG_INF = -INFINITY;
-  const int HD = p.Hkv * D;
+  const int HD = p.Hkv_total * D;  // B rows span every KV head
   const int n_pairs = si.n_ag * D;
   // The B columns of this thread's first (agent, dim) pairs are requested
   // before the record is published, so that their latency overlaps the
@@ -410,7 +410,7 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
       const int e = e0 + k * NTH;
       if (e >= n_pairs) continue;
       const uint16_t* bp =
-          static_cast<const uint16_t*>(p.b) + ((size_t)(si.i_lo + e / D) * RK) * HD + (size_t)si.g * D + e % D;
+          static_cast<const uint16_t*>(p.b) + ((size_t)(si.i_lo + e / D) * RK) * HD + (size_t)(p.g_base + si.g) * D + e % D;
 #pragma unroll
       for (int r = 0; r < RK; ++r) bb[k][r] = bf16_to_f32(__ldg(bp + (size_t)r * HD));
     }
@@ -547,7 +547,7 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
         const float L = mL[row];
         const float o = L > 0.f ? acc / L : 0.f;
         const int grow = si.row_lo + row;
-        const int h = si.g * p.G + grow % p.G;
+        const int h = (p.g_base + si.g) * p.G + grow % p.G;
         const size_t oi = (((size_t)si.s * p.N + agent) * p.Hq + h) * D + dim;
         if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
         else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);

@@ -180,9 +180,12 @@ struct DecodePlan {
   size_t tickets_off, partials_off, bytes;
 };
 
-lrkv_status plan_decode(const lrkv_problem* p, int max_seq_len, const DeviceInfo& dev, DecodePlan* pl) {
+// Work partition of one decode launch over `hkv` KV heads (all of the
+// problem's, or a shard of them).
+lrkv_status plan_decode(const lrkv_problem* p, int hkv, int max_seq_len, const DeviceInfo& dev, DecodePlan* pl) {
   lrkv_status s = check_problem(p);
   if (s != LRKV_OK) return s;
+  if (hkv < 1 || hkv > p->num_kv_heads) return fail(LRKV_ERR_INVALID_ARGUMENT, "KV-head count %d of %d", hkv, p->num_kv_heads);
   if (max_seq_len < 0) return fail(LRKV_ERR_INVALID_ARGUMENT, "max_seq_len must be >= 0");
   pl->G = p->num_q_heads / p->num_kv_heads;
   pl->R = p->num_agents * pl->G;
@@ -199,7 +202,7 @@ lrkv_status plan_decode(const lrkv_problem* p, int max_seq_len, const DeviceInfo
   }
   pl->n_u_slots = p->mode == LRKV_BASE_SHARED ? max_ag : 1;
   pl->nt = max_seq_len > 0 ? (max_seq_len + lrkv::kKeysPerTile - 1) / lrkv::kKeysPerTile : 1;
-  pl->items = p->num_sessions * p->num_kv_heads * pl->n_rg;
+  pl->items = p->num_sessions * hkv * pl->n_rg;
   pl->W = (long long)pl->items * pl->nt;
   const int sms = dev.sms > 0 ? dev.sms : 148;
   pl->ctas = (int)(pl->W < sms ? pl->W : sms);
@@ -431,16 +434,25 @@ size_t lrkv_decode_workspace_bytes(const lrkv_problem* p, int32_t max_seq_len) {
     dev.smem_optin = 232448;
   }
   DecodePlan pl;
-  if (plan_decode(p, max_seq_len, dev, &pl) != LRKV_OK) return 0;
+  if (plan_decode(p, p ? p->num_kv_heads : 0, max_seq_len, dev, &pl) != LRKV_OK) return 0;
   return pl.bytes;
 }
 
-lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv, const int32_t* seq_lens,
-                             int32_t max_seq_len, const lrkv_u_view* u, const void* b,
-                             const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
-                             size_t workspace_bytes, lrkv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Decode over KV heads [g_begin, g_begin + g_count) of the problem: the K/V
+// view holds those heads only (its head 0 is head g_begin); q, out and B are
+// the whole problem's, and only the query heads of these KV heads are written.
+lrkv_status decode_heads(const lrkv_problem* p, int g_begin, int g_count, const void* q, const lrkv_kv_view* kv,
+                         const int32_t* seq_lens, int32_t max_seq_len, const lrkv_u_view* u, const void* b,
+                         const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
+                         size_t workspace_bytes, lrkv_stream_t stream) {
   lrkv_status s = check_problem(p);
   if (s != LRKV_OK) return s;
+  if (g_begin < 0 || g_count < 1 || (long long)g_begin + g_count > p->num_kv_heads)
+    return fail(LRKV_ERR_INVALID_ARGUMENT, "KV heads [%d, %d + %d) outside [0, %d)", g_begin, g_begin, g_count, p->num_kv_heads);
   if (!q || !seq_lens || !b || !out || !workspace) return fail(LRKV_ERR_INVALID_ARGUMENT, "q, seq_lens, b, out and workspace must not be NULL");
   if (!aligned16(q) || !aligned16(b) || !aligned16(out) || !aligned16(workspace)) return fail(LRKV_ERR_MISALIGNED, "q, b, out and workspace must be 16-byte aligned");
   if (out_dtype != LRKV_BF16 && out_dtype != LRKV_F32) return fail(LRKV_ERR_INVALID_ARGUMENT, "out_dtype %d", out_dtype);
@@ -449,7 +461,7 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
   DeviceInfo dev;
   if ((s = device_info(&dev)) != LRKV_OK) return s;
   DecodePlan pl;
-  if ((s = plan_decode(p, max_seq_len, dev, &pl)) != LRKV_OK) return s;
+  if ((s = plan_decode(p, g_count, max_seq_len, dev, &pl)) != LRKV_OK) return s;
   if (workspace_bytes < pl.bytes) return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", workspace_bytes, pl.bytes);
 
   const int D = p->head_dim, RK = p->rank;
@@ -457,12 +469,12 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
   alignas(64) CUtensorMap tmK, tmV, tmU;
   const uint32_t kbox[4] = {64, (uint32_t)lrkv::kKeysPerTile, 1, 1};
   if (kv->page_table) {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)kv->page_size, (uint64_t)p->num_kv_heads, (uint64_t)kv->num_pages};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)kv->page_size, (uint64_t)g_count, (uint64_t)kv->num_pages};
     const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_page};
     if ((s = make_map4(&tmK, kv->k, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "K pages")) != LRKV_OK) return s;
     if ((s = make_map4(&tmV, kv->v, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "V pages")) != LRKV_OK) return s;
   } else {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Lmap, (uint64_t)p->num_kv_heads, (uint64_t)p->num_sessions};
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Lmap, (uint64_t)g_count, (uint64_t)p->num_sessions};
     const int64_t str[3] = {kv->stride_token, kv->stride_head, kv->stride_session};
     if ((s = make_map4(&tmK, kv->k, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "K")) != LRKV_OK) return s;
     if ((s = make_map4(&tmV, kv->v, dims, str, kbox, CU_TENSOR_MAP_SWIZZLE_128B, "V")) != LRKV_OK) return s;
@@ -487,7 +499,9 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
   dp.S = p->num_sessions;
   dp.N = p->num_agents;
   dp.Hq = p->num_q_heads;
-  dp.Hkv = p->num_kv_heads;
+  dp.Hkv = g_count;
+  dp.g_base = g_begin;
+  dp.Hkv_total = p->num_kv_heads;
   dp.G = pl.G;
   dp.rows_total = pl.R;
   dp.rows_per_group = pl.rows_per_group;
@@ -531,6 +545,38 @@ lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv
   s = lrkv::launch_decode(dp, D, pl.NT, RK, &tmK, &tmV, &tmU, pl.smem, pl.ctas, stream);
   if (s != LRKV_OK) return fail(s, "decode launch failed: %s", cudaGetErrorString(cudaGetLastError()));
   return LRKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lrkv_status lrkv_attn_decode(const lrkv_problem* p, const void* q, const lrkv_kv_view* kv, const int32_t* seq_lens,
+                             int32_t max_seq_len, const lrkv_u_view* u, const void* b,
+                             const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
+                             size_t workspace_bytes, lrkv_stream_t stream) {
+  return decode_heads(p, 0, p ? p->num_kv_heads : 0, q, kv, seq_lens, max_seq_len, u, b, alora_offsets, out,
+                      out_dtype, workspace, workspace_bytes, stream);
+}
+
+size_t lrkv_decode_kv_heads_workspace_bytes(const lrkv_problem* p, int32_t kv_head_count, int32_t max_seq_len) {
+  DeviceInfo dev;
+  if (device_info(&dev) != LRKV_OK) {
+    dev.sms = 148;
+    dev.smem_optin = 232448;
+  }
+  DecodePlan pl;
+  if (plan_decode(p, kv_head_count, max_seq_len, dev, &pl) != LRKV_OK) return 0;
+  return pl.bytes;
+}
+
+lrkv_status lrkv_attn_decode_kv_heads(const lrkv_problem* p, int32_t kv_head_begin, int32_t kv_head_count,
+                                      const void* q, const lrkv_kv_view* kv, const int32_t* seq_lens,
+                                      int32_t max_seq_len, const lrkv_u_view* u, const void* b,
+                                      const int32_t* alora_offsets, void* out, int32_t out_dtype, void* workspace,
+                                      size_t workspace_bytes, lrkv_stream_t stream) {
+  return decode_heads(p, kv_head_begin, kv_head_count, q, kv, seq_lens, max_seq_len, u, b, alora_offsets, out,
+                      out_dtype, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -580,7 +626,7 @@ lrkv_status lrkv_attn_decode_static_scratch(const lrkv_problem* p, const void* q
   DeviceInfo dev;
   if ((s = device_info(&dev)) != LRKV_OK) return s;
   DecodePlan pl;
-  if ((s = plan_decode(p, max_seq_len, dev, &pl)) != LRKV_OK) return s;
+  if ((s = plan_decode(p, p->num_kv_heads, max_seq_len, dev, &pl)) != LRKV_OK) return s;
   if (pl.bytes > kStaticScratchBytes)
     return fail(LRKV_ERR_WORKSPACE_TOO_SMALL,
                 "this shape needs %zu bytes of decode scratch; the library's fixed scratch holds %zu "

@@ -37,7 +37,8 @@ struct DecodeParams {
   long long pt_stride;
   void* out;
   int out_f32;
-  int S, N, Hq, Hkv, G;
+  int S, N, Hq, Hkv, G;      // Hkv: KV heads of this launch (the K/V view's heads)
+  int g_base, Hkv_total;     // global index of the view's head 0; KV heads of the model (q, out, B)
   int rows_total;            // N * G
   int rows_per_group;        // rows of one work item (<= 32)
   int n_rg;                  // row groups per (session, KV head)

@@ -171,6 +171,25 @@ def test_decode_workspace_follows_the_stream_k_plan(S, N, Hq, Hkv, d, r, L):
     assert lrkv.lib().lrkv_decode_workspace_bytes(ctypes.byref(prob), L) == _decode_ws_expected(S, N, Hq, Hkv, d, r, L)
 
 
+def test_kv_head_range_decode_argument_errors_and_workspace():
+    L = lrkv.lib()
+    kv, uv = _views()
+    prob = _problem(S=2, N=3, Hq=12, Hkv=2)
+
+    def f(g0, ng):
+        return L.lrkv_attn_decode_kv_heads(ctypes.byref(prob), g0, ng, ctypes.c_void_p(FAKE), ctypes.byref(kv),
+                                           ctypes.c_void_p(FAKE), 8192, ctypes.byref(uv), ctypes.c_void_p(FAKE), None,
+                                           ctypes.c_void_p(FAKE), 0, ctypes.c_void_p(FAKE), 1 << 30, None)
+    for g0, ng in [(-1, 1), (0, 0), (1, 2), (2, 1), (0, 3)]:
+        assert f(g0, ng) == 1, (g0, ng)
+    # a shard's workspace is the plan of a launch over its heads only
+    for ng in (1, 2):
+        got = L.lrkv_decode_kv_heads_workspace_bytes(ctypes.byref(prob), ng, 8192)
+        assert got == _decode_ws_expected(2, 3, 12 // 2 * ng, ng, 128, 16, 8192)
+    assert L.lrkv_decode_kv_heads_workspace_bytes(ctypes.byref(prob), 3, 8192) == 0
+    assert L.lrkv_decode_kv_heads_workspace_bytes(ctypes.byref(prob), 0, 8192) == 0
+
+
 def _prefill_ws_expected(T, L0, G, Hkv, N, d, sms=148):
     # the stream-K plan, derived here independently: 128-row tiles of 128/G
     # tokens, each needing the 128-key blocks its last row sees; the blocks of
