@@ -2,8 +2,9 @@
 through the C ABI, against the fp64 oracle.
 
 Each output element is a bf16 rounding of an fp32 tensor-core sum, so it must
-sit within one bf16 half-ulp (2^-9 relative) of the exact value, plus a small
-allowance for the fp32 accumulation.  Rows outside [start_row, start_row + T),
+sit within bf16's unit roundoff (2^-8 relative: one rounding to the nearest of
+8 significand bits) of the exact value, plus a small allowance for the fp32
+accumulation.  Rows outside [start_row, start_row + T),
 other sessions and the K cache stay untouched.  Token counts and Dm that are
 not tile multiples, both sharing modes, a paged value cache and both tile
 widths (64 columns for few tiles, 128 for many) are covered."""
