@@ -580,7 +580,8 @@ def value_projection_timing(cfg, inp, prob, device, steps=20, warmup=5):
     v = torch.empty_like(inp.v)
     kv = lrkv.kv_view_dense(inp.k, v)
     u = torch.empty_like(inp.u)
-    ws = torch.zeros(256, dtype=torch.uint8, device=device)
+    ws = torch.zeros(max(256, lrkv.lrkv_value_projection_workspace_bytes(prob, cfg.T, cfg.Dm)), dtype=torch.uint8,
+                     device=device)
     rows = inp.v.shape[2]
 
     def step():

@@ -300,6 +300,7 @@ lrkv_status lrkv_value_projection(const lrkv_problem* p, const void* x, int32_t 
     return fail(LRKV_ERR_MISALIGNED, "x, w, kv->v, u and workspace must be 16-byte aligned");
   if (workspace_bytes < (size_t)lrkv::kWsHeaderBytes)
     return fail(LRKV_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %d bytes", workspace_bytes, lrkv::kWsHeaderBytes);
+  if (!aligned16(workspace)) return fail(LRKV_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   if ((kv->stride_token % 8) || (kv->stride_head % 8) || (!kv->page_table && (kv->stride_session % 8)) ||
       (kv->page_table && (kv->stride_page % 8)))
     return fail(LRKV_ERR_MISALIGNED, "kv strides must be multiples of 8 elements");
@@ -353,9 +354,30 @@ lrkv_status lrkv_value_projection(const lrkv_problem* p, const void* x, int32_t 
   vp.u_sa = u_dst->stride_agent;
   vp.u_st = u_dst->stride_token;
   vp.flags = static_cast<unsigned*>(workspace);
-  s = lrkv::launch_vproj(vp, &maps[0], &maps[1], dev.sms, stream);
+  // split K when the caller's workspace holds the partial tiles; otherwise narrow tiles
+  const lrkv::VprojPlan pl = lrkv::plan_vproj(T, ncols, Dm, dev.sms);
+  if (pl.ksplit > 1 && workspace_bytes >= pl.bytes) {
+    vp.bn = 128;
+    vp.ksplit = pl.ksplit;
+    vp.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + pl.tickets_off);
+    vp.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pl.partials_off);
+  } else {
+    const long long tiles128 = (long long)((T + 127) / 128) * ((ncols + 127) / 128);
+    vp.bn = tiles128 * 2 <= dev.sms ? 64 : 128;
+    vp.ksplit = 1;
+  }
+  s = lrkv::launch_vproj(vp, &maps[0], &maps[1], stream);
   if (s != LRKV_OK) return fail(s, "value projection launch failed: %s", cudaGetErrorString(cudaGetLastError()));
   return LRKV_OK;
+}
+
+size_t lrkv_value_projection_workspace_bytes(const lrkv_problem* p, int32_t T, int32_t Dm) {
+  if (check_problem(p) != LRKV_OK || T < 0 || Dm < 1) return 0;
+  DeviceInfo dev;
+  if (device_info(&dev) != LRKV_OK) dev.sms = 148;
+  const int n_u = p->mode == LRKV_BASE_SHARED ? p->num_agents : 1;
+  const int ncols = p->num_kv_heads * p->head_dim + n_u * p->rank;
+  return lrkv::plan_vproj(T, ncols, Dm, dev.sms).bytes;
 }
 
 lrkv_status lrkv_workspace_reset(void* workspace, size_t workspace_bytes, lrkv_stream_t stream) {
