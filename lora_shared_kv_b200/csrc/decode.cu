@@ -50,58 +50,21 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((v + 1023) & ~uintptr_t(1023));
 }
 
-// Per-segment facts every role derives from the segment's descriptor.
+// Per-segment facts both roles derive identically.
 struct Seg {
   int item, s, g, rg;
-  int lo, hi;        // key tiles [lo, hi) of this CTA on this item (visiting order)
+  int lo, hi;        // key tiles [lo, hi) of this CTA on this item, clipped to the session's length
   int sl;            // session length (clamped)
   int row_lo, rows;  // query rows [row_lo, row_lo + rows) of the N*G rows of this KV head
   int i_lo, n_ag;    // agents spanned by the rows
-  int slot, segs;    // partial-record slot; segments of the item in all
 };
 
-// Static segment at flattened static tile t of this CTA's range [.., t_end):
-// the item's tiles [lo, hi) within its first ns.  Its slot is the CTA's rank
-// among the CTAs whose static ranges meet the item; the item's segment count
-// adds its nchk dynamic chunks.
-__device__ __forceinline__ SegDesc static_desc(const DecodeParams& p, long long t, long long t_end) {
-  SegDesc d;
-  d.item = (int)(t / p.ns);
-  d.lo = (int)(t - (long long)d.item * p.ns);
-  const long long hi = t_end - (long long)d.item * p.ns;
-  d.hi = hi < p.ns ? (int)hi : p.ns;
-  const long long C = gridDim.x;
-  const long long c_first = owner_cta((long long)d.item * p.ns, p.Ws, C);
-  const long long c_last = owner_cta((long long)(d.item + 1) * p.ns - 1, p.Ws, C);
-  d.slot = (int)((long long)blockIdx.x - c_first);
-  d.segs = (int)(c_last - c_first + 1) + p.nchk;
-  return d;
-}
-
-// Dynamic chunk j (handed out item by item): tiles [ns + c cw, ns + (c + 1) cw)
-// of item j / nchk, c = j % nchk; its slot follows the item's static ones.
-__device__ __forceinline__ SegDesc dynamic_desc(const DecodeParams& p, int j) {
-  SegDesc d;
-  d.item = j / p.nchk;
-  const int c = j % p.nchk;
-  d.lo = p.ns + c * p.cw;
-  d.hi = d.lo + p.cw;
-  const long long C = gridDim.x;
-  const long long c_first = owner_cta((long long)d.item * p.ns, p.Ws, C);
-  const long long c_last = owner_cta((long long)(d.item + 1) * p.ns - 1, p.Ws, C);
-  const int n_static = (int)(c_last - c_first + 1);
-  d.slot = n_static + c;
-  d.segs = n_static + p.nchk;
-  return d;
-}
-
-__device__ __forceinline__ Seg make_seg(const DecodeParams& p, const SegDesc& d, bool flag_errors) {
+__device__ __forceinline__ Seg make_seg(const DecodeParams& p, long long t, long long t_end, bool flag_errors) {
   Seg sg;
-  sg.item = d.item;
-  sg.lo = d.lo;
-  sg.hi = d.hi;
-  sg.slot = d.slot;
-  sg.segs = d.segs;
+  sg.item = (int)(t / p.nt);
+  sg.lo = (int)(t - (long long)sg.item * p.nt);
+  long long hi = t_end - (long long)sg.item * p.nt;
+  sg.hi = hi < p.nt ? (int)hi : p.nt;
   sg.rg = sg.item % p.n_rg;
   const int sh = sg.item / p.n_rg;
   sg.g = sh % p.Hkv;
@@ -115,50 +78,6 @@ __device__ __forceinline__ Seg make_seg(const DecodeParams& p, const SegDesc& d,
   }
   sg.sl = sl;
   return sg;
-}
-
-// The segment descriptor ring in shared memory.  The producer warp writes
-// descriptor k into entry k % kDescRing and then the entry's sequence word;
-// the consumer warps and the epilogue warp read descriptors in order and
-// report how far they got, so that the producer overwrites an entry only
-// when both are done with it.
-struct DescRing {
-  SegDesc* desc;
-  volatile int* seq;
-  volatile int* progress;   // [0] consumers, [1] epilogue warp: descriptors below it are no longer read
-  SegDesc* bcast;           // [0] consumers, [1] epilogue warp: a descriptor read by one thread for its group
-};
-
-__device__ __forceinline__ DescRing desc_ring(uint8_t* smem, const DecodeSmem& lay) {
-  DescRing r;
-  r.desc = reinterpret_cast<SegDesc*>(smem + lay.desc_off);
-  r.seq = reinterpret_cast<volatile int*>(r.desc + kDescRing);
-  r.progress = r.seq + kDescRing;
-  r.bcast = reinterpret_cast<SegDesc*>(const_cast<int*>(r.progress) + 4);
-  return r;
-}
-
-// Wait (bounded) for descriptor k; false when the wait gave up or the CTA
-// aborted (the caller then treats it as the end of its segments).
-__device__ __forceinline__ bool desc_read(const DecodeParams& p, const DescRing& r, int k, SegDesc* out,
-                                          volatile int* abort_flag) {
-  uint32_t spins = 0;
-  while (r.seq[k % kDescRing] != k) {
-    if (*abort_flag) return false;
-    if (++spins >= p.spin_cap) {
-      *abort_flag = 1;
-      atomicOr(p.flags, LRKV_DEVFLAG_TIMEOUT);
-      return false;
-    }
-  }
-  __threadfence_block();
-  const volatile SegDesc* e = reinterpret_cast<const volatile SegDesc*>(r.desc + k % kDescRing);
-  out->item = e->item;
-  out->lo = e->lo;
-  out->hi = e->hi;
-  out->slot = e->slot;
-  out->segs = e->segs;
-  return true;
 }
 
 __device__ __forceinline__ void seg_rows(const DecodeParams& p, Seg& sg) {
@@ -240,8 +159,8 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t v) { return __uint_as_floa
 template <int D, int RK>
 __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                 const CUtensorMap* tmU, uint8_t* ring, int stage_bytes, uint64_t* full,
-                                uint64_t* empty, volatile int* seq, const DescRing& dr, volatile int* abort_flag,
-                                long long t_begin, long long t_end) {
+                                uint64_t* empty, volatile int* seq, volatile int* abort_flag, long long t_begin,
+                                long long t_end) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = policy_evict_first();
   const uint64_t pol_u = policy_evict_last();
@@ -251,68 +170,9 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
   uint32_t phase = 0;
   int n = 0;
   bool stop = p.stall != 0;  // the test hook: issue nothing, so the consumers' waits run out
-  long long t = t_begin;
-  // Lane 0 decides the next segment: the CTA's static range first, then
-  // dynamic chunks from the counter.  The chunk counter returns to zero for
-  // the next launch: every CTA's last take is the one that finds no chunk
-  // left, and the last of those takes (the counter then reads
-  // chunks + CTAs - 1) resets it.
-  auto next_desc = [&]() {
-    SegDesc d;
-    if (t < t_end) {
-      d = static_desc(p, t, t_end);
-      t += d.hi - d.lo;
-    } else if (p.nchk > 0) {
-      const int total = p.items * p.nchk;
-      const int j = atomicAdd(p.chunk_counter, 1);
-      if (j < total) {
-        d = dynamic_desc(p, j);
-      } else {
-        d.item = -1;
-        if (j == total + (int)gridDim.x - 1) atomicExch(p.chunk_counter, 0);
-      }
-    } else {
-      d.item = -1;
-    }
-    return d;
-  };
-  // Announce descriptor k (lane 0): wait (bounded) until the consumers and the
-  // epilogue warp are done with the entry's previous descriptor.
-  auto publish = [&](int k, const SegDesc& d) {
-    if (k >= kDescRing) {
-      uint32_t spins = 0;
-      while (dr.progress[0] < k - kDescRing + 1 || dr.progress[1] < k - kDescRing + 1) {
-        if (*abort_flag) return false;
-        if (++spins >= p.spin_cap) {
-          *abort_flag = 1;
-          atomicOr(p.flags, LRKV_DEVFLAG_TIMEOUT);
-          return false;
-        }
-      }
-    }
-    volatile SegDesc* e = reinterpret_cast<volatile SegDesc*>(dr.desc + k % kDescRing);
-    e->item = d.item;
-    e->lo = d.lo;
-    e->hi = d.hi;
-    e->slot = d.slot;
-    e->segs = d.segs;
-    __threadfence_block();
-    dr.seq[k % kDescRing] = k;
-    return true;
-  };
-  for (int segk = 0; !stop; ++segk) {
-    SegDesc d;
-    int ok = 1;
-    if (lane == 0) {
-      d = next_desc();
-      ok = publish(segk, d) ? 1 : 0;
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    d.item = __shfl_sync(0xffffffffu, d.item, 0);
-    d.lo = __shfl_sync(0xffffffffu, d.lo, 0);
-    d.hi = __shfl_sync(0xffffffffu, d.hi, 0);
-    if (!ok || d.item < 0) break;
-    Seg sg = make_seg(p, d, false);
+  for (long long t = t_begin; t < t_end && !stop;) {
+    Seg sg = make_seg(p, t, t_end, false);
+    t += sg.hi - sg.lo;
     seg_rows(p, sg);
     const int nts = seg_tiles_valid(sg);
     // lane j < n_ag holds the offset of agent i_lo + j
@@ -503,11 +363,11 @@ __device__ __forceinline__ void load_q_frags(const DecodeParams& p, const Seg& s
 // Facts of one segment's merged record, enough to publish or finish it.
 struct SegInfo {
   int item, s, g, row_lo, rows, i_lo, n_ag;
-  int segs;  // segments of the item (static shares and dynamic chunks)
-  int slot;  // this segment's partial-record slot among them
+  int segs;  // CTAs sharing the item
+  int slot;  // this CTA's partial-record slot among them
 };
 
-__device__ __forceinline__ SegInfo seg_info(const Seg& sg) {
+__device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Seg& sg) {
   SegInfo si;
   si.item = sg.item;
   si.s = sg.s;
@@ -516,8 +376,11 @@ __device__ __forceinline__ SegInfo seg_info(const Seg& sg) {
   si.rows = sg.rows;
   si.i_lo = sg.i_lo;
   si.n_ag = sg.n_ag;
-  si.segs = sg.segs;
-  si.slot = sg.slot;
+  const long long C = gridDim.x;
+  const long long c_first = owner_cta((long long)sg.item * p.nt, p.W, C);
+  const long long c_last = owner_cta((long long)(sg.item + 1) * p.nt - 1, p.W, C);
+  si.segs = (int)(c_last - c_first + 1);
+  si.slot = (int)((long long)blockIdx.x - c_first);
   return si;
 }
 
@@ -630,25 +493,36 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
           }
           sync();
         }
-        for (int jj = 0; jj < nj; ++jj) {
-          const float4* rj = reinterpret_cast<const float4*>(base + (size_t)(j0 + jj) * REC + 2 * RP);
-          float4 v[PERC];
+        // records in groups of RG, the loads of a group issued together (one
+        // round trip to L2 per group instead of one per record); the sums run
+        // in record order either way
+        constexpr int RG = NT >= 4 ? 2 : 4;  // the 32-row instance has the fewest registers to spare
+        for (int jg = 0; jg < nj; jg += RG) {
+          float4 v[RG][PERC];
 #pragma unroll
-          for (int u = 0; u < PERC; ++u) {
-            const int e4 = e0 + tid + u * NTH;
-            v[u] = e4 < E4 ? __ldcg(rj + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int q = 0; q < RG; ++q) {
+            const float4* rj = reinterpret_cast<const float4*>(base + (size_t)(j0 + jg + q) * REC + 2 * RP);
+#pragma unroll
+            for (int u = 0; u < PERC; ++u) {
+              const int e4 = e0 + tid + u * NTH;
+              v[q][u] = (jg + q < nj && e4 < E4) ? __ldcg(rj + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
           }
 #pragma unroll
-          for (int u = 0; u < PERC; ++u) {
-            const int e4 = e0 + tid + u * NTH;
-            if (e4 >= E4) continue;
-            const int e = e4 * 4;
-            const int row = e < RP * D ? e / D : (e - RP * D) / RK;
-            const float sc = scw[jj * RP + row];
-            acc[u].x += v[u].x * sc;
-            acc[u].y += v[u].y * sc;
-            acc[u].z += v[u].z * sc;
-            acc[u].w += v[u].w * sc;
+          for (int q = 0; q < RG; ++q) {
+            if (jg + q >= nj) break;
+#pragma unroll
+            for (int u = 0; u < PERC; ++u) {
+              const int e4 = e0 + tid + u * NTH;
+              if (e4 >= E4) continue;
+              const int e = e4 * 4;
+              const int row = e < RP * D ? e / D : (e - RP * D) / RK;
+              const float sc = scw[(jg + q) * RP + row];
+              acc[u].x += v[q][u].x * sc;
+              acc[u].y += v[q][u].y * sc;
+              acc[u].z += v[q][u].z * sc;
+              acc[u].w += v[q][u].w * sc;
+            }
           }
         }
         if (!one_chunk) sync();  // the next chunk rewrites the scale table
@@ -695,8 +569,8 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
 
 template <int D, int NT, int RK>
 __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const DecodeSmem& lay, uint64_t* full,
-                                 uint64_t* empty, volatile int* seq, const DescRing& dr, volatile int* abort_flag,
-                                 int* bcast) {
+                                 uint64_t* empty, volatile int* seq, volatile int* abort_flag, int* bcast,
+                                 long long t_begin, long long t_end) {
   constexpr int RP = NT * 8;
   constexpr int KS = D / 16;
   constexpr int MT = D / 16;
@@ -737,18 +611,9 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   }
 
   uint32_t qf[KS][2];
-  // Descriptors are read by thread 0 and handed to the group through shared
-  // memory, so that every consumer thread takes the same path (named barriers).
-  volatile int* rec_last = dr.progress + 2;
-  if (tid == 0) {
-    SegDesc d;
-    if (!desc_read(p, dr, 0, &d, abort_flag)) d.item = -1;
-    dr.bcast[0] = d;
-  }
-  named_bar_sync(1, CT);
-  SegDesc nxt = dr.bcast[0];
-  for (int segk = 0; nxt.item >= 0; ++segk) {
-    Seg sg = make_seg(p, nxt, tid == 0);
+  for (long long t = t_begin; t < t_end;) {
+    Seg sg = make_seg(p, t, t_end, tid == 0);
+    t += sg.hi - sg.lo;
     seg_rows(p, sg);
     const int nts = seg_tiles_valid(sg);
     const int sl = sg.sl;
@@ -1000,22 +865,13 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     // formed here rather than kept live through the tile loop, and the last
     // segment's B columns are loaded inside the finish rather than held in
     // registers across the merge: the tile loop needs every register.
-    // the next descriptor decides whether this segment is the CTA's last
-    if (tid == 0) {
-      SegDesc d;
-      if (!desc_read(p, dr, segk + 1, &d, abort_flag)) d.item = -1;
-      dr.bcast[0] = d;
-    }
-    named_bar_sync(1, CT);
-    nxt = dr.bcast[0];
-    if (tid == 0) dr.progress[0] = segk + 2;  // both descriptors are in registers now
-    const bool last_seg = nxt.item < 0;
+    const bool last_seg = t >= t_end;
     const int buf = sn & 1;
     float* merge = reinterpret_cast<float*>(smem + lay.merge_off) + buf * REC;  // records alternate
     uint64_t* rec_full = full + 2 * p.stages;
     uint64_t* rec_free = rec_full + 2;
     if (!last_seg) {
-      Seg nx = make_seg(p, nxt, false);
+      Seg nx = make_seg(p, t, t_end, false);
       seg_rows(p, nx);
       load_q_frags<D>(p, nx, rbase + g8, t4, qf);
     }
@@ -1039,20 +895,16 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     }
     if (og == 0) store_rows<D, RK>(st, merge, RP, rbase, g8, t4);
     named_bar_sync(1, CT);
-    // hand the record to the epilogue warp and go on streaming; the last one
-    // only tells the epilogue warp to stop: the consumers finish it themselves
-    if (tid == 0) {
-      rec_last[buf] = last_seg ? 1 : 0;
-      mbar_arrive(&rec_full[buf]);
-    }
-    if (last_seg) {
-      const SegInfo si = seg_info(sg);
+    if (!last_seg) {
+      // hand the record to the epilogue warp and go on streaming
+      if (tid == 0) mbar_arrive(&rec_full[buf]);
+    } else {
+      const SegInfo si = seg_info(p, sg);
       float* scw = reinterpret_cast<float*>(smem + lay.scw_off);  // the consumers' half
       finish_segment<D, NT, RK, CT, (RK >= 32 ? 2 : 4)>(p, si, merge, scw, bcast, tid, [] { named_bar_sync(1, CT); });
     }
     ++sn;
   }
-  if (tid == 0) dr.progress[0] = 0x7fffffff;
 }
 
 // The epilogue warp: publishes (and, as the last CTA of an item, combines and
@@ -1060,45 +912,28 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
 // consumer warps stream the next segment's tiles.
 template <int D, int NT, int RK>
 __device__ void decode_epilogue(const DecodeParams& p, uint8_t* smem, const DecodeSmem& lay, uint64_t* rec_full,
-                                uint64_t* rec_free, const DescRing& dr, volatile int* abort_flag, int* bcast) {
+                                uint64_t* rec_free, volatile int* abort_flag, int* bcast, long long t_begin,
+                                long long t_end) {
   constexpr int RP = NT * 8;
   constexpr int REC = RP * (D + RK + 2);
   const int lane = threadIdx.x & 31;
   float* merge0 = reinterpret_cast<float*>(smem + lay.merge_off);
   float* scw = reinterpret_cast<float*>(smem + lay.scw_off) + 8 * RP;  // the epilogue warp's half
-  volatile int* rec_last = dr.progress + 2;
-  for (int sn = 0;; ++sn) {
+  int sn = 0;
+  for (long long t = t_begin; t < t_end;) {
+    Seg sg = make_seg(p, t, t_end, false);
+    t += sg.hi - sg.lo;
+    seg_rows(p, sg);
+    if (t >= t_end) break;  // the consumers finish the last segment
     const int buf = sn & 1;
     if (!mbar_wait_bounded(&rec_full[buf], (sn >> 1) & 1, abort_flag, p.flags, p.spin_cap)) break;
-    if (rec_last[buf]) break;  // the consumers finish the CTA's last segment
-    int item = -1, lo = 0, hi = 0, slot = 0, segs = 0;
-    if (lane == 0) {
-      SegDesc d;
-      if (desc_read(p, dr, sn, &d, abort_flag)) {
-        item = d.item;
-        lo = d.lo;
-        hi = d.hi;
-        slot = d.slot;
-        segs = d.segs;
-      }
-      dr.progress[1] = sn + 1;
-    }
-    SegDesc d;
-    d.item = __shfl_sync(0xffffffffu, item, 0);
-    d.lo = __shfl_sync(0xffffffffu, lo, 0);
-    d.hi = __shfl_sync(0xffffffffu, hi, 0);
-    d.slot = __shfl_sync(0xffffffffu, slot, 0);
-    d.segs = __shfl_sync(0xffffffffu, segs, 0);
-    if (d.item < 0) break;
-    Seg sg = make_seg(p, d, false);
-    seg_rows(p, sg);
-    const SegInfo si = seg_info(sg);
+    const SegInfo si = seg_info(p, sg);
     finish_segment<D, NT, RK, 32, (RK >= 32 ? 1 : 2)>(p, si, merge0 + buf * REC, scw, bcast, lane,
                                                       [] { __syncwarp(); });
     __syncwarp();
     if (lane == 0) mbar_arrive(&rec_free[buf]);
+    ++sn;
   }
-  if (lane == 0) dr.progress[1] = 0x7fffffff;
 }
 
 // Warp roles: warps 0 .. decode_groups(NT)*NT-1 consume, then one producer warp
@@ -1123,7 +958,6 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
   volatile int* seq = reinterpret_cast<volatile int*>(rec_free + 2);
   volatile int* abort_flag = seq + p.stages;
   int* bcast = const_cast<int*>(abort_flag) + 1;  // [0] consumers, [1] epilogue warp
-  const DescRing dr = desc_ring(smem, lay);
   const int warp = threadIdx.x >> 5;
   constexpr int PRODUCER = Roles<NT>::CONSUMER_WARPS;
   constexpr int EPILOGUE = PRODUCER + 1;
@@ -1139,9 +973,6 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
     }
     *abort_flag = 0;
     bcast[0] = bcast[1] = 0;
-    for (int e = 0; e < kDescRing; ++e) dr.seq[e] = -1;
-    dr.progress[0] = dr.progress[1] = 0;
-    dr.progress[2] = dr.progress[3] = 0;  // the last-record flags
     fence_barrier_init();
   }
   if (warp == PRODUCER && (threadIdx.x & 31) == 0) {
@@ -1153,16 +984,15 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
   pdl_wait();
   pdl_launch_dependents();
   const long long C = gridDim.x;
-  // this CTA's share of the statically split tiles (the first ns of every item)
-  const long long t_begin = (long long)blockIdx.x * p.Ws / C;
-  const long long t_end = (long long)(blockIdx.x + 1) * p.Ws / C;
+  const long long t_begin = (long long)blockIdx.x * p.W / C;
+  const long long t_end = (long long)(blockIdx.x + 1) * p.W / C;
   if (warp == PRODUCER) {
-    decode_producer<D, RK>(p, &tmK, &tmV, &tmU, smem, lay.stage_bytes, full, empty, seq, dr, abort_flag, t_begin,
+    decode_producer<D, RK>(p, &tmK, &tmV, &tmU, smem, lay.stage_bytes, full, empty, seq, abort_flag, t_begin,
                            t_end);
   } else if (warp == EPILOGUE) {
-    decode_epilogue<D, NT, RK>(p, smem, lay, rec_full, rec_free, dr, abort_flag, bcast + 1);
+    decode_epilogue<D, NT, RK>(p, smem, lay, rec_full, rec_free, abort_flag, bcast + 1, t_begin, t_end);
   } else {
-    decode_consumers<D, NT, RK>(p, smem, lay, full, empty, seq, dr, abort_flag, bcast);
+    decode_consumers<D, NT, RK>(p, smem, lay, full, empty, seq, abort_flag, bcast, t_begin, t_end);
   }
 }
 

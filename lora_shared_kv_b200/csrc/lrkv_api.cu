@@ -176,32 +176,9 @@ lrkv_status check_u(const lrkv_u_view* u, const lrkv_problem* p, int rows_needed
 // ---------------------------------------------------------------------------
 struct DecodePlan {
   int G, R, n_rg, rows_per_group, NT, n_u_slots, nt, items, ctas, max_segs, stages, smem;
-  int ns, nchk, cw;  // static tiles per item; dynamic chunks per item and their tiles
-  long long W, Ws;
+  long long W;
   size_t tickets_off, partials_off, bytes;
 };
-
-// The decode work split.  Every item (session, KV head, row group) has nt key
-// tiles in its visiting order.  The first ns of them are split evenly over
-// the CTAs (stream-K); the last nt - ns form nchk chunks of cw tiles that the
-// CTAs take from a counter as they run out of work, so that CTAs whose share
-// took longer (uneven HBM service, more low-rank tiles, a merge to finish)
-// take fewer.  Chunks are kTileRun tiles; an item keeps about an eighth of its
-// tiles for them, at most 8 chunks (one merge round); with fewer than four
-// tiles per CTA, or items shorter than two chunks, everything is static.
-void plan_decode_split(DecodePlan* pl, int sms) {
-  pl->ns = pl->nt;
-  pl->nchk = 0;
-  pl->cw = lrkv::kTileRun;
-  if (pl->W >= 4LL * sms && pl->nt >= 2 * lrkv::kTileRun) {
-    const int td_raw = (pl->nt + 7) / 8;
-    int nchk = (td_raw + lrkv::kTileRun - 1) / lrkv::kTileRun;
-    nchk = nchk < 1 ? 1 : (nchk > 8 ? 8 : nchk);
-    pl->nchk = nchk;
-    pl->ns = pl->nt - nchk * pl->cw;
-  }
-  pl->Ws = (long long)pl->items * pl->ns;
-}
 
 // Work partition of one decode launch over `hkv` KV heads (all of the
 // problem's, or a shard of them).
@@ -228,14 +205,12 @@ lrkv_status plan_decode(const lrkv_problem* p, int hkv, int max_seq_len, const D
   pl->items = p->num_sessions * hkv * pl->n_rg;
   pl->W = (long long)pl->items * pl->nt;
   const int sms = dev.sms > 0 ? dev.sms : 148;
-  plan_decode_split(pl, sms);
-  pl->ctas = (int)(pl->Ws < sms ? pl->Ws : sms);
-  // partial records per item: one per CTA whose static range meets it, one per dynamic chunk
+  pl->ctas = (int)(pl->W < sms ? pl->W : sms);
   int ms = 1;
   for (int it = 0; it < pl->items; ++it) {
-    const long long cf = lrkv::owner_cta((long long)it * pl->ns, pl->Ws, pl->ctas);
-    const long long cl = lrkv::owner_cta((long long)(it + 1) * pl->ns - 1, pl->Ws, pl->ctas);
-    const int n = (int)(cl - cf + 1) + pl->nchk;
+    const long long cf = lrkv::owner_cta((long long)it * pl->nt, pl->W, pl->ctas);
+    const long long cl = lrkv::owner_cta((long long)(it + 1) * pl->nt - 1, pl->W, pl->ctas);
+    const int n = (int)(cl - cf + 1);
     ms = n > ms ? n : ms;
   }
   pl->max_segs = ms;
@@ -580,10 +555,7 @@ lrkv_status decode_heads(const lrkv_problem* p, int g_begin, int g_count, const 
     dp.tile_stride = stride;
   }
   dp.items = pl.items;
-  dp.ns = pl.ns;
-  dp.nchk = pl.nchk;
-  dp.cw = pl.cw;
-  dp.Ws = pl.Ws;
+  dp.W = pl.W;
   dp.max_segs = pl.max_segs;
   dp.stages = pl.stages;
   dp.scale_log2 = scale_of(p) * 1.4426950408889634f;
@@ -591,7 +563,6 @@ lrkv_status decode_heads(const lrkv_problem* p, int g_begin, int g_count, const 
   dp.flags = reinterpret_cast<unsigned*>(ws);
   dp.tickets = reinterpret_cast<int*>(ws + pl.tickets_off);
   dp.partials = reinterpret_cast<float*>(ws + pl.partials_off);
-  dp.chunk_counter = reinterpret_cast<int*>(ws + lrkv::kChunkCounterOffset);
   take_stall_hook(&dp.spin_cap, &dp.stall);
   s = lrkv::launch_decode(dp, D, pl.NT, RK, &tmK, &tmV, &tmU, pl.smem, pl.ctas, stream);
   if (s != LRKV_OK) return fail(s, "decode launch failed: %s", cudaGetErrorString(cudaGetLastError()));

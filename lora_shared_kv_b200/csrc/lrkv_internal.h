@@ -51,13 +51,7 @@ struct DecodeParams {
   int nt;                    // key tiles per work item
   int tile_stride;           // runs of kTileRun tiles of an item are visited in the order (j * tile_stride) mod runs
   int items;                 // S * Hkv * n_rg
-  // Work split: the first ns tiles of every item (in visiting order) are
-  // split evenly over the CTAs (stream-K over the items * ns flattened
-  // tiles, Ws); the last nt - ns form nchk chunks of cw tiles per item that
-  // CTAs take, as they run out of work, from a counter in the workspace.
-  int ns, nchk, cw;
-  long long Ws;
-  int* chunk_counter;        // chunks handed out so far; zero between launches
+  long long W;               // items * nt (flattened tile count)
   int max_segs;              // partial slots per item
   int stages;
   float scale_log2;          // softmax_scale * log2(e)
@@ -79,19 +73,8 @@ __host__ __device__ constexpr int decode_groups(int NT) { return NT <= 2 ? 3 : 2
 
 // Shared-memory plan of the decode kernel (bytes from a 1024-aligned base).
 struct DecodeSmem {
-  int stage_bytes, ring_bytes, merge_off, scw_off, a_off, desc_off, bar_off, total;
+  int stage_bytes, ring_bytes, merge_off, scw_off, a_off, bar_off, total;
 };
-
-// A CTA's segments (its share of one item's tiles) as the producer warp
-// announces them to the other roles, in a ring of kDescRing entries.
-struct SegDesc {
-  int item;        // -1: no more segments
-  int lo, hi;      // tiles [lo, hi) of the item, in visiting order
-  int slot;        // partial-record slot of this segment
-  int segs;        // segments of the item in all (the merge ticket's target)
-};
-constexpr int kDescRing = 16;
-constexpr int kChunkCounterOffset = 64;  // byte offset of the chunk counter in the workspace header
 
 __host__ __device__ inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
@@ -104,10 +87,7 @@ __host__ __device__ inline DecodeSmem decode_smem_plan(int D, int NT, int RK, in
   const int rec = RP * (D + RK + 2) * 4;
   s.scw_off = s.merge_off + 2 * rec;      // two records: segments alternate
   s.a_off = s.scw_off + 2 * 8 * RP * 4;   // scale tables of the consumers and of the epilogue warp
-  // segment descriptor ring, its sequence words, the consumers' and the epilogue's
-  // progress, and one broadcast descriptor each for the consumers and the epilogue
-  s.desc_off = round_up(s.a_off + kMaxAgents * 4, 16);
-  s.bar_off = round_up(s.desc_off + kDescRing * (int)sizeof(SegDesc) + kDescRing * 4 + 16 + 2 * (int)sizeof(SegDesc), 16);
+  s.bar_off = round_up(s.a_off + kMaxAgents * 4, 16);
   s.total = s.bar_off + (2 * stages + 4) * 8 + stages * 4 + 64;
   return s;
 }

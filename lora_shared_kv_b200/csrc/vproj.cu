@@ -199,29 +199,34 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
       tmem_ld32(tmem + lane_addr + c * 32, r);
       tmem_wait_ld();
       if (!ok || t >= p.T) continue;
-      if (add_parts) {  // sum of the parts 0, 1, ... in order (this CTA's own from its registers)
-        float sum[32];
-        const float* base = p.partials + (size_t)tile * p.ksplit * VP_BM * VP_BN + (size_t)row * VP_BN + c * 32;
-#pragma unroll 1
-        for (int z = 0; z < p.ksplit; ++z) {
+      if (add_parts) {
+        // the parts of these 32 columns (this CTA's own included, as stored), all
+        // loads in one round, then added in part order 0, 1, ...
+        const float4* base = reinterpret_cast<const float4*>(
+            p.partials + (size_t)tile * p.ksplit * VP_BM * VP_BN + (size_t)row * VP_BN + c * 32);
+        float4 v[4][8];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float4 v;
-            if (z == (int)blockIdx.z) {
-              v = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
-                              __uint_as_float(r[e + 3]));
-            } else {
-              v = __ldcg(reinterpret_cast<const float4*>(base + (size_t)z * VP_BM * VP_BN + e));
-            }
-            if (z == 0) {
-              sum[e] = v.x; sum[e + 1] = v.y; sum[e + 2] = v.z; sum[e + 3] = v.w;
-            } else {
-              sum[e] += v.x; sum[e + 1] += v.y; sum[e + 2] += v.z; sum[e + 3] += v.w;
+        for (int z = 0; z < 4; ++z)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            v[z][e] = z < p.ksplit ? __ldcg(base + (size_t)z * (VP_BM * VP_BN / 4) + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float4 acc = v[0][e];
+#pragma unroll
+          for (int z = 1; z < 4; ++z) {
+            if (z < p.ksplit) {
+              acc.x += v[z][e].x;
+              acc.y += v[z][e].y;
+              acc.z += v[z][e].z;
+              acc.w += v[z][e].w;
             }
           }
+          r[4 * e] = __float_as_uint(acc.x);
+          r[4 * e + 1] = __float_as_uint(acc.y);
+          r[4 * e + 2] = __float_as_uint(acc.z);
+          r[4 * e + 3] = __float_as_uint(acc.w);
         }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(sum[e]);
       }
       uint32_t pk[16];
 #pragma unroll

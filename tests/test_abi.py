@@ -134,37 +134,24 @@ def test_workspace_bytes_shape_rules():
     assert n >= 256
 
 
-def decode_split(nt, items, sms=148):
-    """The decode work split, derived here independently: (ns, nchk) = static
-    tiles per item and dynamic 4-tile chunks per item.  About an eighth of an
-    item's tiles (at most 8 chunks) go to the dynamic chunks, when there are at
-    least four tiles per SM and an item has at least 8 tiles."""
-    if items * nt >= 4 * sms and nt >= 8:
-        nchk = min(8, max(1, -(-(-(-nt // 8)) // 4)))
-        return nt - 4 * nchk, nchk
-    return nt, 0
-
-
 def _decode_ws_expected(S, N, Hq, Hkv, d, r, L, sms=148):
     # the decode plan, derived here independently: the N*G rows of a KV head
     # in as few groups of at most 32 as cover them, each padded to a multiple
     # of 8; work items (session, KV head, row group) of ceil(L/64) key tiles;
-    # the first ns tiles of every item split evenly over min(static tiles, SMs)
-    # CTAs, CTA c taking [c W / C, (c + 1) W / C) of the flattened static
-    # tiles; one partial record per CTA that touches an item plus one per
-    # dynamic chunk, when that makes more than one
+    # the flattened tiles split evenly over min(tiles, SMs) CTAs, CTA c taking
+    # [c W / C, (c + 1) W / C); one partial record per CTA that touches an
+    # item, when more than one does
     R = N * (Hq // Hkv)
     n_rg = -(-R // 32)
     NT = -(-(-(-R // n_rg)) // 8)
     nt = max(1, -(-L // 64))
     items = S * Hkv * n_rg
-    ns, nchk = decode_split(nt, items, sms)
-    W = items * ns
+    W = items * nt
     C = min(W, sms)
-    touching = [nchk] * items
+    touching = [0] * items
     for c in range(C):
         lo, hi = c * W // C, (c + 1) * W // C
-        for it in range(lo // ns, (hi - 1) // ns + 1):
+        for it in range(lo // nt, (hi - 1) // nt + 1):
             touching[it] += 1
     segs = max(touching)
     partials_off = 256 + -(-(4 * items) // 256) * 256

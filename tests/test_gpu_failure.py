@@ -31,7 +31,7 @@ def _decode_case(seed, S=3, N=3, Hq=12, Hkv=2, d=128, r=16, L=3000):
     u = _normal((S, N, L, r), 1.0, g, DEV)
     b = _normal((N, r, Hkv * d), 0.05, g, DEV)
     offs = torch.tensor([[0, 1000, 2500]] * S, dtype=torch.int32, device=DEV)
-    seq = torch.tensor([L, L - 5, 1500][:S], dtype=torch.int32, device=DEV)
+    seq = torch.tensor([L, L - 5, L // 2][:S], dtype=torch.int32, device=DEV)
     return q, k, v, u, b, offs, seq
 
 

@@ -206,37 +206,3 @@ def test_prefill_two_o_ready_barriers_order_every_read_of_o():
 def test_prefill_one_o_ready_barrier_can_pass_on_an_old_phase():
     bad = sum(1 for nb in range(3, 8) for seed in range(150) if prefill_handshake(nb, False, seed))
     assert bad > 0
-
-
-def chunk_counter(ctas, chunks, seed):
-    """The decode kernel's dynamic chunks: every CTA takes chunks from one
-    counter (an atomic add) until it gets an index past the last chunk, then
-    stops; the take that returns chunks + ctas - 1 (the last of the failing
-    takes, one per CTA) puts the counter back to zero for the next launch.
-    Returns (chunks handed out per index, final counter, resets seen)."""
-    rnd = random.Random(seed)
-    counter = 0
-    got = [0] * chunks
-    resets = 0
-    active = list(range(ctas))
-    while active:
-        c = rnd.choice(active)
-        j = counter
-        counter += 1                  # atomicAdd
-        if j < chunks:
-            got[j] += 1
-            continue
-        active.remove(c)              # no chunk left: this CTA is done taking
-        if j == chunks + ctas - 1:
-            counter = 0               # atomicExch(counter, 0)
-            resets += 1
-    return got, counter, resets
-
-
-def test_chunk_counter_hands_out_each_chunk_once_and_returns_to_zero():
-    for seed in range(300):
-        rnd = random.Random(seed)
-        ctas, chunks = rnd.randint(1, 20), rnd.randint(0, 60)
-        got, counter, resets = chunk_counter(ctas, chunks, seed)
-        assert got == [1] * chunks
-        assert counter == 0 and resets == 1

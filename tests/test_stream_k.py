@@ -61,60 +61,21 @@ def _check_cover(sizes, C, max_parts):
     assert len(seen) == sum(sizes)
 
 
-def _decode_split(nt, items, sms=148):
-    # about an eighth of an item's tiles (at most 8 chunks of 4) are handed out
-    # dynamically, when there are at least 4 tiles per SM and 8 per item
-    if items * nt >= 4 * sms and nt >= 8:
-        nchk = min(8, max(1, -(-(-(-nt // 8)) // 4)))
-        return nt - 4 * nchk, nchk
-    return nt, 0
-
-
 @pytest.mark.parametrize("S,N,Hq,Hkv,L", [(32, 3, 12, 2, 8192), (16, 2, 16, 8, 1024), (1, 3, 12, 2, 4097),
-                                          (1, 5, 8, 1, 300), (4, 8, 16, 8, 65536 // 16), (4, 8, 16, 8, 65536),
-                                          (16, 2, 16, 8, 2048), (200, 1, 4, 4, 64), (3, 2, 4, 2, 512)])
+                                          (1, 5, 8, 1, 300), (4, 8, 16, 8, 65536 // 16)])
 def test_decode_items_split_over_the_ctas(S, N, Hq, Hkv, L):
-    """Static shares by stream-K over the first ns tiles of every item, then
-    nchk dynamic chunks of 4 tiles per item, handed out item by item: every
-    tile of every item is covered exactly once, and the record slots (static
-    shares first, then one per chunk) stay below the item's segment count and
-    the workspace's bound."""
     R = N * (Hq // Hkv)
     n_rg = -(-R // 32)
     nt = -(-L // 64)
     items = S * Hkv * n_rg
-    ns, nchk = _decode_split(nt, items)
-    assert ns >= 1 and ns + 4 * nchk == nt
-    W = items * ns
+    W = items * nt
     C = min(W, 148)
+    # the workspace holds, per item, as many records as the most CTAs any item touches
     touching = [0] * items
     for lo, hi in ranges(W, C):
-        for it in range(lo // ns, (hi - 1) // ns + 1):
+        for it in range(lo // nt, (hi - 1) // nt + 1):
             touching[it] += 1
-    max_segs = max(t + nchk for t in touching)
-    # the static shares
-    _check_cover([ns] * items, C, max(touching))
-    seen = set()
-    slots = {}
-    for c, it, lo, hi, parts, slot in _walk([ns] * items, C):
-        for u in range(lo, hi):
-            seen.add((it, u))
-        slots.setdefault(it, set()).add(slot)
-        assert parts + nchk == touching[it] + nchk <= max_segs
-    # the dynamic chunks, in the order the counter hands them out
-    for j in range(items * nchk):
-        it, ch = divmod(j, nchk)
-        lo, hi = ns + 4 * ch, ns + 4 * ch + 4
-        for u in range(lo, hi):
-            assert (it, u) not in seen
-            seen.add((it, u))
-        slot = touching[it] + ch
-        assert slot not in slots.setdefault(it, set())
-        slots[it].add(slot)
-        assert slot < touching[it] + nchk <= max_segs
-    assert seen == {(it, u) for it in range(items) for u in range(nt)}
-    for it in range(items):  # the ticket counts every segment of the item once
-        assert slots[it] == set(range(touching[it] + nchk))
+    _check_cover([nt] * items, C, max(touching))
 
 
 @pytest.mark.parametrize("T,L0,G,Hkv,N", [(512, 16384, 2, 8, 4), (100, 300, 2, 2, 2), (1, 77, 2, 4, 2),
