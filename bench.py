@@ -580,8 +580,7 @@ def value_projection_timing(cfg, inp, prob, device, steps=20, warmup=5):
     v = torch.empty_like(inp.v)
     kv = lrkv.kv_view_dense(inp.k, v)
     u = torch.empty_like(inp.u)
-    ws = torch.zeros(max(256, lrkv.lrkv_value_projection_workspace_bytes(prob, cfg.T, cfg.Dm)), dtype=torch.uint8,
-                     device=device)
+    ws = torch.zeros(256, dtype=torch.uint8, device=device)
     rows = inp.v.shape[2]
 
     def step():
@@ -618,27 +617,38 @@ def bench_prefill(device, steps=20, warmup=5):
     ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=device)
     out = torch.empty((cfg.N, cfg.T, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=device)
 
-    def step():
+    def append():
         lrkv.lrkv_append_lr_cache(inp.x, inp.a_down, inp.u, session=0, start_row=cfg.L0, uview=uv)
+
+    def chunk():
         lrkv.lrkv_attn_prefill_chunk(prob, inp.q, kv, 0, cfg.L0, cfg.T, uv, inp.b, inp.offsets, out, ws)
+
+    def step():
+        append()
+        chunk()
 
     try:
         step()
     except Exception as e:  # noqa: BLE001
         return {"status": f"unavailable: {e}"}
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
-    times = []
-    for i in range(warmup + steps):
-        flush.zero_()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        step()
-        e1.record()
-        e1.synchronize()
-        if i >= warmup:
-            times.append(e0.elapsed_time(e1))
-    ms = statistics.median(times)
+
+    def median_ms(fn):
+        times = []
+        for i in range(warmup + steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            if i >= warmup:
+                times.append(e0.elapsed_time(e1))
+        return statistics.median(times)
+
+    ms = median_ms(step)
+    append_ms, chunk_ms = median_ms(append), median_ms(chunk)
     vproj = value_projection_timing(cfg, inp, prob, device)
     keys = cfg.T * cfg.L0 + cfg.T * (cfg.T + 1) // 2
     rows = cfg.N * cfg.Hq
@@ -646,7 +656,11 @@ def bench_prefill(device, steps=20, warmup=5):
     flops += 2.0 * cfg.N * cfg.T * cfg.Dm * cfg.r
     _, bf16_peak, _, src = _peaks()
     tf = flops / (ms * 1e-3) / 1e12
+    chunk_flops = flops - 2.0 * cfg.N * cfg.T * cfg.Dm * cfg.r
     return {"workload": cfg.name, "ms_per_step": ms, "tflops": tf, "flops_per_step": flops,
+            "append_ms": append_ms, "chunk_ms": chunk_ms,
+            "chunk_tflops": chunk_flops / (chunk_ms * 1e-3) / 1e12,
+            "chunk_frac": chunk_flops / (chunk_ms * 1e-3) / 1e12 / bf16_peak,
             "peak_tflops": bf16_peak, "frac": tf / bf16_peak, "peak_source": src,
             "nominal_peak_tflops": NOMINAL_BF16_TFLOPS, "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS,
             "prefill_kernel_traffic": profiled_traffic("prefill_kernel", cfg.name),

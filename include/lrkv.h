@@ -328,14 +328,6 @@ lrkv_status lrkv_attn_prefill_chunk(const lrkv_problem* p, const void* q, const 
 /* ---------------------------------------------------------------------- */
 
 /*
- * Bytes of workspace with which lrkv_value_projection splits its K loop over
- * several CTAs per output tile (few tiles: the fp32 partial tiles are added by
- * the last CTA of each tile, in part order); 0 if the shape is invalid.  With
- * a smaller workspace (at least 256 bytes) the call runs without the split.
- */
-size_t lrkv_value_projection_workspace_bytes(const lrkv_problem* p, int32_t T, int32_t Dm);
-
-/*
  * [V_base | U_1 ... U_n] = X [W0_v | A_1 ... A_n] for T new tokens, written
  * into the caches: base value rows start_row .. start_row+T-1 of session
  * `session` for every KV head (kv->v; kv->k is not touched), and the same rows
@@ -348,11 +340,7 @@ size_t lrkv_value_projection_workspace_bytes(const lrkv_problem* p, int32_t T, i
  *            n_u = N in BaseShared, 1 in BaseLRShared
  *   kv       dense: kv_rows is the row capacity of each (session, head);
  *            paged: rows map through the session's page-table row
- *   workspace  device, 16-byte aligned, >= 256 bytes, zero-filled once:
- *            status flags; with lrkv_value_projection_workspace_bytes bytes
- *            also the split-K tickets and partial tiles (the tickets return to
- *            zero by the end of every call; calls sharing a workspace must be
- *            ordered on one stream)
+ *   workspace  device, >= 256 bytes, zero-filled once: status flags
  * Numerics: bf16 inputs, fp32 accumulation on the tensor cores in an
  * unspecified order, round to nearest even bf16.  The U rows are therefore not
  * bit-identical to lrkv_append_lr_cache's fixed-order ones.

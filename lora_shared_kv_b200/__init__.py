@@ -44,7 +44,6 @@ EXPORTS = (
     "lrkv_append_lr_cache",
     "lrkv_append_lr_cache_ranges",
     "lrkv_value_projection",
-    "lrkv_value_projection_workspace_bytes",
     "lrkv_decode_workspace_bytes",
     "lrkv_attn_decode",
     "lrkv_decode_kv_heads_workspace_bytes",
@@ -106,8 +105,6 @@ def lib():
         L.lrkv_append_lr_cache_ranges.argtypes = [vp, i32, vp, i32, i32, i32, P(i32), P(i32), P(UView), i32, vp]
         L.lrkv_value_projection.argtypes = [P(Problem), vp, i32, i32, vp, P(KVView), i32, P(UView), i32, i32, vp, sz,
                                             vp]
-        L.lrkv_value_projection_workspace_bytes.argtypes = [P(Problem), i32, i32]
-        L.lrkv_value_projection_workspace_bytes.restype = sz
         L.lrkv_decode_workspace_bytes.argtypes = [P(Problem), i32]
         L.lrkv_decode_workspace_bytes.restype = sz
         L.lrkv_attn_decode.argtypes = [P(Problem), vp, P(KVView), vp, i32, P(UView), vp, vp, vp, i32, vp, sz, vp]
@@ -253,11 +250,6 @@ def lrkv_value_projection(problem, x, w, kv, kv_rows, u, session, start_row, wor
     _check(lib().lrkv_value_projection(ctypes.byref(problem), _ptr(x), T, Dm, _ptr(w), ctypes.byref(kv), int(kv_rows),
                                        ctypes.byref(uv), session, start_row, _ptr(workspace),
                                        workspace.numel() * workspace.element_size(), _stream(stream)))
-
-
-def lrkv_value_projection_workspace_bytes(problem, T, Dm):
-    """Workspace bytes with which lrkv_value_projection splits its K loop (256 bytes suffice without)."""
-    return lib().lrkv_value_projection_workspace_bytes(ctypes.byref(problem), int(T), int(Dm))
 
 
 def lrkv_decode_workspace_bytes(problem, max_seq_len):

@@ -147,14 +147,15 @@ void launch_generic(const void* x, const void* a, const AppendRows& rows, int n,
 // Fast path (Dm a multiple of 8, x and a 16-byte aligned): a warp owns 32
 // tokens (one per lane) x 4 columns, so a lane runs 4 fmaf chains and a block
 // of 4 warps covers 32 tokens x 16 columns (64 x 8 when r = 8).  X and A
-// k-chunks stream through a 4-stage cp.async ring, so three chunks are in
-// flight while one is consumed; a lane reads 8 k of its token's X row with one
-// 128-bit load (rows padded to 144 B: conflict-free) and each k's 4 A values
-// (converted to fp32 once per chunk) with one broadcast load.
+// k-chunks of 128 stream through a cp.async ring deep enough (12 stages, 6 for
+// 64-token blocks) that the whole of a 2048-wide hidden state is requested at
+// the start: the chunks' global latency overlaps the chains instead of
+// stalling them.  A lane reads 8 k of its token's X row with one 128-bit load
+// (rows padded to 272 B: conflict-free) and each k's 4 A values (converted to
+// fp32 once per chunk) with one broadcast load.
 // ---------------------------------------------------------------------------
-constexpr int F_NS = 4;   // ring stages
-constexpr int F_KC = 64;  // k per chunk
-constexpr int F_XP = F_KC + 8;  // X row pitch in bf16 (144 B)
+constexpr int F_KC = 128;       // k per chunk
+constexpr int F_XP = F_KC + 8;  // X row pitch in bf16 (272 B)
 
 template <int R>
 struct FastShape {
@@ -163,9 +164,13 @@ struct FastShape {
   static constexpr int TB = 32 * TGB;                 // tokens per block
   static constexpr int CB = 4 * CGB;                  // columns per block
   static constexpr int NCB = R / CB;                  // column blocks
+  static constexpr int NS = TB == 32 ? 12 : 6;        // ring stages
   static constexpr int XCP = TB * (F_KC / 8);         // 16-byte X copies per chunk
   static constexpr int ACP = F_KC * CB / 8;           // 16-byte A copies per chunk
-  static_assert(XCP % APP_THREADS == 0 && ACP <= APP_THREADS && (F_KC * CB) % APP_THREADS == 0, "shape");
+  static constexpr int X_STAGE = TB * F_XP;           // bf16 elements
+  static constexpr int A_STAGE = F_KC * CB;           // bf16 elements
+  static constexpr int SMEM = NS * (X_STAGE + A_STAGE) * 2 + F_KC * CB * 4;
+  static_assert(XCP % APP_THREADS == 0 && ACP % APP_THREADS == 0 && (F_KC * CB) % APP_THREADS == 0, "shape");
 };
 
 template <int R>
@@ -173,9 +178,11 @@ __global__ void __launch_bounds__(APP_THREADS)
     append_kernel_fast(const uint16_t* __restrict__ x, const uint16_t* __restrict__ a, const AppendRows rows, int Dm,
                        __nv_bfloat16* __restrict__ u, long long u_ss, long long u_sa, long long u_st, int session) {
   using S = FastShape<R>;
-  __shared__ __align__(16) uint16_t xr[F_NS][S::TB * F_XP];
-  __shared__ __align__(16) uint16_t ar[F_NS][F_KC * S::CB];
-  __shared__ __align__(16) float af[F_KC * S::CB];
+  constexpr int NS = S::NS;
+  extern __shared__ __align__(16) uint8_t app_smem[];
+  uint16_t* xr = reinterpret_cast<uint16_t*>(app_smem);            // [NS][TB * F_XP]
+  uint16_t* ar = xr + NS * S::X_STAGE;                             // [NS][F_KC * CB]
+  float* af = reinterpret_cast<float*>(ar + NS * S::A_STAGE);      // [F_KC * CB]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cg = warp % S::CGB;
   const int tl = (warp / S::CGB) * 32 + lane;  // token within the block
@@ -189,41 +196,43 @@ __global__ void __launch_bounds__(APP_THREADS)
 
   auto issue = [&](int c) {
     if (c < n_chunks) {
-      const int k0 = c * F_KC, st = c % F_NS;
+      const int k0 = c * F_KC, st = c % NS;
 #pragma unroll
       for (int i = 0; i < S::XCP / APP_THREADS; ++i) {
         const int e = tid + i * APP_THREADS;
         const int row = e / (F_KC / 8), seg = e % (F_KC / 8);
         const bool ok = t0 + row < T && k0 + seg * 8 < Dm;
         const uint16_t* src = ok ? x + (size_t)(t0 + row) * Dm + k0 + seg * 8 : x;
-        cp_async16(&xr[st][row * F_XP + seg * 8], src, ok ? 16u : 0u);
+        cp_async16(&xr[st * S::X_STAGE + row * F_XP + seg * 8], src, ok ? 16u : 0u);
       }
-      if (tid < S::ACP) {
-        const int row = tid / (S::CB / 8), seg = tid % (S::CB / 8);
+#pragma unroll
+      for (int i = 0; i < S::ACP / APP_THREADS; ++i) {
+        const int e = tid + i * APP_THREADS;
+        const int row = e / (S::CB / 8), seg = e % (S::CB / 8);
         const bool ok = k0 + row < Dm;
         const uint16_t* src = ok ? a_ag + (size_t)(k0 + row) * R + c0 + seg * 8 : a_ag;
-        cp_async16(&ar[st][row * S::CB + seg * 8], src, ok ? 16u : 0u);
+        cp_async16(&ar[st * S::A_STAGE + row * S::CB + seg * 8], src, ok ? 16u : 0u);
       }
     }
     cp_async_commit();  // one group per chunk index, empty past the end
   };
 
   float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
-#pragma unroll
-  for (int c = 0; c < F_NS - 1; ++c) issue(c);
+#pragma unroll 1
+  for (int c = 0; c < NS - 1; ++c) issue(c);
   for (int c = 0; c < n_chunks; ++c) {
-    cp_async_wait<F_NS - 2>();  // this thread's copies of chunk c have landed
-    __syncthreads();            // everyone's; and chunk c - 1 is no longer read
-    const int st = c % F_NS;
+    cp_async_wait<NS - 2>();  // this thread's copies of chunk c have landed
+    __syncthreads();          // everyone's; and chunk c - 1 is no longer read
+    const int st = c % NS;
 #pragma unroll
     for (int i = 0; i < F_KC * S::CB / APP_THREADS; ++i) {
       const int e = tid + i * APP_THREADS;
-      af[e] = __uint_as_float((uint32_t)ar[st][e] << 16);
+      af[e] = __uint_as_float((uint32_t)ar[st * S::A_STAGE + e] << 16);
     }
     __syncthreads();
-    issue(c + F_NS - 1);  // into the stage chunk c - 1 used
+    issue(c + NS - 1);  // into the stage chunk c - 1 used
     const int kc = min(F_KC, Dm - c * F_KC);  // a multiple of 8
-    const uint4* xrow = reinterpret_cast<const uint4*>(&xr[st][tl * F_XP]);
+    const uint4* xrow = reinterpret_cast<const uint4*>(&xr[st * S::X_STAGE + tl * F_XP]);
     const float4* acol = reinterpret_cast<const float4*>(af) + cg;
     for (int k8 = 0; k8 < kc / 8; ++k8) {
       const uint4 xv = xrow[k8];
@@ -260,10 +269,12 @@ void launch_r(const void* x, const void* a, const AppendRows& rows, int n, int m
     return;
   }
   using S = FastShape<R>;
+  if (ensure_dynamic_smem<append_kernel_fast<R>>(S::SMEM) != cudaSuccess) return;  // reported by the caller's check
   dim3 grid((max_len + S::TB - 1) / S::TB, n, S::NCB);
-  append_kernel_fast<R><<<grid, APP_THREADS, 0, stream>>>(static_cast<const uint16_t*>(x),
-                                                          static_cast<const uint16_t*>(a), rows, Dm,
-                                                          static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st, session);
+  append_kernel_fast<R><<<grid, APP_THREADS, S::SMEM, stream>>>(static_cast<const uint16_t*>(x),
+                                                                 static_cast<const uint16_t*>(a), rows, Dm,
+                                                                 static_cast<__nv_bfloat16*>(u), u_ss, u_sa, u_st,
+                                                                 session);
 }
 
 }  // namespace

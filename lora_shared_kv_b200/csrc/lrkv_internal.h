@@ -112,19 +112,7 @@ struct VprojParams {
   uint16_t* u;                       // low-rank caches (bf16)
   long long u_ss, u_sa, u_st;
   unsigned* flags;                   // device status word
-  // split of the K loop over ksplit CTAs per output tile (1: none); the last
-  // CTA of a tile (ticket) adds the others' fp32 partial tiles in part order
-  int ksplit, bn;
-  int* tickets;                      // [tiles], zero between launches
-  float* partials;                   // [tiles][ksplit][128 rows][bn]
 };
-
-// Split-K plan of a value projection and its workspace.
-struct VprojPlan {
-  int bn, tiles, ksplit;
-  size_t tickets_off, partials_off, bytes;
-};
-VprojPlan plan_vproj(int T, int ncols, int Dm, int sms);
 
 // ---------------------------------------------------------------------------
 // launchers (defined in the kernel translation units)
@@ -135,7 +123,7 @@ lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, const vo
                           const void* tmU, int smem_bytes, int ctas, void* stream);
 int decode_max_smem_optin();
 int vproj_smem_bytes();
-lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, void* stream);
+lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, int sms, void* stream);
 
 lrkv_status launch_append(const void* x, const void* a, int n_a, const int* row_begin, const int* row_end,
                           int u_shift, int Dm, int r, void* u, long long u_ss, long long u_sa, long long u_st,

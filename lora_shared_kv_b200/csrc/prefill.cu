@@ -19,17 +19,16 @@
 // there (atomic ticket), which merges the others' partial (m, l, O + Z B) rows.
 // Roles:
 //   warp 0        TMA producer: B_i,g of each tile segment (double buffer),
-//                 then its 128-key blocks of K into a 2-stage ring (a stage
+//                 then its 128-key blocks of K into a 3-stage ring (a stage
 //                 frees as soon as its S is computed).
-//   warp 2        TMA producer of the V and U blocks (3-stage ring: a stage
-//                 frees only when its PV is done, and its loads take longest).
+//   warp 2        TMA producer of the V and U blocks (2-stage ring).
 //   warp 1        TMEM owner and MMA issuer (one thread): S_j = Q K_j^T with
 //                 the Q tile read from TMEM, into a double-buffered S; then
-//                 [O | Z] += P_j [V_j | U_j] with P_j read from TMEM (it
-//                 overwrites S_j): V_j and U_j lie side by side in shared
-//                 memory as one operand, so a k-step is one MMA of N = d + r,
-//                 and one more of N = r against a constant block whose column
-//                 0 is one gives the row sums l of exactly the bf16 weights.  U rows
+//                 [O | Z | l] += P_j [V_j | U_j | 1] with P_j read from TMEM
+//                 (it overwrites S_j).  V_j, U_j and a constant block whose
+//                 column 0 is one lie side by side in shared memory as one
+//                 operand, so a k-step is one MMA of N = d + r + 16 and the row
+//                 sums l of exactly the bf16 weights come out with O.  U rows
 //                 before the aLoRA offset are zero-filled (the U of blocks
 //                 wholly before it is not loaded).  At the end of a segment it
 //                 adds Z B_i,g to O with two more MMA pairs (Z split into bf16
@@ -56,8 +55,8 @@ namespace {
 
 constexpr int BM = 128;   // rows per tile (TMEM lanes)
 constexpr int BN = 128;   // keys per block
-constexpr int KST = 2;    // K ring: a stage is free once S = Q K^T has been computed
-constexpr int VST = 3;    // V/U ring: a stage is free once the PV MMA is done (its loads take longest)
+constexpr int KST = 3;    // K ring: a stage is free once S = Q K^T has been computed
+constexpr int VST = 2;    // V/U ring: a stage is free once the PV MMA is done
 constexpr int THREADS = 384;      // K producer, MMA, V/U producer, idle, 2 softmax warpgroups
 constexpr int SMX_THREADS = 256;  // the two softmax warpgroups (named barrier 1); the two warps of
                                   // one 32-row lane quarter pair up on named barriers 2..5
@@ -68,23 +67,22 @@ struct PrefillLayout {
   static constexpr int B_BYTES = RK * D * 2;
   static constexpr int K_BYTES = BN * D * 2;
   static constexpr int U_BYTES = BN * RK * 2;
-  // V block (D / RK atoms) then the U block of one stage; one constant atom
-  // (column 0 is 1) shared by all stages gives the row sums of P as one more
-  // MMA of N = RK beside O and Z
-  static constexpr int V_STAGE = K_BYTES + U_BYTES;
+  // V block (D / RK atoms), the U block, then a constant atom whose column 0
+  // is 1, so that the row sums of P come out of the same MMA as O and Z
+  static constexpr int V_STAGE = K_BYTES + 2 * U_BYTES;
   static constexpr int U_OFF = K_BYTES;
+  static constexpr int ONES_OFF = K_BYTES + U_BYTES;
   static constexpr int B_OFF = 0;  // two B buffers: segments alternate
   static constexpr int K_OFF = (B_OFF + 2 * B_BYTES + 1023) / 1024 * 1024;
   static constexpr int V_OFF = K_OFF + KST * K_BYTES;
-  static constexpr int ONES_OFF = V_OFF + VST * V_STAGE;
-  static constexpr int BAR_OFF = ONES_OFF + U_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VST * V_STAGE;
   static constexpr int XCH_OFF = BAR_OFF + 256;  // row max [2 blocks][2 halves][BM], then a ticket word
   static constexpr int TOTAL = XCH_OFF + 4 * BM * 4 + 16;
-  // TMEM columns: S double buffer; then [O | Z], the accumulator of P [V | U],
-  // and the RK columns of P [ones] (column 0 is the row sum l)
+  // TMEM columns: S double buffer; then [O | Z | L], the accumulator of
+  // P [V | U | ones] (column 0 of the 16 L columns is the row sum l)
   static constexpr uint32_t COL_S0 = 0, COL_S1 = BN, COL_O = 2 * BN, COL_Z = 2 * BN + D, COL_L = 2 * BN + D + RK;
   static constexpr uint32_t COL_Q = 448;  // the Q tile, bf16 pairs: the A operand of S = Q K^T
-  static_assert(2 * BN + D + 2 * RK <= (int)COL_Q && COL_Q + D / 2 <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * BN + D + RK + 16 <= (int)COL_Q && COL_Q + D / 2 <= TMEM_COLS, "TMEM budget");
   static_assert(K_BYTES % 1024 == 0 && V_STAGE % 1024 == 0, "stage alignment");
   static constexpr int REC = BM * (D + 2);  // floats of a partial record: m, l, O + Z B per row
 };
@@ -328,10 +326,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
-    // Over the CTA's blocks n = 0, 1, ...: S_n, then [O | Z] += P_{n-1} [V | U] and l += P_{n-1} 1.
+    // Over the CTA's blocks n = 0, 1, ...: S_n, then [O | Z | l] += P_{n-1} [V | U | 1].
     constexpr uint32_t ID_QK = umma_idesc_bf16(BM, BN, 0, 0);
-    constexpr uint32_t ID_PVU = umma_idesc_bf16(BM, D + RK, 0, 1);  // [O | Z] += P [V | U]
-    constexpr uint32_t ID_ONE = umma_idesc_bf16(BM, RK, 0, 1);      // l (column 0) += P [1]
+    constexpr uint32_t ID_PVU = umma_idesc_bf16(BM, D + RK + 16, 0, 1);  // [O | Z | l] += P [V | U | 1]
     constexpr uint32_t VU_LAYOUT = RK == 32 ? 4u : 6u;  // 64B / 32B swizzle: atoms of RK bf16 per key row
     constexpr uint32_t VU_LBO = Lay::U_BYTES;           // next atom along d + r
     constexpr uint32_t VU_SBO = 8 * RK * 2;             // next eight key rows
@@ -360,15 +357,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) {
         tc_fence_after();
         const uint32_t v_base = smem_u32(smem + Lay::V_OFF + st * Lay::V_STAGE);
-        const uint32_t ones_base = smem_u32(smem + Lay::ONES_OFF);
         const uint32_t a_p = tmem + (pv_n & 1 ? Lay::COL_S1 : Lay::COL_S0);
         // the segment's first block overwrites O, Z and l
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t b = umma_desc(v_base + kk * (16 * RK * 2), VU_LBO, VU_SBO, VU_LAYOUT);
           umma_ts(tmem + Lay::COL_O, a_p + kk * 8, b, ID_PVU, (!pv_first || kk > 0) ? 1u : 0u);
-          const uint64_t b1 = umma_desc(ones_base + kk * (16 * RK * 2), VU_LBO, VU_SBO, VU_LAYOUT);
-          umma_ts(tmem + Lay::COL_L, a_p + kk * 8, b1, ID_ONE, (!pv_first || kk > 0) ? 1u : 0u);
         }
         umma_commit(&bars->v_empty[st]);
         umma_commit(&bars->o_ready[pv_n & 1]);
@@ -471,14 +465,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
 
     if (wg == 1) {
-      // the constant atom: logical column 0 of each key row is bf16 1.0.  Its
-      // rows use the RK-wide swizzle of V and U: 16-byte chunk c of row r sits
-      // at chunk c ^ (r >> 1) & 3 (64-byte rows) or c ^ (r >> 2) & 1 (32-byte rows).
+      // the constant atom of every V stage: logical column 0 of each key row is
+      // bf16 1.0.  Its rows use the RK-wide swizzle of V and U: 16-byte chunk c
+      // of row r sits at chunk c ^ (r >> 1) & 3 (64-byte rows) or c ^ (r >> 2) & 1
+      // (32-byte rows).
       constexpr int CPR = RK / 8;  // 16-byte chunks per row
-      for (int q = row; q < BN * CPR; q += BM) {
-        const int r = q / CPR, pc = q % CPR;
+      for (int q = row; q < VST * BN * CPR; q += BM) {
+        const int stg = q / (BN * CPR), r = (q / CPR) % BN, pc = q % CPR;
         const int swz = RK == 32 ? (r >> 1) & 3 : (r >> 2) & 1;
-        uint4* dst = reinterpret_cast<uint4*>(smem + Lay::ONES_OFF) + r * CPR + pc;
+        uint4* dst = reinterpret_cast<uint4*>(smem + Lay::V_OFF + stg * Lay::V_STAGE + Lay::ONES_OFF) + r * CPR + pc;
         *dst = make_uint4((pc ^ swz) == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();  // the tensor core reads it through the async proxy

@@ -6,12 +6,10 @@
 // projection as X W0 + (X A_i) B_i; both parts read the same hidden states, so
 // one GEMM produces the shared base values and every U_i row at once.
 //
-// A tcgen05 GEMM: one CTA per 128-token x BN-column tile and K part (BN = 128;
-// when the tiles would leave more than half of the SMs idle, the K loop is
-// split over up to 4 CTAs whose fp32 partial tiles the last of them adds in
-// part order, or, without room for the partials, BN = 64), K in 64-wide steps
-// through a TMA ring of 6 or 8 stages (X K-major, W column-major atoms, both
-// 128B swizzled), fp32 accumulation in TMEM, and an epilogue that converts to bf16
+// A tcgen05 GEMM: one CTA per 128-token x BN-column tile (BN = 128, or 64 when
+// 128-wide tiles would leave SMs idle), K in 64-wide steps through a TMA ring
+// of 6 or 8 stages (X K-major, W column-major atoms, both 128B swizzled), fp32
+// accumulation in TMEM, and an epilogue that converts to bf16
 // and scatters each row's columns to its cache: column c < Hkv d goes to KV
 // head c / d of the base value cache, the rest to agent slot (c - Hkv d) / r.
 // The summation order inside the tensor core is not specified, so U rows made
@@ -43,7 +41,6 @@ struct VpBars {
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
-  int last_flag;  // this CTA adds the parts of its tile (split K)
 };
 
 template <int BN>
@@ -61,10 +58,7 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * VP_BM;  // first token
   const int n0 = blockIdx.y * VP_BN;  // first output column
-  const int nk_all = (p.Dm + VP_BK - 1) / VP_BK;
-  // this CTA's share of the K loop: part blockIdx.z of ksplit
-  const int k_lo = (int)((long long)blockIdx.z * nk_all / p.ksplit);
-  const int nk = (int)((long long)(blockIdx.z + 1) * nk_all / p.ksplit) - k_lo;
+  const int nk = (p.Dm + VP_BK - 1) / VP_BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < VP_ST; ++s) {
@@ -102,11 +96,10 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
         uint8_t* xs = smem + st * VP_STAGE;
         uint8_t* ws = xs + VP_X_BYTES;
         mbar_arrive_expect_tx(&bars->full[st], VP_STAGE);
-        const int kg = (k_lo + kt) * VP_BK;  // global k of this step
-        tma_load_4d(xs, &tmX, &bars->full[st], kg, m0, 0, 0, pol);
+        tma_load_4d(xs, &tmX, &bars->full[st], kt * VP_BK, m0, 0, 0, pol);
 #pragma unroll
         for (int at = 0; at < BN / 64; ++at)
-          tma_load_4d(ws + at * (VP_BK * 128), &tmW, &bars->full[st], n0 + at * 64, kg, 0, 0, pol);
+          tma_load_4d(ws + at * (VP_BK * 128), &tmW, &bars->full[st], n0 + at * 64, kt * VP_BK, 0, 0, pol);
       }
       if (*abort_flag) {
         for (int kt = issued > VP_ST ? issued - VP_ST : 0; kt < issued; ++kt) {
@@ -143,39 +136,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
     // ---- epilogue: one token row per thread (TMEM lane), bf16 into the caches
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-    bool ok = mbar_wait_bounded(&bars->acc_full, 0, abort_flag, p.flags);
+    const bool ok = mbar_wait_bounded(&bars->acc_full, 0, abort_flag, p.flags);
     tc_fence_after();
-    // With the K loop split over ksplit CTAs, each publishes its fp32 partial
-    // tile and the last to arrive (atomic ticket) adds them in part order.
-    const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-    volatile int* last_flag = &bars->last_flag;
-    bool add_parts = false;
-    if (p.ksplit > 1) {
-      float* mine = p.partials + ((size_t)tile * p.ksplit + blockIdx.z) * VP_BM * VP_BN + (size_t)row * VP_BN;
-#pragma unroll 1
-      for (int c = 0; c < VP_BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          __stcg(reinterpret_cast<float4*>(mine + c * 32 + e),
-                 make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
-                             __uint_as_float(r[e + 3])));
-      }
-      __threadfence();
-      named_bar_sync(1, 128);
-      if (threadIdx.x == 128) {
-        const int prev = atomicAdd(p.tickets + tile, 1);
-        const int last = prev == p.ksplit - 1;
-        if (last) p.tickets[tile] = 0;
-        *last_flag = last;
-      }
-      named_bar_sync(1, 128);
-      if (!*last_flag) ok = false;  // another CTA finishes this tile
-      add_parts = true;
-      __threadfence();
-    }
     const int t = m0 + row;
     const int pos = p.start_row + t;  // cache row
     const int hd = p.Hkv * p.d;
@@ -199,35 +161,6 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
       tmem_ld32(tmem + lane_addr + c * 32, r);
       tmem_wait_ld();
       if (!ok || t >= p.T) continue;
-      if (add_parts) {
-        // the parts of these 32 columns (this CTA's own included, as stored), all
-        // loads in one round, then added in part order 0, 1, ...
-        const float4* base = reinterpret_cast<const float4*>(
-            p.partials + (size_t)tile * p.ksplit * VP_BM * VP_BN + (size_t)row * VP_BN + c * 32);
-        float4 v[4][8];
-#pragma unroll
-        for (int z = 0; z < 4; ++z)
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            v[z][e] = z < p.ksplit ? __ldcg(base + (size_t)z * (VP_BM * VP_BN / 4) + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float4 acc = v[0][e];
-#pragma unroll
-          for (int z = 1; z < 4; ++z) {
-            if (z < p.ksplit) {
-              acc.x += v[z][e].x;
-              acc.y += v[z][e].y;
-              acc.z += v[z][e].z;
-              acc.w += v[z][e].w;
-            }
-          }
-          r[4 * e] = __float_as_uint(acc.x);
-          r[4 * e + 1] = __float_as_uint(acc.y);
-          r[4 * e + 2] = __float_as_uint(acc.z);
-          r[4 * e + 3] = __float_as_uint(acc.w);
-        }
-      }
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
@@ -263,40 +196,18 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
 
 int vproj_smem_bytes() { return VpShape<128>::SMEM + 1024; }
 
-// Output tiles of 128 tokens x bn columns.  When 128-wide tiles would leave
-// more than half of the SMs idle, the K loop is split over up to 4 CTAs per
-// tile (ksplit) when the caller's workspace holds the partial tiles, else the
-// tiles narrow to 64 columns.
-VprojPlan plan_vproj(int T, int ncols, int Dm, int sms) {
-  VprojPlan pl = {};
-  const int mt = (T + VP_BM - 1) / VP_BM;
-  const long long tiles128 = (long long)mt * ((ncols + 127) / 128);
-  const int nk = (Dm + VP_BK - 1) / VP_BK;
-  pl.bn = 128;
-  pl.tiles = (int)tiles128;
-  pl.ksplit = 1;
-  if (tiles128 > 0 && tiles128 * 2 <= sms) {
-    long long ks = sms / tiles128;
-    ks = ks > 4 ? 4 : ks;
-    ks = ks > nk / 2 ? nk / 2 : ks;  // at least two K steps per part
-    pl.ksplit = ks < 1 ? 1 : (int)ks;
-  }
-  pl.tickets_off = kWsHeaderBytes;
-  pl.partials_off = (pl.tickets_off + (size_t)pl.tiles * 4 + 255) / 256 * 256;
-  pl.bytes = pl.ksplit > 1 ? pl.partials_off + (size_t)pl.tiles * pl.ksplit * VP_BM * 128 * 4 : kWsHeaderBytes;
-  return pl;
-}
-
-lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, void* stream) {
-  const int bn = p.bn;
-  const bool narrow = bn == 64;
+lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, int sms, void* stream) {
+  // 128-wide tiles, unless they would leave more than half of the SMs idle
+  const long long tiles128 = (long long)((p.T + VP_BM - 1) / VP_BM) * ((p.ncols + 127) / 128);
+  const bool narrow = tiles128 * 2 <= sms;
+  const int bn = narrow ? 64 : 128;
   const int smem = (narrow ? VpShape<64>::SMEM : VpShape<128>::SMEM) + 1024;
   auto kern = narrow ? vproj_kernel<64> : vproj_kernel<128>;
   if ((narrow ? ensure_dynamic_smem<vproj_kernel<64>>(smem) : ensure_dynamic_smem<vproj_kernel<128>>(smem)) !=
       cudaSuccess)
     return LRKV_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.T + VP_BM - 1) / VP_BM, (p.ncols + bn - 1) / bn, p.ksplit);
+  cfg.gridDim = dim3((p.T + VP_BM - 1) / VP_BM, (p.ncols + bn - 1) / bn);
   cfg.blockDim = dim3(VP_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);

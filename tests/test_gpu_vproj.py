@@ -7,10 +7,7 @@ sit within bf16's unit roundoff (2^-8 relative: one rounding to the nearest of
 accumulation.  Rows outside [start_row, start_row + T),
 other sessions and the K cache stay untouched.  Token counts and Dm that are
 not tile multiples, both sharing modes, a paged value cache and both tile
-widths (64 columns for few tiles, 128 for many) are covered, each with a
-256-byte workspace (no split) and with the queried workspace (few tiles split
-their K loop over several CTAs, the last adding the parts), the latter twice
-in a row on the same workspace."""
+widths (64 columns for few tiles, 128 for many) are covered."""
 
 import numpy as np
 import pytest
@@ -39,8 +36,7 @@ def _close_bf16(got, ref):
     (3, 3, 2, 128, 16, 0, 150, 512, 100, True),    # paged value cache
     (1, 4, 8, 128, 32, 0, 2100, 256, 3, False),    # enough tiles for the 128-column tile shape
 ])
-@pytest.mark.parametrize("split", [False, True], ids=["ws256", "split-k"])
-def test_value_projection_matches_oracle(S, N, Hkv, d, r, mode, T, Dm, start, paged, split):
+def test_value_projection_matches_oracle(S, N, Hkv, d, r, mode, T, Dm, start, paged):
     g = torch.Generator(device=DEV)
     g.manual_seed(T * 13 + Dm + start)
     n_u = N if mode == 0 else 1
@@ -51,9 +47,7 @@ def test_value_projection_matches_oracle(S, N, Hkv, d, r, mode, T, Dm, start, pa
     session = S - 1
     prob = lrkv.make_problem(S, N, 2 * Hkv, Hkv, d, r, mode)
     u = torch.full((S, n_u, L, r), float("nan"), dtype=torch.bfloat16, device=DEV)
-    # a 256-byte workspace runs unsplit; the queried size lets few tiles split their K loop
-    nws = lrkv.lrkv_value_projection_workspace_bytes(prob, T, Dm) if split else 256
-    ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
     if not paged:
         k = torch.full((S, Hkv, L, d), float("nan"), dtype=torch.bfloat16, device=DEV)
         v = torch.full_like(k, float("nan"))
@@ -69,8 +63,7 @@ def test_value_projection_matches_oracle(S, N, Hkv, d, r, mode, T, Dm, start, pa
         table = torch.randperm(n_pages, generator=gcpu)[:S * n_lp].view(S, n_lp).to(torch.int32).to(DEV)
         kv = lrkv.kv_view_paged(k, v, table)
     v_before, u_before, k_before = v.clone(), u.clone(), k.clone()
-    for _ in range(2 if split else 1):  # twice: the split's tickets return to zero
-        lrkv.lrkv_value_projection(prob, x, w, kv, L, u, session, start, ws)
+    lrkv.lrkv_value_projection(prob, x, w, kv, L, u, session, start, ws)
     torch.cuda.synchronize()
     st, flags = lrkv.lrkv_query_device_status(ws)
     assert st == "LRKV_OK", (st, hex(flags))
