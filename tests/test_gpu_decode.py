@@ -55,6 +55,11 @@ SHAPES = [
     (2, 2, 4, 2, 64, 8, 96, 1, [95, 3, 0, 0], [96, 65]),
     (1, 3, 12, 2, 128, 32, 4097, 0, [4000, 4096, 1], [4097]),
     (4, 2, 2, 1, 64, 16, 200, 0, [0, 0, 50, 300, 10, 10, 199, 0], [1, 0, 200, 63]),  # L=1, empty session
+    # 17 to 24 rows per KV head (the key-split consumers): rank 8, shared U with
+    # offsets inside a warp's 16 keys, an empty session
+    (2, 3, 6, 1, 128, 8, 515, 1, [0, 250, 514, 3, 3, 0], [515, 0]),
+    (3, 4, 5, 1, 64, 16, 450, 0, [0, 7, 449, 100, 1, 1, 1, 1, 64, 65, 200, 0], [450, 1, 449]),  # 20 rows
+    (1, 3, 24, 3, 128, 16, 2000, 1, [0, 0, 0], [2000]),  # 24 rows, every offset 0: one Z pass
 ]
 
 
