@@ -388,34 +388,31 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Seg& sg
 // row), or, when this CTA is the last of the item's CTAs to get there (atomic
 // ticket), combine every partial record of the item and write
 // out = (O + Z B_i,g) / l: the up-projection of Eq. 12, once per row.  Run by a
-// team of NTH threads (tid in [0, NTH)) that `sync` synchronises; each thread
-// holds the B columns of PB (agent, dim) pairs at a time.
-template <int D, int NT, int RK, int NTH, int PB, typename Sync>
+// team of NTH threads (tid in [0, NTH)) that `sync` synchronises.
+template <int D, int NT, int RK, int NTH, typename Sync>
 __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegInfo& si, float* rec, float* scw,
                                                int* bcast, int tid, Sync sync) {
   constexpr int RP = NT * 8;
   constexpr int REC = RP * (D + RK + 2);
   constexpr int E4 = RP * (D + RK) / 4;
   constexpr int PERC = 6;  // float4 elements per thread per combine pass
+  constexpr int D2 = D / 2;
   const float NEG_INF = -INFINITY;
   const int HD = p.Hkv_total * D;  // B rows span every KV head
-  const int n_pairs = si.n_ag * D;
-  // The B columns of this thread's first (agent, dim) pairs are requested
-  // before the record is published, so that their latency overlaps the
-  // publish, the ticket and the combine rather than following them.
-  float bb[PB][RK];
-  auto load_b = [&](int e0) {
-#pragma unroll
-    for (int k = 0; k < PB; ++k) {
-      const int e = e0 + k * NTH;
-      if (e >= n_pairs) continue;
-      const uint16_t* bp =
-          static_cast<const uint16_t*>(p.b) + ((size_t)(si.i_lo + e / D) * RK) * HD + (size_t)(p.g_base + si.g) * D + e % D;
-#pragma unroll
-      for (int r = 0; r < RK; ++r) bb[k][r] = bf16_to_f32(__ldg(bp + (size_t)r * HD));
-    }
+  const int n_units = si.n_ag * D2;  // (agent, pair of adjacent dims)
+  // B columns of the (agent, dim pair) units this thread will write
+  auto b_col = [&](int u) {
+    return reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.b) +
+                                             ((size_t)(si.i_lo + u / D2) * RK) * HD + (size_t)(p.g_base + si.g) * D +
+                                             2 * (u % D2));
   };
-  load_b(tid);
+  // Bring this thread's first unit's B columns into L1 now (no registers held),
+  // so that their latency overlaps the publish, the ticket and the combine.
+  if (tid < n_units) {
+    const uint32_t* bp = b_col(tid);
+#pragma unroll
+    for (int r = 0; r < RK; ++r) asm volatile("prefetch.L1 [%0];" ::"l"(bp + (size_t)r * (HD / 2)));
+  }
   bool finish = true;
   if (si.segs > 1) {
     float* grec = p.partials + ((size_t)si.item * p.max_segs + (size_t)si.slot) * REC;
@@ -536,33 +533,51 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
     }
     sync();
   }
-  // out = (O + Z B_i,g) / l; one thread per (agent, dim), the agent's B column serves its GQA rows
+  // out = (O + Z B_i,g) / l.  A thread takes (agent, two adjacent dims): the
+  // agent's B columns (bf16 pairs) serve all its GQA rows, a Z row is read as
+  // float4s (the same row across the warp), O and the output go as pairs.
   const float* mL = rec + RP;
   const float* mO = rec + 2 * RP;
   const float* mZ = mO + RP * D;
-  for (int e0 = tid; e0 < n_pairs; e0 += PB * NTH) {
-    if (e0 != tid) load_b(e0);  // the first pairs' columns were requested at the start
+  if (tid < RP) scw[tid] = mL[tid] > 0.f ? 1.f / mL[tid] : 0.f;  // 1 / l per row (the scale table is free)
+  sync();
+  const int h0 = (p.g_base + si.g) * p.G;
+  for (int u = tid; u < n_units; u += NTH) {
+    const int agent = si.i_lo + u / D2;
+    const int dim = 2 * (u % D2);
+    const uint32_t* bp = b_col(u);
+    float b0[RK], b1[RK];
 #pragma unroll
-    for (int k = 0; k < PB; ++k) {
-      const int e = e0 + k * NTH;
-      if (e >= n_pairs) continue;
-      const int dim = e % D;
-      const int agent = si.i_lo + e / D;
-      int r_begin = agent * p.G - si.row_lo, r_end = r_begin + p.G;
-      r_begin = r_begin < 0 ? 0 : r_begin;
-      r_end = r_end > si.rows ? si.rows : r_end;
-      for (int row = r_begin; row < r_end; ++row) {
-        float acc = mO[row * D + dim];
+    for (int r = 0; r < RK; ++r) {
+      const uint32_t w = __ldg(bp + (size_t)r * (HD / 2));
+      b0[r] = __uint_as_float(w << 16);
+      b1[r] = __uint_as_float(w & 0xffff0000u);
+    }
+    int r_begin = agent * p.G - si.row_lo, r_end = r_begin + p.G;
+    r_begin = r_begin < 0 ? 0 : r_begin;
+    r_end = r_end > si.rows ? si.rows : r_end;
+    for (int row = r_begin; row < r_end; ++row) {
+      float2 o = *reinterpret_cast<const float2*>(mO + row * D + dim);
+      const float4* z4 = reinterpret_cast<const float4*>(mZ + row * RK);
 #pragma unroll
-        for (int r = 0; r < RK; ++r) acc = fmaf(mZ[row * RK + r], bb[k][r], acc);
-        const float L = mL[row];
-        const float o = L > 0.f ? acc / L : 0.f;
-        const int grow = si.row_lo + row;
-        const int h = (p.g_base + si.g) * p.G + grow % p.G;
-        const size_t oi = (((size_t)si.s * p.N + agent) * p.Hq + h) * D + dim;
-        if (p.out_f32) static_cast<float*>(p.out)[oi] = o;
-        else static_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(o);
+      for (int q = 0; q < RK / 4; ++q) {
+        const float4 z = z4[q];
+        o.x = fmaf(z.x, b0[4 * q], o.x);
+        o.y = fmaf(z.x, b1[4 * q], o.y);
+        o.x = fmaf(z.y, b0[4 * q + 1], o.x);
+        o.y = fmaf(z.y, b1[4 * q + 1], o.y);
+        o.x = fmaf(z.z, b0[4 * q + 2], o.x);
+        o.y = fmaf(z.z, b1[4 * q + 2], o.y);
+        o.x = fmaf(z.w, b0[4 * q + 3], o.x);
+        o.y = fmaf(z.w, b1[4 * q + 3], o.y);
       }
+      const float il = scw[row];
+      o.x *= il;
+      o.y *= il;
+      const int grow = si.row_lo + row;
+      const size_t oi = (((size_t)si.s * p.N + agent) * p.Hq + h0 + grow % p.G) * D + dim;
+      if (p.out_f32) *reinterpret_cast<float2*>(static_cast<float*>(p.out) + oi) = o;
+      else *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.out) + oi) = __floats2bfloat162_rn(o.x, o.y);
     }
   }
 }
@@ -901,7 +916,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     } else {
       const SegInfo si = seg_info(p, sg);
       float* scw = reinterpret_cast<float*>(smem + lay.scw_off);  // the consumers' half
-      finish_segment<D, NT, RK, CT, (RK >= 32 ? 2 : 4)>(p, si, merge, scw, bcast, tid, [] { named_bar_sync(1, CT); });
+      finish_segment<D, NT, RK, CT>(p, si, merge, scw, bcast, tid, [] { named_bar_sync(1, CT); });
     }
     ++sn;
   }
@@ -928,8 +943,7 @@ __device__ void decode_epilogue(const DecodeParams& p, uint8_t* smem, const Deco
     const int buf = sn & 1;
     if (!mbar_wait_bounded(&rec_full[buf], (sn >> 1) & 1, abort_flag, p.flags, p.spin_cap)) break;
     const SegInfo si = seg_info(p, sg);
-    finish_segment<D, NT, RK, 32, (RK >= 32 ? 1 : 2)>(p, si, merge0 + buf * REC, scw, bcast, lane,
-                                                      [] { __syncwarp(); });
+    finish_segment<D, NT, RK, 32>(p, si, merge0 + buf * REC, scw, bcast, lane, [] { __syncwarp(); });
     __syncwarp();
     if (lane == 0) mbar_arrive(&rec_free[buf]);
     ++sn;

@@ -206,6 +206,15 @@ lrkv_status plan_decode(const lrkv_problem* p, int hkv, int max_seq_len, const D
   pl->W = (long long)pl->items * pl->nt;
   const int sms = dev.sms > 0 ? dev.sms : 148;
   pl->ctas = (int)(pl->W < sms ? pl->W : sms);
+  // Whole items, one per CTA, when there are no more items than SMs and the even
+  // split would take fewer than kWholeItemSlackTiles tiles off a CTA: an item
+  // split over CTAs pays for publishing its partial records, a ticket and their
+  // merge at the end of the launch.  (Measured on Qwen3 shapes with 128 items
+  // of 16 / 32 / 64 tiles: 0.633 -> 0.510, 0.869 -> 0.779 and 1.378 -> 1.332 ms
+  // per 28 layers; a fit gives about 5.4 us per launch for the split against
+  // 0.44 us per extra tile.)
+  if (pl->items <= sms && pl->nt <= (int)((pl->W + pl->ctas - 1) / pl->ctas) + lrkv::kWholeItemSlackTiles)
+    pl->ctas = pl->items;
   int ms = 1;
   for (int it = 0; it < pl->items; ++it) {
     const long long cf = lrkv::owner_cta((long long)it * pl->nt, pl->W, pl->ctas);

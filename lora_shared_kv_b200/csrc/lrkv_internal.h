@@ -19,6 +19,7 @@ constexpr int kKeysPerTile = 64;        // keys per K/V tile (one TMA box, one p
 constexpr int kMaxRowsPerItem = 32;     // query rows (agents x GQA heads) per decode work item
 constexpr int kMaxAgents = 16;
 constexpr int kTileRun = 4;             // decode tiles visited contiguously (see TileOrder in decode.cu)
+constexpr int kWholeItemSlackTiles = 12;  // decode: whole items per CTA if that adds at most this many tiles
 
 // Spin cap of every bounded wait.  A try_wait suspends for a short while per
 // attempt, so this is well over a second of waiting: far beyond any healthy

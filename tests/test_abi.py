@@ -139,8 +139,9 @@ def _decode_ws_expected(S, N, Hq, Hkv, d, r, L, sms=148):
     # in as few groups of at most 32 as cover them, each padded to a multiple
     # of 8; work items (session, KV head, row group) of ceil(L/64) key tiles;
     # the flattened tiles split evenly over min(tiles, SMs) CTAs, CTA c taking
-    # [c W / C, (c + 1) W / C); one partial record per CTA that touches an
-    # item, when more than one does
+    # [c W / C, (c + 1) W / C), unless whole items fit one per SM and add at
+    # most 12 tiles to a CTA's share (then one CTA per item); one partial
+    # record per CTA that touches an item, when more than one does
     R = N * (Hq // Hkv)
     n_rg = -(-R // 32)
     NT = -(-(-(-R // n_rg)) // 8)
@@ -148,6 +149,8 @@ def _decode_ws_expected(S, N, Hq, Hkv, d, r, L, sms=148):
     items = S * Hkv * n_rg
     W = items * nt
     C = min(W, sms)
+    if items <= sms and nt <= -(-W // C) + 12:
+        C = items
     touching = [0] * items
     for c in range(C):
         lo, hi = c * W // C, (c + 1) * W // C

@@ -70,11 +70,15 @@ def test_decode_items_split_over_the_ctas(S, N, Hq, Hkv, L):
     items = S * Hkv * n_rg
     W = items * nt
     C = min(W, 148)
+    whole = items <= 148 and nt <= -(-W // C) + 12  # the planner's whole-item rule
+    if whole:
+        C = items
     # the workspace holds, per item, as many records as the most CTAs any item touches
     touching = [0] * items
     for lo, hi in ranges(W, C):
         for it in range(lo // nt, (hi - 1) // nt + 1):
             touching[it] += 1
+    assert not whole or max(touching) == 1  # one CTA per item: nothing to merge
     _check_cover([nt] * items, C, max(touching))
 
 
