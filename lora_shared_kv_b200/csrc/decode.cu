@@ -16,7 +16,9 @@
 //    K/V tile is read from HBM once for all agents.
 //  * The flattened (item, key tile) space is split evenly over one CTA per SM
 //    (stream-K style); an item cut by a CTA boundary is merged by the last CTA
-//    to finish it (atomic ticket), which also applies Z B_i and the 1/l.
+//    to finish it (atomic ticket), which also applies Z B_i and the 1/l.  When
+//    the items fit one per SM and that adds only a few tiles to a CTA's share,
+//    the host gives each CTA one whole item instead (nothing to merge).
 //  * A producer warp moves 64-key K/V tiles (128B-swizzled) and the rank-r U
 //    tiles with the Tensor Memory Accelerator into a ring of stages guarded by
 //    mbarriers.  U tiles wholly before an agent's offset are never loaded.
