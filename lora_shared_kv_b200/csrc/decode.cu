@@ -650,6 +650,10 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
     const int ag_lo = w_rows > 0 ? w_row_lo / p.G - sg.i_lo : 0;
     const int ag_hi = w_rows > 0 ? (w_row_lo + w_rows - 1) / p.G - sg.i_lo : -1;
     const int my_agent = qvalid ? (sg.row_lo + qrow) / p.G - sg.i_lo : -1;
+    // the first key any of this warp's agents keeps a U row for: tiles wholly
+    // before it skip the low-rank passes at one compare
+    int a_first = 0x7fffffff;
+    for (int ag = ag_lo; ag <= ag_hi; ++ag) a_first = min(a_first, a_sm[ag]);
 
     RowState<D, RK> st;
     st.m[0] = st.m[1] = NEG_INF;
@@ -813,7 +817,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       // Tiles wholly inside [a_i, seq_len) need no masks: one ldmatrix and one MMA per key block.
       const bool lr_full = p.mode == LRKV_BASE_LR_SHARED && !boundary && a_max <= tile_key0;
       const int pass_lo = lr_full ? 0 : ag_lo;
-      const int pass_hi = lr_full ? 0 : ag_hi;
+      const int pass_hi = lr_full ? 0 : (tile_key0 + KT > a_first ? ag_hi : ag_lo - 1);
       for (int ag = pass_lo; ag <= pass_hi; ++ag) {
         const int a_i = lr_full ? 0 : a_sm[ag];
         if (tile_key0 + KT <= a_i) continue;  // producer did not load this U tile
