@@ -270,7 +270,10 @@ template <int D, int RK>
 struct RowState {
   static constexpr int MT = D / 16;
   static constexpr int MTZ = RK >= 16 ? RK / 16 : 1;
-  float m[2], l[2];       // rows 2 t4, 2 t4 + 1 of the warp's 8
+  float m[2];
+  // row sums as the accumulator of (all-ones 16 x 16) x P^T: l[0], l[1] are rows
+  // 2 t4 and 2 t4 + 1, complete over every key of the segment; l[2], l[3] repeat them
+  float l[4];       // rows 2 t4, 2 t4 + 1 of the warp's 8
   float o[MT][4];         // O^T: dims (16 mt + g8, + 8) x rows
   float z[MTZ][4];        // Z^T: ranks x rows
 };
@@ -657,7 +660,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
 
     RowState<D, RK> st;
     st.m[0] = st.m[1] = NEG_INF;
-    st.l[0] = st.l[1] = 0.f;
+    st.l[0] = st.l[1] = st.l[2] = st.l[3] = 0.f;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -726,8 +729,6 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       float mx0 = NEG_INF, mx1 = NEG_INF;
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sacc[kb][e] *= p.scale_log2;
         if (boundary) {  // keys at or past seq_len are selected out
           const bool va = tile_key0 + 16 * kb + g8 < sl;
           const bool vb = tile_key0 + 16 * kb + g8 + 8 < sl;
@@ -744,6 +745,10 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
+      // the scale is positive and rounding monotonic: the max of the scaled
+      // scores is the scaled max, and each weight takes the scale in one fma
+      mx0 *= p.scale_log2;
+      mx1 *= p.scale_log2;
       const bool need = (mx0 > st.m[0] + 8.f) || (mx1 > st.m[1] + 8.f);
       if (__any_sync(0xffffffffu, need)) {
         float al[2];
@@ -754,6 +759,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           al[e] = mn == NEG_INF ? 1.f : fast_exp2(st.m[e] - mn);
           st.m[e] = mn;
           st.l[e] *= al[e];
+          st.l[e + 2] *= al[e];
         }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
@@ -773,16 +779,16 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       const float mu0 = st.m[0] == NEG_INF ? 0.f : st.m[0];
       const float mu1 = st.m[1] == NEG_INF ? 0.f : st.m[1];
       uint32_t pb[4][2];
+      const float sc = p.scale_log2;
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
-        const float p0 = fast_exp2(sacc[kb][0] - mu0), p1 = fast_exp2(sacc[kb][1] - mu1);
-        const float p2 = fast_exp2(sacc[kb][2] - mu0), p3 = fast_exp2(sacc[kb][3] - mu1);
-        const uint32_t w01 = pack_bf16x2(p0, p1), w23 = pack_bf16x2(p2, p3);
-        // the row sums of exactly the bf16 weights the value MMA uses
-        st.l[0] += __uint_as_float(w01 << 16) + __uint_as_float(w23 << 16);
-        st.l[1] += __uint_as_float(w01 & 0xffff0000u) + __uint_as_float(w23 & 0xffff0000u);
-        pb[kb][0] = movmatrix_t(w01);
-        pb[kb][1] = movmatrix_t(w23);
+        const float p0 = fast_exp2(fmaf(sacc[kb][0], sc, -mu0)), p1 = fast_exp2(fmaf(sacc[kb][1], sc, -mu1));
+        const float p2 = fast_exp2(fmaf(sacc[kb][2], sc, -mu0)), p3 = fast_exp2(fmaf(sacc[kb][3], sc, -mu1));
+        pb[kb][0] = movmatrix_t(pack_bf16x2(p0, p1));
+        pb[kb][1] = movmatrix_t(pack_bf16x2(p2, p3));
+        // the row sums of exactly the bf16 weights the value MMA uses: ones x P^T
+        constexpr uint32_t kOnes = 0x3F803F80u;  // two bf16 1.0
+        mma_bf16_16816(st.l, kOnes, kOnes, kOnes, kOnes, pb[kb][0], pb[kb][1]);
       }
 
       // ---- O^T += V^T P^T ; V rows past seq_len are selected out
@@ -895,15 +901,6 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
       Seg nx = make_seg(p, t, t_end, false);
       seg_rows(p, nx);
       load_q_frags<D>(p, nx, rbase + g8, t4, qf);
-    }
-    // reduce l over the lanes that share a row
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float v = st.l[e];
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 16);
-      st.l[e] = v;
     }
     // the record buffer of segment sn - 2 must have been released by the epilogue warp
     if (sn >= 2) mbar_wait_bounded(&rec_free[buf], ((sn >> 1) - 1) & 1, abort_flag, p.flags, p.spin_cap);
