@@ -697,7 +697,8 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           }
         }
       }
-      mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags, p.spin_cap);
+      if (!mbar_test(&full[my_stage], my_phase))  // most tiles have landed by now
+        mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags, p.spin_cap);
       const uint32_t Ks = ring_s + my_stage * lay.stage_bytes;
       const uint32_t Vs = Ks + KV_BYTES;
       const uint32_t Us = Vs + KV_BYTES;
