@@ -86,10 +86,13 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait on a phase of an mbarrier.  Returns false (and records a
 // timeout flag and raises the CTA's abort word) when `cap` failed attempts are
-// reached or another thread of the CTA has already aborted.
+// reached or another thread of the CTA has already aborted.  With `test_first`
+// a phase that has already completed is seen by a non-blocking test, without
+// the blocking try (measured faster on the waits that usually find it done).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort_flag, unsigned* err,
-                                                  uint32_t cap = kSpinCap) {
+                                                  uint32_t cap = kSpinCap, bool test_first = false) {
+  if (test_first && mbar_test(bar, parity)) return true;  // already complete: no blocking try
   uint32_t spins = 0;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;

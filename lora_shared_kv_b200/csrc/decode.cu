@@ -197,7 +197,7 @@ __device__ void decode_producer(const DecodeParams& p, const CUtensorMap* tmK, c
       const unsigned umask = p.mode == LRKV_BASE_SHARED ? need : (need ? 1u : 0u);
       const bool page_ok = !p.paged || (phys >= 0 && phys < p.num_pages);
       const uint32_t bytes = (page_ok ? 2 * KV_BYTES : 0) + __popc(umask) * U_BYTES;
-      const bool freed = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.flags, p.spin_cap);
+      const bool freed = mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, p.flags, p.spin_cap, true);
       // After an abort the consumers release stages without waiting for their
       // copies, so nothing more may be issued: a stage could receive a second
       // copy while the first is still landing.  The abort word is read after the
@@ -697,8 +697,7 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
           }
         }
       }
-      if (!mbar_test(&full[my_stage], my_phase))  // most tiles have landed by now
-        mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags, p.spin_cap);
+      mbar_wait_bounded(&full[my_stage], my_phase, abort_flag, p.flags, p.spin_cap, true);  // most tiles have landed
       const uint32_t Ks = ring_s + my_stage * lay.stage_bytes;
       const uint32_t Vs = Ks + KV_BYTES;
       const uint32_t Us = Vs + KV_BYTES;

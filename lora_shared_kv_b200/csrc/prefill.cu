@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           // B_i,g of this segment into buffer si & 1, once segment si - 2's epilogue is done with it
           // After an abort the softmax warps release B buffers whose copies may still be
           // landing: issue nothing more (the abort word is read after the wait's acquire).
-          if ((si >= 2 && !mbar_wait_bounded(&bars->b_free[si & 1], ((si >> 1) - 1) & 1, abort_flag, p.flags, p.spin_cap)) ||
+          if ((si >= 2 && !mbar_wait_bounded(&bars->b_free[si & 1], ((si >> 1) - 1) & 1, abort_flag, p.flags, p.spin_cap, true)) ||
               *abort_flag) {
             ok = false;
             break;
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int jb = sg.lo; jb < sg.hi; ++jb, ++n) {
           const int st = n % NS;
-          if (!mbar_wait_bounded(&empty[st], ((n / NS) & 1) ^ 1, abort_flag, p.flags, p.spin_cap) || *abort_flag) {
+          if (!mbar_wait_bounded(&empty[st], ((n / NS) & 1) ^ 1, abort_flag, p.flags, p.spin_cap, true) || *abort_flag) {
             ok = false;
             break;
           }
@@ -341,8 +341,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr uint32_t ID_ZB = umma_idesc_bf16(BM, D, 0, 1);  // O += Z B_i,g
     auto issue_pv = [&]() -> bool {
       const int st = pv_n % VST;
-      if (!mbar_wait_bounded(&bars->p_full[pv_n & 1], (pv_n >> 1) & 1, abort_flag, p.flags, p.spin_cap)) return false;
-      if (!mbar_wait_bounded(&bars->v_full[st], (pv_n / VST) & 1, abort_flag, p.flags, p.spin_cap)) return false;
+      if (!mbar_wait_bounded(&bars->p_full[pv_n & 1], (pv_n >> 1) & 1, abort_flag, p.flags, p.spin_cap, true)) return false;
+      if (!mbar_wait_bounded(&bars->v_full[st], (pv_n / VST) & 1, abort_flag, p.flags, p.spin_cap, true)) return false;
       uint8_t* Us = smem + Lay::V_OFF + st * Lay::V_STAGE + Lay::U_OFF;
       if (pv_jb * BN < pv_a) {
         // U rows before the offset are zero-filled before the MMA reads them: all
@@ -370,8 +370,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (pv_last) {
         // the segment's O += Z B_i,g: Z (bf16 pairs) in the S buffer of its last block, B in buffer pv_si & 1
-        if (!mbar_wait_bounded(&bars->zb_full, pv_si & 1, abort_flag, p.flags, p.spin_cap)) return false;
-        if (!mbar_wait_bounded(&bars->b_full[pv_si & 1], (pv_si >> 1) & 1, abort_flag, p.flags, p.spin_cap)) return false;
+        if (!mbar_wait_bounded(&bars->zb_full, pv_si & 1, abort_flag, p.flags, p.spin_cap, true)) return false;
+        if (!mbar_wait_bounded(&bars->b_full[pv_si & 1], (pv_si >> 1) & 1, abort_flag, p.flags, p.spin_cap, true)) return false;
         if (lane == 0) {
           tc_fence_after();
           const uint32_t b_base = smem_u32(smem + Lay::B_OFF + (pv_si & 1) * Lay::B_BYTES);
@@ -395,10 +395,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       f += sg.hi - sg.lo;
       const int a_i = agent_offset(p, sg.agent, false);
       // the segment's Q is in TMEM (its previous content was read by the last S issued)
-      ok = mbar_wait_bounded(&bars->q_full, si & 1, abort_flag, p.flags, p.spin_cap);
+      ok = mbar_wait_bounded(&bars->q_full, si & 1, abort_flag, p.flags, p.spin_cap, true);
       for (int jb = sg.lo; jb < sg.hi && ok; ++jb, ++n) {
         const int st = n % KST;
-        ok = mbar_wait_bounded(&bars->k_full[st], (n / KST) & 1, abort_flag, p.flags, p.spin_cap);
+        ok = mbar_wait_bounded(&bars->k_full[st], (n / KST) & 1, abort_flag, p.flags, p.spin_cap, true);
         if (!ok) break;
         if (lane == 0) {
           tc_fence_after();
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int limit = p.L0 + token;  // last visible key of this row
       float m_ref = NEG_INF;
       for (int jb = sg.lo; jb < sg.hi; ++jb, ++n) {
-        if (ok) ok = mbar_wait_bounded(&bars->s_full[n & 1], (n >> 1) & 1, abort_flag, p.flags, p.spin_cap);
+        if (ok) ok = mbar_wait_bounded(&bars->s_full[n & 1], (n >> 1) & 1, abort_flag, p.flags, p.spin_cap, true);
         tc_fence_after();
         const uint32_t s_col = n & 1 ? Lay::COL_S1 : Lay::COL_S0;
         float x[HB];
@@ -525,7 +525,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (jb > sg.lo) {
             // O, Z and l hold the segment's blocks before this one: rescale this
             // half's share of their columns in TMEM once the previous PV is done
-            if (ok) ok = mbar_wait_bounded(&bars->o_ready[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, p.flags, p.spin_cap);
+            if (ok) ok = mbar_wait_bounded(&bars->o_ready[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, p.flags, p.spin_cap, true);
             tc_fence_after();
 #pragma unroll
             for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
@@ -576,7 +576,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // last block, free once its PV is done) for the O += Z B_i,g MMA; then
       // out = O / l, or this segment's rows are published for the tile's last CTA.
       const int nl = n - 1;  // the segment's last block
-      if (ok) ok = mbar_wait_bounded(&bars->o_ready[nl & 1], (nl >> 1) & 1, abort_flag, p.flags, p.spin_cap);
+      if (ok) ok = mbar_wait_bounded(&bars->o_ready[nl & 1], (nl >> 1) & 1, abort_flag, p.flags, p.spin_cap, true);
       tc_fence_after();
       float l;
       {
@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->zb_full);
-      if (ok) ok = mbar_wait_bounded(&bars->zb_done, si & 1, abort_flag, p.flags, p.spin_cap);
+      if (ok) ok = mbar_wait_bounded(&bars->zb_done, si & 1, abort_flag, p.flags, p.spin_cap, true);
       tc_fence_after();
       const bool whole = sg.lo == 0 && sg.hi == sg.nb;
       bool finish = true;
