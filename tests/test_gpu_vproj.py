@@ -6,8 +6,9 @@ sit within bf16's unit roundoff (2^-8 relative: one rounding to the nearest of
 8 significand bits) of the exact value, plus a small allowance for the fp32
 accumulation.  Rows outside [start_row, start_row + T),
 other sessions and the K cache stay untouched.  Token counts and Dm that are
-not tile multiples, both sharing modes, a paged value cache and both tile
-widths (64 columns for few tiles, 128 for many) are covered."""
+not tile multiples, both sharing modes, a paged value cache, the K loop split
+over clusters of 2 to 8 CTAs (few tiles; uneven K ranges) and unsplit (many
+tiles) are covered."""
 
 import numpy as np
 import pytest
@@ -34,7 +35,9 @@ def _close_bf16(got, ref):
     (2, 2, 8, 128, 16, 1, 64, 200, 17, False),     # BaseLRShared: one U; Dm not a multiple of 64
     (1, 2, 2, 64, 8, 0, 300, 136, 64, False),
     (3, 3, 2, 128, 16, 0, 150, 512, 100, True),    # paged value cache
-    (1, 4, 8, 128, 32, 0, 2100, 256, 3, False),    # enough tiles for the 128-column tile shape
+    (1, 4, 8, 128, 32, 0, 2100, 256, 3, False),    # enough tiles that the K loop is not split
+    (1, 2, 2, 64, 8, 0, 100, 1024, 0, False),      # one tile: K split over a cluster of 8
+    (2, 3, 1, 128, 16, 1, 77, 136, 9, True),       # K split 3 ways, ragged last K step, paged
 ])
 def test_value_projection_matches_oracle(S, N, Hkv, d, r, mode, T, Dm, start, paged):
     g = torch.Generator(device=DEV)
