@@ -6,18 +6,19 @@
 // projection as X W0 + (X A_i) B_i; both parts read the same hidden states, so
 // one GEMM produces the shared base values and every U_i row at once.
 //
-// A tcgen05 GEMM over 128-token x 256-column tiles: X (K-major) and W
-// (column-major atoms), both 128B-swizzled, stream through a 4-stage TMA ring
-// in 64-wide K steps; fp32 accumulation in TMEM.  An M = 128 MMA from shared
-// memory costs about the same for every N up to 256, so the tiles are as wide
-// as the instruction allows; when there are fewer tiles than SMs, the K loop of
-// a tile is split over a thread-block cluster of S CTAs (S <= 8, one K range
-// each).  Each CTA parks its fp32 partial tile in its own shared memory (the
-// ring is idle by then) and, after a cluster barrier, sums one slice of the
-// tile's rows over all S partials through distributed shared memory, in rank
-// order (so the result does not depend on timing), converts to bf16 and
-// scatters each row's columns to its cache: column c < Hkv d goes to KV head
-// c / d of the base value cache, the rest to agent slot (c - Hkv d) / r.
+// A tcgen05 GEMM over 128-token x BN-column tiles: X (K-major) and W
+// (column-major atoms), both 128B-swizzled, stream through a TMA ring in
+// 64-wide K steps; fp32 accumulation in TMEM.  An M = 128 MMA from shared
+// memory costs about the same for every N up to 256, so BN is 256 when there
+// are many tiles.  When there are few, the K loop of a tile is split over a
+// thread-block cluster of S CTAs (S <= 8, one K range each) and BN is 128:
+// each CTA parks its fp32 partial tile in its own shared memory (the ring is
+// idle by then) and, after a cluster barrier, sums one slice of the tile's
+// rows over all S partials through distributed shared memory, in rank order
+// (so the result does not depend on timing); that traffic, not the MMAs,
+// bounds a split tile, and it halves with BN.  The sums are converted to bf16
+// and each row's columns scattered to its cache: column c < Hkv d goes to KV
+// head c / d of the base value cache, the rest to agent slot (c - Hkv d) / r.
 // The summation order inside the tensor core is not specified, so U rows made
 // here are not bit-identical to the fixed-order append.
 #include "common.cuh"
@@ -27,20 +28,27 @@ namespace lrkv {
 
 namespace {
 
-constexpr int VP_BM = 128;                                        // tokens per tile (TMEM lanes)
-constexpr int VP_BN = 256;                                        // columns per tile (TMEM columns)
-constexpr int VP_BK = 64;                                         // K per stage
+constexpr int VP_BM = 128;                      // tokens per tile (TMEM lanes)
+constexpr int VP_BK = 64;                       // K per stage
 constexpr int VP_THREADS = 256;
-constexpr int VP_ATOMS = VP_BN / 64;                              // 64-column W atoms per stage
-constexpr int VP_X_BYTES = VP_BM * VP_BK * 2;                     // 16 KB
-constexpr int VP_ATOM_BYTES = VP_BK * 128;                        // 8 KB: 64 k-rows x 128 B
-constexpr int VP_STAGE = VP_X_BYTES + VP_ATOMS * VP_ATOM_BYTES;   // 48 KB
-constexpr int VP_ST = 4;                                          // ring stages
-constexpr int VP_RING = VP_ST * VP_STAGE;                         // 192 KB
-constexpr int VP_RP = VP_BN + 4;     // fp32 pitch of a partial-tile row: conflict-free 16-byte stores
+constexpr int VP_X_BYTES = VP_BM * VP_BK * 2;   // 16 KB
+constexpr int VP_ATOM_BYTES = VP_BK * 128;      // 8 KB: 64 k-rows x 128 B
+constexpr int VP_RING = 192 * 1024;             // shared memory for the ring
 constexpr int VP_SMEM = VP_RING + 256;
-constexpr int VP_MAX_SPLIT = 8;      // portable cluster size
-static_assert(VP_BM * VP_RP * 4 <= VP_RING, "the partial tile reuses the ring");
+constexpr int VP_MAX_ST = 6;
+constexpr int VP_MAX_SPLIT = 8;                 // portable cluster size
+
+// A tile of 128 tokens x BN columns (BN = 256, or 128 when the K loop is split:
+// each CTA's partial tile, which the split moves across the cluster, halves).
+template <int BN>
+struct VpTile {
+  static constexpr int ATOMS = BN / 64;                            // 64-column W atoms per stage
+  static constexpr int STAGE = VP_X_BYTES + ATOMS * VP_ATOM_BYTES;  // 32 or 48 KB
+  static constexpr int ST = VP_RING / STAGE;                        // 6 or 4 stages
+  static constexpr int RP = BN + 4;  // fp32 pitch of a partial-tile row: conflict-free 16-byte stores
+  static_assert(ST <= VP_MAX_ST, "barrier slots");
+  static_assert(VP_BM * RP * 4 <= VP_RING, "the partial tile reuses the ring");
+};
 
 // Thread-block clusters: distributed shared memory.
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -75,17 +83,22 @@ __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
 }
 
 struct VpBars {
-  uint64_t full[VP_ST];
-  uint64_t empty[VP_ST];
+  uint64_t full[VP_MAX_ST];
+  uint64_t empty[VP_MAX_ST];
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort_flag;
   int ok;  // this CTA's partial tile is complete
 };
 
+template <int BN>
 __global__ void __launch_bounds__(VP_THREADS, 1)
     vproj_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const VprojParams p) {
+  using Sh = VpTile<BN>;
+  constexpr int VP_ST = Sh::ST;
+  constexpr int VP_STAGE = Sh::STAGE;
+  constexpr int VP_RP = Sh::RP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   VpBars* bars = reinterpret_cast<VpBars*>(smem + VP_RING);
@@ -93,13 +106,13 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * VP_BM;  // first token
-  const int n0 = blockIdx.y * VP_BN;  // first output column
+  const int n0 = blockIdx.y * BN;  // first output column
   const int S = gridDim.z;            // K split = cluster size; cluster dims (1, 1, S)
   const int z = (int)cluster_ctarank();
   const int nk_all = (p.Dm + VP_BK - 1) / VP_BK;
   const int kt0 = (int)((long long)z * nk_all / S);
   const int nk = (int)((long long)(z + 1) * nk_all / S) - kt0;  // >= 1: the launcher keeps S <= nk_all
-  const int natoms = min(VP_ATOMS, (p.ncols - n0 + 63) / 64);   // W atoms that reach into the weights
+  const int natoms = min(Sh::ATOMS, (p.ncols - n0 + 63) / 64);   // W atoms that reach into the weights
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < VP_ST; ++s) {
@@ -112,7 +125,7 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, VP_BN);
+    tmem_alloc(&bars->tmem_base, BN);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -154,7 +167,7 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
   } else if (warp == 1) {
     // ---- MMA issuer: D[128 tokens x 256 columns] += X[tokens, k] W[k, columns]
     // (atoms past the weights' last column are not loaded; their columns are never read)
-    constexpr uint32_t ID = umma_idesc_bf16(VP_BM, VP_BN, 0, 1);
+    constexpr uint32_t ID = umma_idesc_bf16(VP_BM, BN, 0, 1);
     bool ok = true;
     for (int j = 0; j < nk && ok; ++j) {
       const int st = j % VP_ST;
@@ -184,7 +197,7 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
     if (!ok) {
       bars->ok = 0;
     } else {
-      const int nch = (min(VP_BN, p.ncols - n0) + 31) / 32;
+      const int nch = (min(BN, p.ncols - n0) + 31) / 32;
       float4* dst = reinterpret_cast<float4*>(part + row * VP_RP);
 #pragma unroll 1
       for (int c = 0; c < nch; ++c) {
@@ -203,8 +216,10 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
   cluster_sync();  // every partial tile of the cluster is in place
 
   // ---- rows [row_lo, row_hi) of the tile: the sum of the S partials, a warp per
-  // two rows at a time, 4 + 4 columns per lane, written as bf16 to the caches
+  // two rows at a time, 4 columns per lane in each 128-column half, written as
+  // bf16 to the caches
   {
+    constexpr int NH = BN / 128;
     int all_ok = 1;
     for (int q = 0; q < S; ++q) all_ok &= ld_cluster_s32(cluster_map(smem_u32(&bars->ok), (uint32_t)q));
     const int row_lo = z * VP_BM / S, row_hi = min((z + 1) * VP_BM / S, p.T - m0);
@@ -240,16 +255,18 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
             if (q < S) {
               const uint32_t a = cluster_map(src, (uint32_t)q);
               lo[q] = ld_cluster_f4(a);
-              hi[q] = ld_cluster_f4(a + VP_BN / 2 * 4);  // past ncols: never stored
+              if constexpr (NH == 2) hi[q] = ld_cluster_f4(a + 128 * 4);  // past ncols: never stored
             }
           }
           acc[h][0] = lo[0];
-          acc[h][1] = hi[0];
+          if constexpr (NH == 2) acc[h][1] = hi[0];
 #pragma unroll
           for (int q = 1; q < VP_MAX_SPLIT; ++q) {
             if (q < S) {
               acc[h][0].x += lo[q].x; acc[h][0].y += lo[q].y; acc[h][0].z += lo[q].z; acc[h][0].w += lo[q].w;
-              acc[h][1].x += hi[q].x; acc[h][1].y += hi[q].y; acc[h][1].z += hi[q].z; acc[h][1].w += hi[q].w;
+              if constexpr (NH == 2) {
+                acc[h][1].x += hi[q].x; acc[h][1].y += hi[q].y; acc[h][1].z += hi[q].z; acc[h][1].w += hi[q].w;
+              }
             }
           }
         }
@@ -259,8 +276,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
         if (h < nr) {
           const int row = r0 + h * (VP_THREADS / 32);
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            uint16_t* dst = dest(row, n0 + 4 * lane + VP_BN / 2 * e);
+          for (int e = 0; e < NH; ++e) {
+            uint16_t* dst = dest(row, n0 + 4 * lane + 128 * e);
             if (dst)
               *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[h][e].x, acc[h][e].y),
                                                           pack_bf16x2(acc[h][e].z, acc[h][e].w));
@@ -273,12 +290,13 @@ __global__ void __launch_bounds__(VP_THREADS, 1)
   cluster_sync();  // the other CTAs have finished reading this CTA's partial tile
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, VP_BN);
+    tmem_dealloc(tmem, BN);
   }
 }
 
 // Largest K split S <= cap whose clusters all fit on the device at once for
-// `tiles` tiles (queried once per device and S; -1 records a failed query).
+// `tiles` tiles (queried once per device, tile width and S; -1 records a failed query).
+template <int BN>
 int pick_split(int tiles, int cap) {
   constexpr int kDevices = 64;
   static std::atomic<int> cache[kDevices][VP_MAX_SPLIT + 1];
@@ -298,7 +316,7 @@ int pick_split(int tiles, int cap) {
       attr[0].val.clusterDim.z = S;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, vproj_kernel, &cfg) != cudaSuccess || n < 1) {
+      if (cudaOccupancyMaxActiveClusters(&n, vproj_kernel<BN>, &cfg) != cudaSuccess || n < 1) {
         cudaGetLastError();
         n = -1;
       }
@@ -309,21 +327,18 @@ int pick_split(int tiles, int cap) {
   return 1;
 }
 
-}  // namespace
-
-int vproj_smem_bytes() { return VP_SMEM + 1024; }
-
-lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, int sms, void* stream) {
+template <int BN>
+lrkv_status launch_t(const VprojParams& p, const void* tmX, const void* tmW, int sms, void* stream) {
   const int smem = VP_SMEM + 1024;
-  if (ensure_dynamic_smem<vproj_kernel>(smem) != cudaSuccess) return LRKV_ERR_CUDA;
-  const int tiles = ((p.T + VP_BM - 1) / VP_BM) * ((p.ncols + VP_BN - 1) / VP_BN);
+  if (ensure_dynamic_smem<vproj_kernel<BN>>(smem) != cudaSuccess) return LRKV_ERR_CUDA;
+  const int tiles = ((p.T + VP_BM - 1) / VP_BM) * ((p.ncols + BN - 1) / BN);
   const int nk = (p.Dm + VP_BK - 1) / VP_BK;
   int cap = sms / tiles;
   cap = cap < VP_MAX_SPLIT ? cap : VP_MAX_SPLIT;
   cap = cap < nk ? cap : nk;
-  const int S = cap > 1 ? pick_split(tiles, cap) : 1;
+  const int S = cap > 1 ? pick_split<BN>(tiles, cap) : 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.T + VP_BM - 1) / VP_BM, (p.ncols + VP_BN - 1) / VP_BN, S);
+  cfg.gridDim = dim3((p.T + VP_BM - 1) / VP_BM, (p.ncols + BN - 1) / BN, S);
   cfg.blockDim = dim3(VP_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = static_cast<cudaStream_t>(stream);
@@ -336,10 +351,22 @@ lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW,
   attr[1].val.clusterDim.z = S;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, vproj_kernel, *static_cast<const CUtensorMap*>(tmX),
+  if (cudaLaunchKernelEx(&cfg, vproj_kernel<BN>, *static_cast<const CUtensorMap*>(tmX),
                          *static_cast<const CUtensorMap*>(tmW), p) != cudaSuccess)
     return LRKV_ERR_CUDA;
   return LRKV_OK;
+}
+
+}  // namespace
+
+int vproj_smem_bytes() { return VP_SMEM + 1024; }
+
+lrkv_status launch_vproj(const VprojParams& p, const void* tmX, const void* tmW, int sms, void* stream) {
+  // 128-column tiles when there are few enough of them that the K loop gets split
+  // (half the partial tile to move per CTA), else 256 (half the MMAs per column)
+  const int tiles128 = ((p.T + VP_BM - 1) / VP_BM) * ((p.ncols + 127) / 128);
+  if (tiles128 * 2 <= sms) return launch_t<128>(p, tmX, tmW, sms, stream);
+  return launch_t<256>(p, tmX, tmW, sms, stream);
 }
 
 }  // namespace lrkv

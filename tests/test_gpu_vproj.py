@@ -7,8 +7,8 @@ sit within bf16's unit roundoff (2^-8 relative: one rounding to the nearest of
 accumulation.  Rows outside [start_row, start_row + T),
 other sessions and the K cache stay untouched.  Token counts and Dm that are
 not tile multiples, both sharing modes, a paged value cache, the K loop split
-over clusters of 2 to 8 CTAs (few tiles; uneven K ranges) and unsplit (many
-tiles) are covered."""
+over clusters of 2 to 8 CTAs (few tiles; uneven K ranges; 128- and 256-column
+tiles) and unsplit (many tiles) are covered."""
 
 import numpy as np
 import pytest
@@ -35,7 +35,8 @@ def _close_bf16(got, ref):
     (2, 2, 8, 128, 16, 1, 64, 200, 17, False),     # BaseLRShared: one U; Dm not a multiple of 64
     (1, 2, 2, 64, 8, 0, 300, 136, 64, False),
     (3, 3, 2, 128, 16, 0, 150, 512, 100, True),    # paged value cache
-    (1, 4, 8, 128, 32, 0, 2100, 256, 3, False),    # enough tiles that the K loop is not split
+    (1, 4, 8, 128, 32, 0, 2100, 256, 3, False),    # enough tiles that the K loop is not split (256 columns)
+    (1, 4, 8, 128, 32, 0, 1100, 256, 0, False),    # 256-column tiles with the K loop split
     (1, 2, 2, 64, 8, 0, 100, 1024, 0, False),      # one tile: K split over a cluster of 8
     (2, 3, 1, 128, 16, 1, 77, 136, 9, True),       # K split 3 ways, ragged last K step, paged
 ])
