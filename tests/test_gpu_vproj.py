@@ -93,3 +93,33 @@ def test_value_projection_matches_oracle(S, N, Hkv, d, r, mode, T, Dm, start, pa
     else:
         v_mask[pg, :, pos % 64] = False
     assert torch.equal(v[v_mask].view(torch.int16), v_before[v_mask].view(torch.int16))
+
+
+@pytest.mark.parametrize("T,Dm,Hkv,d,n_u,r", [
+    (512, 2048, 8, 128, 4, 32),   # the prefill workload's shape: 128-column tiles, K split over a cluster
+    (1100, 256, 8, 128, 4, 32),   # 256-column tiles, K split
+    (100, 1024, 2, 64, 2, 8),     # one column tile, split 8 ways
+])
+def test_value_projection_is_deterministic(T, Dm, Hkv, d, n_u, r):
+    # the split K loop's partial tiles are summed in cluster-rank order, so repeated
+    # calls give the same bits whatever order the CTAs finish in
+    g = torch.Generator(device=DEV)
+    g.manual_seed(T + Dm)
+    ncols = Hkv * d + n_u * r
+    x = _normal((T, Dm), 1.0, g, DEV)
+    w = _normal((Dm, ncols), Dm ** -0.5, g, DEV)
+    prob = lrkv.make_problem(1, n_u, 2 * Hkv, Hkv, d, r, 0)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    outs = []
+    for _ in range(3):
+        k = torch.zeros((1, Hkv, T, d), dtype=torch.bfloat16, device=DEV)
+        v = torch.zeros_like(k)
+        u = torch.zeros((1, n_u, T, r), dtype=torch.bfloat16, device=DEV)
+        lrkv.lrkv_value_projection(prob, x, w, lrkv.kv_view_dense(k, v), T, u, 0, 0, ws)
+        outs.append((v, u))
+    torch.cuda.synchronize()
+    st, flags = lrkv.lrkv_query_device_status(ws)
+    assert st == "LRKV_OK", (st, hex(flags))
+    for v, u in outs[1:]:
+        assert torch.equal(v.view(torch.int16), outs[0][0].view(torch.int16))
+        assert torch.equal(u.view(torch.int16), outs[0][1].view(torch.int16))
