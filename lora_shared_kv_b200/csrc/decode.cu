@@ -587,7 +587,7 @@ __device__ __forceinline__ void finish_segment(const DecodeParams& p, const SegI
   }
 }
 
-template <int D, int NT, int RK>
+template <int D, int NT, int RK, int NOG>
 __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const DecodeSmem& lay, uint64_t* full,
                                  uint64_t* empty, volatile int* seq, volatile int* abort_flag, int* bcast,
                                  long long t_begin, long long t_end) {
@@ -598,7 +598,6 @@ __device__ void decode_consumers(const DecodeParams& p, uint8_t* smem, const Dec
   constexpr int KV_BYTES = KT * D * 2;
   constexpr int U_BYTES = KT * RK * 2;
   constexpr int REC = RP * (D + RK + 2);
-  constexpr int NOG = decode_groups(NT);
   constexpr int CT = NOG * NT * 32;   // consumer threads
   const int tid = threadIdx.x;        // consumers are warps 0 .. NOG*NT-1
   const int warp = tid >> 5, lane = tid & 31;
@@ -953,16 +952,16 @@ __device__ void decode_epilogue(const DecodeParams& p, uint8_t* smem, const Deco
   }
 }
 
-// Warp roles: warps 0 .. decode_groups(NT)*NT-1 consume, then one producer warp
-// and one epilogue warp.
-template <int NT>
+// Warp roles: warps 0 .. NOG*NT-1 consume (NOG owner groups of NT warps), then
+// one producer warp and one epilogue warp.
+template <int NT, int NOG>
 struct Roles {
-  static constexpr int CONSUMER_WARPS = decode_groups(NT) * NT;
+  static constexpr int CONSUMER_WARPS = NOG * NT;
   static constexpr int THREADS = (CONSUMER_WARPS + 2) * 32;
 };
 
-template <int D, int NT, int RK>
-__global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
+template <int D, int NT, int RK, int NOG>
+__global__ void __launch_bounds__(Roles<NT, NOG>::THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmU, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -976,7 +975,7 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
   volatile int* abort_flag = seq + p.stages;
   int* bcast = const_cast<int*>(abort_flag) + 1;  // [0] consumers, [1] epilogue warp
   const int warp = threadIdx.x >> 5;
-  constexpr int PRODUCER = Roles<NT>::CONSUMER_WARPS;
+  constexpr int PRODUCER = Roles<NT, NOG>::CONSUMER_WARPS;
   constexpr int EPILOGUE = PRODUCER + 1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -1009,18 +1008,18 @@ __global__ void __launch_bounds__(Roles<NT>::THREADS, 1)
   } else if (warp == EPILOGUE) {
     decode_epilogue<D, NT, RK>(p, smem, lay, rec_full, rec_free, abort_flag, bcast + 1, t_begin, t_end);
   } else {
-    decode_consumers<D, NT, RK>(p, smem, lay, full, empty, seq, abort_flag, bcast, t_begin, t_end);
+    decode_consumers<D, NT, RK, NOG>(p, smem, lay, full, empty, seq, abort_flag, bcast, t_begin, t_end);
   }
 }
 
-template <int D, int NT, int RK>
+template <int D, int NT, int RK, int NOG>
 lrkv_status launch_one(const DecodeParams& p, const void* tmK, const void* tmV, const void* tmU, int smem,
                        int ctas, cudaStream_t stream) {
-  auto kern = decode_kernel<D, NT, RK>;
-  if (ensure_dynamic_smem<decode_kernel<D, NT, RK>>(smem) != cudaSuccess) return LRKV_ERR_CUDA;
+  auto kern = decode_kernel<D, NT, RK, NOG>;
+  if (ensure_dynamic_smem<decode_kernel<D, NT, RK, NOG>>(smem) != cudaSuccess) return LRKV_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
-  cfg.blockDim = dim3(Roles<NT>::THREADS);
+  cfg.blockDim = dim3(Roles<NT, NOG>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1036,30 +1035,33 @@ lrkv_status launch_one(const DecodeParams& p, const void* tmK, const void* tmV, 
 }
 
 template <int D, int RK>
-lrkv_status dispatch_nt(const DecodeParams& p, int NT, const void* tmK, const void* tmV, const void* tmU,
+lrkv_status dispatch_nt(const DecodeParams& p, int NT, int groups, const void* tmK, const void* tmV, const void* tmU,
                         int smem, int ctas, cudaStream_t st) {
+  if (groups != decode_groups(NT, false) && groups != decode_groups(NT, true)) return LRKV_ERR_UNSUPPORTED;
   switch (NT) {
-    case 1: return launch_one<D, 1, RK>(p, tmK, tmV, tmU, smem, ctas, st);
-    case 2: return launch_one<D, 2, RK>(p, tmK, tmV, tmU, smem, ctas, st);
-    case 3: return launch_one<D, 3, RK>(p, tmK, tmV, tmU, smem, ctas, st);
-    case 4: return launch_one<D, 4, RK>(p, tmK, tmV, tmU, smem, ctas, st);
+    case 1:
+      return groups == 4 ? launch_one<D, 1, RK, 4>(p, tmK, tmV, tmU, smem, ctas, st)
+                         : launch_one<D, 1, RK, 3>(p, tmK, tmV, tmU, smem, ctas, st);
+    case 2: return launch_one<D, 2, RK, 3>(p, tmK, tmV, tmU, smem, ctas, st);
+    case 3: return launch_one<D, 3, RK, 2>(p, tmK, tmV, tmU, smem, ctas, st);
+    case 4: return launch_one<D, 4, RK, 2>(p, tmK, tmV, tmU, smem, ctas, st);
   }
   return LRKV_ERR_UNSUPPORTED;
 }
 
 }  // namespace
 
-lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, const void* tmK, const void* tmV,
+lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, int groups, const void* tmK, const void* tmV,
                           const void* tmU, int smem_bytes, int ctas, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (D == 128) {
-    if (RK == 8) return dispatch_nt<128, 8>(p, NT, tmK, tmV, tmU, smem_bytes, ctas, st);
-    if (RK == 16) return dispatch_nt<128, 16>(p, NT, tmK, tmV, tmU, smem_bytes, ctas, st);
-    if (RK == 32) return dispatch_nt<128, 32>(p, NT, tmK, tmV, tmU, smem_bytes, ctas, st);
+    if (RK == 8) return dispatch_nt<128, 8>(p, NT, groups, tmK, tmV, tmU, smem_bytes, ctas, st);
+    if (RK == 16) return dispatch_nt<128, 16>(p, NT, groups, tmK, tmV, tmU, smem_bytes, ctas, st);
+    if (RK == 32) return dispatch_nt<128, 32>(p, NT, groups, tmK, tmV, tmU, smem_bytes, ctas, st);
   } else if (D == 64) {
-    if (RK == 8) return dispatch_nt<64, 8>(p, NT, tmK, tmV, tmU, smem_bytes, ctas, st);
-    if (RK == 16) return dispatch_nt<64, 16>(p, NT, tmK, tmV, tmU, smem_bytes, ctas, st);
-    if (RK == 32) return dispatch_nt<64, 32>(p, NT, tmK, tmV, tmU, smem_bytes, ctas, st);
+    if (RK == 8) return dispatch_nt<64, 8>(p, NT, groups, tmK, tmV, tmU, smem_bytes, ctas, st);
+    if (RK == 16) return dispatch_nt<64, 16>(p, NT, groups, tmK, tmV, tmU, smem_bytes, ctas, st);
+    if (RK == 32) return dispatch_nt<64, 32>(p, NT, groups, tmK, tmV, tmU, smem_bytes, ctas, st);
   }
   return LRKV_ERR_UNSUPPORTED;
 }

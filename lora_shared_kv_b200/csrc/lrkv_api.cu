@@ -175,7 +175,7 @@ lrkv_status check_u(const lrkv_u_view* u, const lrkv_problem* p, int rows_needed
 // decode plan
 // ---------------------------------------------------------------------------
 struct DecodePlan {
-  int G, R, n_rg, rows_per_group, NT, n_u_slots, nt, items, ctas, max_segs, stages, smem;
+  int G, R, n_rg, rows_per_group, NT, n_u_slots, nt, items, ctas, max_segs, groups, stages, smem;
   long long W;
   size_t tickets_off, partials_off, bytes;
 };
@@ -223,6 +223,7 @@ lrkv_status plan_decode(const lrkv_problem* p, int hkv, int max_seq_len, const D
     ms = n > ms ? n : ms;
   }
   pl->max_segs = ms;
+  pl->groups = lrkv::decode_groups(pl->NT, ms > 1);
   // shared memory: as many stages as fit (2..8)
   const int optin = dev.smem_optin > 0 ? dev.smem_optin : 232448;
   int stages = 8;
@@ -554,7 +555,7 @@ lrkv_status decode_heads(const lrkv_problem* p, int g_begin, int g_count, const 
   dp.tickets = reinterpret_cast<int*>(ws + pl.tickets_off);
   dp.partials = reinterpret_cast<float*>(ws + pl.partials_off);
   take_stall_hook(&dp.spin_cap, &dp.stall);
-  s = lrkv::launch_decode(dp, D, pl.NT, RK, &tmK, &tmV, &tmU, pl.smem, pl.ctas, stream);
+  s = lrkv::launch_decode(dp, D, pl.NT, RK, pl.groups, &tmK, &tmV, &tmU, pl.smem, pl.ctas, stream);
   if (s != LRKV_OK) return fail(s, "decode launch failed: %s", cudaGetErrorString(cudaGetLastError()));
   return LRKV_OK;
 }

@@ -69,8 +69,15 @@ struct DecodeParams {
 // Consumer warp groups of the decode kernel (NT warps each, eight query rows
 // per warp).  Tile n of a CTA goes to group n % groups and to ring stage
 // n % stages.  More groups keep more tiles in flight per SM; three fit the
-// register file for up to 16 rows per item (NT <= 2), two for 24.
-__host__ __device__ constexpr int decode_groups(int NT) { return NT <= 2 ? 3 : 2; }
+// register file for up to 16 rows per item (NT <= 2), two for 24.  Items of
+// up to 8 rows that are split over CTAs take four (measured on Qwen3 shapes
+// with 128 items: 8192 keys, split over 148 CTAs, 2.428 -> 2.329 ms per 28
+// layers); whole items keep three (1024 / 2048 / 4096 keys, one item per CTA,
+// 1.7 / 3.7 / 4.5% slower with four: a group holds its ring stage while it
+// computes, and those launches need more stages loading per SM).
+__host__ __device__ constexpr int decode_groups(int NT, bool split) {
+  return NT == 1 && split ? 4 : (NT <= 2 ? 3 : 2);
+}
 
 // Shared-memory plan of the decode kernel (bytes from a 1024-aligned base).
 struct DecodeSmem {
@@ -120,7 +127,7 @@ struct VprojParams {
 // ---------------------------------------------------------------------------
 struct TmaMaps;  // opaque; holds CUtensorMap objects
 
-lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, const void* tmK, const void* tmV,
+lrkv_status launch_decode(const DecodeParams& p, int D, int NT, int RK, int groups, const void* tmK, const void* tmV,
                           const void* tmU, int smem_bytes, int ctas, void* stream);
 int decode_max_smem_optin();
 int vproj_smem_bytes();

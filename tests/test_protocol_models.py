@@ -178,7 +178,7 @@ def prefill_handshake(nb, two_barriers, seed):
 
 def test_decode_ring_with_sequence_words_never_reads_a_stale_stage():
     for stages in range(2, 9):
-        for groups in (2, 3):
+        for groups in (2, 3, 4):  # 2 for 24-row items, 3 for up to 16, 4 for split 8-row items
             for warps in (1, 3):
                 for seed in range(12):
                     errs = decode_ring(stages, groups, warps, 40, seed, guard=True)
