@@ -53,6 +53,13 @@ namespace lrkv {
 
 namespace {
 
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 constexpr int BM = 128;   // rows per tile (TMEM lanes)
 constexpr int BN = 128;   // keys per block
 constexpr int KST = 3;    // K ring: a stage is free once S = Q K^T has been computed
@@ -507,14 +514,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int cc = 0; cc < HB; ++cc) x[cc] = key0 + cc <= limit ? x[cc] : NEG_INF;
         }
         // row max over the half: eight independent chains, then a tree; then the other half's
+        static_assert(HB % 16 == 8 || HB % 16 == 0, "row-max chains");
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = x[e];
 #pragma unroll
-        for (int cc = 8; cc < HB; ++cc) mx8[cc & 7] = fmaxf(mx8[cc & 7], x[cc]);
+        for (int cc = 8; cc + 16 <= HB; cc += 16) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = fmax3(mx8[e], x[cc + e], x[cc + 8 + e]);
+        }
+        if constexpr (HB % 16 == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[HB - 8 + e]);
+        }
         float* xm = xmax + (n & 1) * 2 * BM;
-        xm[wg * BM + row] = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                  fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        xm[wg * BM + row] = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         named_bar_sync(2 + (warp & 3), 64);  // the two warps of these 32 rows; both have read their S columns
         float mx = fmaxf(xm[row], xm[BM + row]);
         mx *= p.scale_log2;  // the scale is positive: the max commutes with it
@@ -558,11 +572,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float mu = m_ref == NEG_INF ? 0.f : m_ref;
         // (the row sum l of exactly these bf16 weights is accumulated by the MMA)
         uint32_t pk[HB / 2];
+        unsigned long long ss, mm;  // (scale, scale) and (-mu, -mu)
+        asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(p.scale_log2));
+        asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(-mu));
 #pragma unroll
         for (int cc = 0; cc < HB / 2; ++cc) {
-          const float p0 = fast_exp2(fmaf(x[2 * cc], p.scale_log2, -mu));
-          const float p1 = fast_exp2(fmaf(x[2 * cc + 1], p.scale_log2, -mu));
-          pk[cc] = pack_bf16x2(p0, p1);
+          unsigned long long xx, aa;
+          asm("mov.b64 %0, {%1, %2};" : "=l"(xx) : "f"(x[2 * cc]), "f"(x[2 * cc + 1]));
+          asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(aa) : "l"(xx), "l"(ss), "l"(mm));
+          float a0, a1;
+          asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(aa));
+          pk[cc] = pack_bf16x2(fast_exp2(a0), fast_exp2(a1));
         }
         // P of keys [c0, c0 + 64) as bf16 pairs: TMEM columns s_col + c0 / 2 + [0, 32)
         tmem_st32(tmem + lane_addr + s_col + c0 / 2, pk);
