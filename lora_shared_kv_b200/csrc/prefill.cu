@@ -513,7 +513,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int cc = 0; cc < HB; ++cc) x[cc] = key0 + cc <= limit ? x[cc] : NEG_INF;
         }
-        // row max over the half: eight independent chains, then a tree; then the other half's
+        // row max over the half: eight independent chains of three-input maxima, then a
+        // tree; then the other half's.  The softmax warps' instruction streams pace this
+        // phase, so every instruction saved here shortens the block.
         static_assert(HB % 16 == 8 || HB % 16 == 0, "row-max chains");
         float mx8[8];
 #pragma unroll
@@ -571,6 +573,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         const float mu = m_ref == NEG_INF ? 0.f : m_ref;
         // (the row sum l of exactly these bf16 weights is accumulated by the MMA)
+        // Two weights' exponent arguments per packed fma (each lane a correctly rounded
+        // fma, the same value fmaf gives).
         uint32_t pk[HB / 2];
         unsigned long long ss, mm;  // (scale, scale) and (-mu, -mu)
         asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(p.scale_log2));
